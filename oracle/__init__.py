@@ -1,0 +1,158 @@
+"""CPU oracle for the 3D (shifted-)window attention layer.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``; never
+by the product package. It shares no code with the CUDA library.
+
+Two independent formulations live here:
+
+* ``forward`` -- ``vswin_oracle.cpp``, double precision, the pages' steps in
+  order (pad, roll by -shift, window partition, QKV, masked
+  softmax(QK^T/sqrt(d) + B)V, projection, reverse partition, roll by +shift,
+  un-pad). "Video Swin Transformer" summary page, Method steps 3-6 and the
+  window_msa pseudocode; eq. 2.
+* ``group_rule.forward`` -- a NumPy float64 brute force over all token pairs of
+  the padded grid with no roll and no partition (see that module).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "vswin_oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+NO_MASK = 1
+POS_ROLL = 2
+NO_BIAS = 4
+ROLL_THEN_PAD = 8
+MASK_ADD100 = 16
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``vswin_oracle.cpp`` into ``liboracle.so`` (g++, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["g++", "-O2", "-std=c++17", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.vswin_oracle_forward_ex.argtypes = [
+            dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ip, ip, dp, dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_long, ctypes.c_int, dp,
+        ]
+        lib.vswin_oracle_forward_ex.restype = ctypes.c_int
+        lib.vswin_oracle_index_maps.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ip, ip, ip, ip,
+        ]
+        lib.vswin_oracle_index_maps.restype = ctypes.c_int
+        lib.vswin_oracle_max_threads.argtypes = [ctypes.c_int]
+        lib.vswin_oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _dptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _iarr(v) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(v, dtype=np.int32).reshape(3))
+
+
+def _iptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def max_threads(nthreads: int = 0) -> int:
+    """OpenMP threads the oracle uses with ``nthreads`` (0 = library default)."""
+    return int(_load().vswin_oracle_max_threads(int(nthreads)))
+
+
+def geometry(T, H, W, window, shift=(0, 0, 0)):
+    """Padded extents, windows per axis, windows per clip and tokens per window."""
+    L = (T, H, W)
+    Lp = tuple(-(-L[a] // window[a]) * window[a] for a in range(3))
+    nw = tuple(Lp[a] // window[a] for a in range(3))
+    return {
+        "Lp": Lp,
+        "nw": nw,
+        "nW": nw[0] * nw[1] * nw[2],
+        "N": window[0] * window[1] * window[2],
+    }
+
+
+def forward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, flags=0, nthreads=0,
+            probe=None):
+    """Layer forward in double precision.
+
+    x: (B,T,H,W,C); Wqkv [C][3C]; bqkv [3C]; Wproj [C][C]; bproj [C];
+    table [(2P-1)(2Mh-1)(2Mw-1)][heads]. window/shift are taken literally.
+    probe=(b, window_index, head) additionally returns that head's N x N
+    attention probabilities.
+    """
+    lib = _load()
+    x = _f64(x)
+    B, T, H, W, C = x.shape
+    g = geometry(T, H, W, window, shift)
+    N = g["N"]
+    out = np.empty_like(x)
+    w_arr, s_arr = _iarr(window), _iarr(shift)
+    Wqkv, bqkv, Wproj, bproj, table = map(_f64, (Wqkv, bqkv, Wproj, bproj, table))
+    assert Wqkv.shape == (C, 3 * C) and bqkv.shape == (3 * C,)
+    assert Wproj.shape == (C, C) and bproj.shape == (C,)
+    nt = (2 * window[0] - 1) * (2 * window[1] - 1) * (2 * window[2] - 1)
+    assert table.shape == (nt, heads)
+    probs = None
+    pb, pw, ph = -1, -1, -1
+    if probe is not None:
+        pb, pw, ph = probe
+        probs = np.zeros((N, N), dtype=np.float64)
+    rc = lib.vswin_oracle_forward_ex(
+        _dptr(x), B, T, H, W, C, heads, _iptr(w_arr), _iptr(s_arr),
+        _dptr(Wqkv), _dptr(bqkv), _dptr(Wproj), _dptr(bproj), _dptr(table), _dptr(out),
+        int(flags), int(nthreads), pb, pw, ph, _dptr(probs) if probs is not None else None,
+    )
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (status {rc})")
+    if probe is not None:
+        return out, probs
+    return out
+
+
+def index_maps(B, T, H, W, window, shift):
+    """(win_src[B*nW*N], region[nW*N], bias_idx[N*N]) as int32 arrays."""
+    lib = _load()
+    g = geometry(T, H, W, window, shift)
+    N, nW = g["N"], g["nW"]
+    win_src = np.empty(B * nW * N, dtype=np.int32)
+    region = np.empty(nW * N, dtype=np.int32)
+    bias_idx = np.empty(N * N, dtype=np.int32)
+    w_arr, s_arr = _iarr(window), _iarr(shift)
+    rc = lib.vswin_oracle_index_maps(B, T, H, W, _iptr(w_arr), _iptr(s_arr),
+                                     _iptr(win_src), _iptr(region), _iptr(bias_idx))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (status {rc})")
+    return win_src, region, bias_idx

@@ -1,0 +1,84 @@
+"""Seeded synthetic inputs shared by the CUDA path, the oracle and the benchmark.
+
+This module holds random-number generation and dtype rounding only -- none of
+the layer's arithmetic. Both sides receive the very same rounded values: the
+CUDA library as torch tensors of the run dtype, the oracle as float64 copies.
+
+Recipe (stands in for Kinetics clips; no dataset is used):
+  * CPU ``torch.Generator`` seeded with ``1000 * workload_index + k + seed_offset``,
+    k = 0: x, 1: Wqkv, 2: Wproj, 3: table, 4: bqkv, 5: bproj;
+  * "baseline" scale: x ~ N(0, 1); Wqkv, Wproj, table ~ N(0, 0.02); biases 0;
+  * "sensitivity" scale (correctness only): x ~ N(0, 1); Wqkv, Wproj ~ N(0, 1/C);
+    table ~ N(0, 1); biases ~ N(0, 0.1), so that dropping the mask, the bias or
+    a bias vector moves the output far outside the tolerances;
+  * values drawn in float32, then rounded once to the run dtype.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@dataclass
+class LayerInputs:
+    x: torch.Tensor
+    Wqkv: torch.Tensor
+    bqkv: torch.Tensor
+    Wproj: torch.Tensor
+    bproj: torch.Tensor
+    table: torch.Tensor
+
+    def as_f64(self):
+        """float64 NumPy copies of the exact (rounded) values, for the oracle."""
+        return {k: getattr(self, k).to(torch.float64).numpy() for k in
+                ("x", "Wqkv", "bqkv", "Wproj", "bproj", "table")}
+
+    def to(self, device):
+        return LayerInputs(*(getattr(self, k).to(device) for k in
+                             ("x", "Wqkv", "bqkv", "Wproj", "bproj", "table")))
+
+
+def table_rows(window) -> int:
+    return (2 * window[0] - 1) * (2 * window[1] - 1) * (2 * window[2] - 1)
+
+
+def _randn(shape, seed, std):
+    g = torch.Generator().manual_seed(int(seed))
+    return torch.randn(*shape, generator=g, dtype=torch.float32) * std
+
+
+def make_layer_inputs(shape, heads, window, dtype="bf16", scale="baseline", seed=1000,
+                      x_seed=None) -> LayerInputs:
+    """Inputs for one layer call. ``shape`` = (B, T, H, W, C)."""
+    B, T, H, W, C = shape
+    dt = _DT[dtype]
+    nt = table_rows(window)
+    xs = seed if x_seed is None else x_seed
+    if scale == "baseline":
+        w_std, t_std, b_std = 0.02, 0.02, 0.0
+    elif scale == "sensitivity":
+        w_std, t_std, b_std = 1.0 / np.sqrt(C), 1.0, 0.1
+    else:
+        raise ValueError(scale)
+    x = _randn((B, T, H, W, C), xs + 0, 1.0)
+    Wqkv = _randn((C, 3 * C), seed + 1, w_std)
+    Wproj = _randn((C, C), seed + 2, w_std)
+    table = _randn((nt, heads), seed + 3, t_std)
+    bqkv = _randn((3 * C,), seed + 4, b_std) if b_std else torch.zeros(3 * C)
+    bproj = _randn((C,), seed + 5, b_std) if b_std else torch.zeros(C)
+    return LayerInputs(*(t.to(dt).contiguous() for t in (x, Wqkv, bqkv, Wproj, bproj, table)))
+
+
+def workload_layer_inputs(workload, layer, scale="baseline") -> LayerInputs:
+    """Inputs of one layer of a named workload (see ``workloads.py``).
+
+    The two layers of the W-MSA + SW-MSA pair get their own weights but the
+    same N(0,1) input (x is seeded without the layer's offset)."""
+    base = 1000 * workload.index
+    return make_layer_inputs(layer.shape, layer.heads, layer.window, workload.dtype, scale,
+                             seed=base + layer.seed_offset, x_seed=base)
