@@ -1,0 +1,158 @@
+/*
+ * vswin -- 3D (shifted-)window multi-head self-attention (Video Swin W-MSA /
+ * SW-MSA) for NVIDIA B200 (sm_100a). C ABI.
+ *
+ * The layer ("Video Swin Transformer" summary page, Method steps 4-6, the
+ * window_msa pseudocode and eq. 2; the Video Swin code walk-through page,
+ * section 1.2, for the op order of WindowAttention3D):
+ *
+ *   1. zero-pad the token grid (T, H, W) at the high end of each axis to
+ *      multiples of the window (P, Mh, Mw);
+ *   2. roll the padded grid by -shift on each axis (content moves toward
+ *      index 0), so that rolled coordinate r holds original o = (r+s) mod Lp;
+ *   3. partition into windows of N = P*Mh*Mw slots, windows (b, wt, wh, ww)
+ *      and slots (pt, ph, pw) both row-major;
+ *   4. qkv = X Wqkv + bqkv; head h uses columns [h*d, (h+1)*d) of the q, k and
+ *      v blocks (d = C / heads);
+ *   5. per window and head: softmax(q k^T / sqrt(d) + B) v over the keys that
+ *      share the query's region (only when some shift is nonzero); B[i][j] =
+ *      bias_table[(dt+P-1)(2Mh-1)(2Mw-1) + (dh+Mh-1)(2Mw-1) + (dw+Mw-1)][h]
+ *      with (dt,dh,dw) = slot position of i minus that of j;
+ *   6. y = concat_h(o_h) Wproj + bproj;
+ *   7. reverse the partition, roll by +shift, drop the padding.
+ *
+ * Regions: on a shifted axis, rolled coordinate r is in region 0 when
+ * r < Lp - w, 1 when r < Lp - s, else 2 (the slices of the last window that
+ * were not neighbours before the roll; summary page, Method step 5). Masked
+ * pairs are excluded from the softmax. Padded slots are ordinary keys with
+ * zero input (k = bk, v = bv).
+ *
+ * Layouts (all row-major, contiguous, no strides):
+ *   x, out       (B, T, H, W, C)           channels last
+ *   Wqkv         [C][3C]                   used as x * Wqkv
+ *   bqkv         [3C]
+ *   Wproj        [C][C]                    used as o * Wproj
+ *   bproj        [C]
+ *   bias_table   [(2P-1)(2Mh-1)(2Mw-1)][heads]
+ *
+ * Conventions for every entry point:
+ *   * tensor pointers are DEVICE pointers unless the name ends in _host;
+ *     the caller owns every buffer; nothing is retained after the call;
+ *   * `stream` is a cudaStream_t (NULL = legacy default stream); work is
+ *     enqueued on it and the call returns without synchronising (except
+ *     vswin_wmsa_forward_host, which synchronises);
+ *   * window and shift are host arrays of 3 ints, taken literally (no
+ *     clamping; see vswin_clamp_window);
+ *   * the return value is a vswin_status; on failure nothing has been
+ *     launched and vswin_last_error() describes the cause. Errors raised by
+ *     kernels (a bounded wait that gave up) are reported by vswin_poll_error.
+ *   * nothing throws across the ABI; the library is thread-safe (the last
+ *     error message is thread-local).
+ */
+#ifndef VSWIN_H_
+#define VSWIN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VSWIN_OK = 0,
+  VSWIN_ERR_INVALID_ARG = 1,  /* bad sizes, window/shift, NULL or misaligned or overlapping pointers */
+  VSWIN_ERR_UNSUPPORTED = 2,  /* valid layer that this path does not implement (see each entry) */
+  VSWIN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  VSWIN_ERR_TIMEOUT = 4,      /* a kernel's bounded wait gave up (reported by vswin_poll_error) */
+  VSWIN_ERR_NO_MEMORY = 5     /* scratch allocation failed */
+} vswin_status;
+
+/*
+ * bf16 layer forward: x, weights, biases, table and out are bf16; products
+ * accumulate in fp32 on the tensor cores (tcgen05). Requires d = C/heads = 32,
+ * C a multiple of 32, N = P*Mh*Mw <= 400, window (P, Mh, Mw) one of the
+ * compiled shapes (8,7,7), (4,7,7), (2,7,7), (1,7,7), (4,4,4), (2,2,2),
+ * (1,1,1); otherwise VSWIN_ERR_UNSUPPORTED. Pointers must be 16-byte aligned
+ * and x must not overlap out.
+ * Scratch: stream-ordered cudaMallocAsync / cudaFreeAsync on `stream`
+ * (about 135 KB per window of 392 slots at C = 96, processed in chunks of at
+ * most 64 MB).
+ */
+int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int heads,
+                       const int* window, const int* shift,
+                       const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                       const void* bias_table, void* out, void* stream);
+
+/*
+ * fp32 layer forward (plain FP32 FMA arithmetic, no tensor cores): every
+ * tensor is float. Any d; N <= 4096. Pointers 4-byte aligned; x must not
+ * overlap out. Scratch: cudaMallocAsync on `stream`.
+ */
+int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads,
+                           const int* window, const int* shift,
+                           const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                           const void* bias_table, void* out, void* stream);
+
+/*
+ * bf16 layer forward with the activations in HOST memory: copies x_host to
+ * the device, runs vswin_wmsa_forward, copies the result to out_host and
+ * synchronises `stream`. Weights, biases and table are device pointers (they
+ * stay resident between calls). Page-locked host buffers give asynchronous
+ * copies; pageable ones work but are slower. Device buffers for x and out
+ * come from cudaMallocAsync on `stream`.
+ */
+int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads,
+                            const int* window, const int* shift,
+                            const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                            const void* bias_table, void* out_host, void* stream);
+
+/*
+ * Index maps of the layer, written to caller-allocated device int32 buffers
+ * (any of them may be NULL to skip it):
+ *   win_src [B*nW*N]  flat source token b*T*H*W + (t*H + h)*W + w of each
+ *                     window slot, or -1 for a padding slot;
+ *   region  [nW*N]    9*rt + 3*rh + rw of each slot (0 when unshifted);
+ *   bias_idx[N*N]     table row used by query slot i and key slot j.
+ * nW = prod(ceil(L/w)), N = P*Mh*Mw.
+ */
+int vswin_wmsa_index_maps(int B, int T, int H, int W, const int* window, const int* shift,
+                          int* win_src, int* region, int* bias_idx, void* stream);
+
+/*
+ * Host helper: the official code's clamp ("Video Swin Transformer" summary
+ * page, "Paper vs code": a window dimension is set to the input size, with
+ * shift 0, when the input is not larger than the window). Writes the clamped
+ * window and shift (3 ints each).
+ */
+int vswin_clamp_window(int T, int H, int W, const int* window_in, const int* shift_in,
+                       int* window_out, int* shift_out);
+
+/* Thread-local description of the last non-OK status returned on this thread. */
+const char* vswin_last_error(void);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word:
+ * VSWIN_OK, or VSWIN_ERR_TIMEOUT if a kernel's bounded wait gave up since the
+ * last poll, or VSWIN_ERR_CUDA if synchronisation failed.
+ */
+int vswin_poll_error(void* stream);
+
+/* Number of kernels this library has launched in this process (all devices). */
+unsigned long long vswin_launch_count(void);
+
+/* Limit, in nanoseconds, of every bounded wait in the kernels (default 1e9). */
+void vswin_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Self-test of the timeout path: launches one kernel that waits, with the
+ * current limit, on a barrier that nothing completes. It must give up and set
+ * the error word, so a following vswin_poll_error returns VSWIN_ERR_TIMEOUT.
+ */
+int vswin_selftest_timeout(void* stream);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int vswin_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSWIN_H_ */

@@ -60,6 +60,11 @@ def _load():
             ctypes.c_int, ctypes.c_long, ctypes.c_int, dp,
         ]
         lib.vswin_oracle_forward_ex.restype = ctypes.c_int
+        lib.vswin_oracle_forward_windows.argtypes = [
+            dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ip, ip, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_long), ctypes.c_int, dp, ctypes.c_int,
+        ]
+        lib.vswin_oracle_forward_windows.restype = ctypes.c_int
         lib.vswin_oracle_index_maps.argtypes = [
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ip, ip, ip, ip,
         ]
@@ -140,6 +145,26 @@ def forward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, flags=0, n
     if probe is not None:
         return out, probs
     return out
+
+
+def forward_windows(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, windows, nthreads=0):
+    """Per-window outputs (len(windows), N, C) in slot order for the listed global
+    windows b * nW + w (no reverse partition): the same arithmetic as ``forward``."""
+    lib = _load()
+    x = _f64(x)
+    B, T, H, W, C = x.shape
+    N = geometry(T, H, W, window, shift)["N"]
+    wl = np.ascontiguousarray(np.asarray(windows, dtype=np.int64))
+    y = np.empty((wl.size, N, C), dtype=np.float64)
+    w_arr, s_arr = _iarr(window), _iarr(shift)
+    Wqkv, bqkv, Wproj, bproj, table = map(_f64, (Wqkv, bqkv, Wproj, bproj, table))
+    rc = lib.vswin_oracle_forward_windows(
+        _dptr(x), B, T, H, W, C, heads, _iptr(w_arr), _iptr(s_arr), _dptr(Wqkv), _dptr(bqkv),
+        _dptr(Wproj), _dptr(bproj), _dptr(table), wl.ctypes.data_as(ctypes.POINTER(ctypes.c_long)),
+        int(wl.size), _dptr(y), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (status {rc})")
+    return y
 
 
 def index_maps(B, T, H, W, window, shift):

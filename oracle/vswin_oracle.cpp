@@ -346,6 +346,46 @@ int vswin_oracle_forward(const double* x, int B, int T, int H, int W, int C, int
                                  bproj, table, out, flags, nthreads, -1, -1, -1, nullptr);
 }
 
+// Outputs of selected windows only, for spot checks of large layers. For each
+// global window index win_list[k] = b * nW + w, writes that window's N x C
+// projection output y (slot order, before the reverse partition) to
+// y_out + k * N * C. Same arithmetic and readings as vswin_oracle_forward.
+int vswin_oracle_forward_windows(const double* x, int B, int T, int H, int W, int C, int heads,
+                                 const int* window, const int* shift, const double* Wqkv,
+                                 const double* bqkv, const double* Wproj, const double* bproj,
+                                 const double* table, const long* win_list, int nlist,
+                                 double* y_out, int nthreads) {
+  Geom g;
+  if (!make_geom(B, T, H, W, C, heads, window, shift, &g)) return 1;
+  for (int k = 0; k < nlist; ++k)
+    if (win_list[k] < 0 || win_list[k] >= (long)B * g.nW) return 1;
+  set_threads(nthreads);
+  const int L[3] = {T, H, W};
+  Grid xin(B, L, C);
+  std::memcpy(xin.v.data(), x, sizeof(double) * xin.v.size());
+  const int sneg[3] = {-g.s[0], -g.s[1], -g.s[2]};
+  Grid xr = roll_grid(pad_grid(xin, g.Lp), sneg);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int k = 0; k < nlist; ++k) {
+    const int b = (int)(win_list[k] / g.nW);
+    const long win = win_list[k] % g.nW;
+    int wp[3];
+    window_pos(g, win, wp);
+    std::vector<double> X((size_t)g.N * C);
+    for (int n = 0; n < g.N; ++n) {
+      int p[3];
+      slot_pos(g, n, p);
+      std::memcpy(&X[(size_t)n * C],
+                  xr.at(b, wp[0] * g.w[0] + p[0], wp[1] * g.w[1] + p[1], wp[2] * g.w[2] + p[2]),
+                  sizeof(double) * C);
+    }
+    std::vector<double> y;
+    window_layer(g, X, win, Wqkv, bqkv, Wproj, bproj, table, 0, y, -1, nullptr);
+    std::memcpy(y_out + (size_t)k * g.N * C, y.data(), sizeof(double) * y.size());
+  }
+  return 0;
+}
+
 // Index maps, built by rolling and partitioning an index tensor exactly as the
 // layer moves data:
 //   win_src[B*nW*N]: flat source token b*T*H*W + (t*H + h)*W + w, or -1 for a

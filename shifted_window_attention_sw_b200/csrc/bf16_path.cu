@@ -1,0 +1,646 @@
+// bf16 path of the layer on sm_100a tensor cores (tcgen05 / TMEM).
+//
+// Per chunk of windows, three launches:
+//   1. gemm_kernel<kQKV>:  gather window slots from x (roll + pad + partition
+//      folded into the row index, padding zero-filled by the copy), tcgen05 GEMM
+//      with Wqkv, epilogue adds bqkv, scales q by log2(e)/sqrt(d) and writes
+//      per-(window, head) q / k / v slabs in the tensor-core operand layout;
+//   2. attention_kernel:   per (window, head): S = q k^T on tcgen05 into TMEM,
+//      relative-position bias + shifted-window mask + softmax in registers
+//      (exp2 domain), P as bf16 back into TMEM, O = P v on tcgen05 with P
+//      read from TMEM; keys in up to three blocks, each with its own running
+//      max, merged in the epilogue;
+//   3. gemm_kernel<kPROJ>: tcgen05 GEMM of the attention output with Wproj,
+//      epilogue adds bproj and scatters rows back through the inverse window
+//      map (un-partition, roll by +shift, drop padding).
+//
+// Shared-memory operand layout everywhere: the no-swizzle canonical layout of
+// 8-row x 16-byte core matrices (128 contiguous bytes).
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace vswin {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ============================================================================ GEMM
+constexpr int kBM = 128;
+constexpr int kBK = 32;
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 128;
+constexpr int kMaxBN = 256;
+constexpr int kAStageBytes = kBM * kBK * 2;      // 8 KB
+constexpr int kBStageMaxBytes = kBK * kMaxBN * 2;  // 16 KB
+
+enum { kQKV = 0, kPROJ = 1 };
+
+struct GemmArgs {
+  Geom g;
+  KernelCtx ctx;
+  const __nv_bfloat16* A;     // kQKV: x (gathered rows); kPROJ: attention output [rows][C]
+  const __nv_bfloat16* Wt;    // [K][Ntot] row-major (used as the MN-major B operand)
+  const __nv_bfloat16* bias;  // [Ntot]
+  __nv_bfloat16* dst;         // kQKV: q/k/v slabs; kPROJ: out (B,T,H,W,C)
+  long long win0;             // first window of the chunk
+  long long rows;             // nwin * N
+  int K, Ntot, BN;
+  float qscale;
+};
+
+__host__ __device__ constexpr int gemm_smem_bytes() {
+  return kStages * (kAStageBytes + kBStageMaxBytes) + kBM * 8 + 256;
+}
+
+// Hardware base-2 exponential (MUFU), flush-to-zero; ex2(-inf) = +0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kAStageBytes;
+  long long* s_src = reinterpret_cast<long long*>(sB + kStages * kBStageMaxBytes);
+  uint64_t* bar_free = reinterpret_cast<uint64_t*>(s_src + kBM);  // kStages
+  uint64_t* bar_done = bar_free + kStages;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_done + 1);
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Geom& g = a.g;
+  const long long m0 = (long long)blockIdx.x * kBM;  // first row of the tile (chunk-relative)
+  const int n0 = blockIdx.y * a.BN;
+  const int BN = a.BN;
+  const uint32_t tcols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+
+  // Row sources: element offset of the row's first channel, or -1 (zero fill).
+  {
+    const long long r = m0 + tid;
+    long long src = -1;
+    if (r < a.rows) {
+      if (MODE == kQKV) {
+        const long long gr = a.win0 * g.N + r;
+        const long long tok = slot_source(g, gr / g.N, (int)(gr % g.N));
+        src = tok < 0 ? -1 : tok * g.C;
+      } else {
+        src = r * (long long)g.C;
+      }
+    }
+    s_src[tid] = src;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bar_free[s], 1);
+    mbar_init(bar_done, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  const int KB = a.K / kBK;
+  const uint32_t lboB = (uint32_t)(BN / 8) * 128u;
+  const int bchunks = kBK * (BN / 8);
+
+  auto load_stage = [&](int kb, int s) {
+    const int k0 = kb * kBK;
+    uint8_t* dA = sA + s * kAStageBytes;
+    // A: 128 rows x 4 chunks of 8 channels; thread = row.
+    const long long src = s_src[tid];
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc) {
+      uint8_t* d = dA + (tid >> 3) * 512 + kc * 128 + (tid & 7) * 16;
+      const __nv_bfloat16* p = a.A + (src < 0 ? 0 : src + k0 + kc * 8);
+      cp_async_16(d, p, src < 0 ? 0u : 16u);
+    }
+    uint8_t* dB = sB + s * kBStageMaxBytes;
+    for (int c = tid; c < bchunks; c += kGemmThreads) {
+      const int kk = c / (BN / 8), nc = c % (BN / 8);
+      uint8_t* d = dB + (kk >> 3) * lboB + nc * 128 + (kk & 7) * 16;
+      cp_async_16(d, a.Wt + (size_t)(k0 + kk) * a.Ntot + n0 + nc * 8, 16u);
+    }
+  };
+
+  const uint32_t idesc = idesc_bf16(kBM, BN, 0, 1);
+#pragma unroll 1
+  for (int p = 0; p < kStages - 1; ++p) {
+    if (p < KB) load_stage(p, p);
+    cp_async_commit();
+  }
+#pragma unroll 1
+  for (int kb = 0; kb < KB; ++kb) {
+    const int s = kb % kStages;
+    cp_async_wait<kStages - 2>();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0 && !s_abort) {
+      tc_fence_after();
+      const uint32_t aaddr = smem_u32(sA + s * kAStageBytes);
+      const uint32_t baddr = smem_u32(sB + s * kBStageMaxBytes);
+#pragma unroll
+      for (int ks = 0; ks < kBK / 16; ++ks) {
+        const uint64_t ad = smem_desc(aaddr + ks * 256, 128, 512);
+        const uint64_t bd = smem_desc(baddr + ks * 2 * lboB, lboB, 128);
+        umma_ss(tmem, ad, bd, idesc, (kb | ks) != 0);
+      }
+      umma_commit(&bar_free[s]);
+    }
+    const int nk = kb + kStages - 1;
+    if (nk < KB) {
+      const int ns = nk % kStages;
+      if (kb >= 1) {
+        // stage ns was last read by the MMAs of k-block kb-1 (its use number (kb-1)/kStages)
+        if (!mbar_wait(&bar_free[ns], ((kb - 1) / kStages) & 1, a.ctx.err, kErrWaitMma, a.ctx.wait_limit))
+          s_abort = 1;
+      }
+      load_stage(nk, ns);
+    }
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  if (tid == 0) {
+    if (!s_abort) umma_commit(bar_done);
+  }
+  __syncthreads();
+  if (!s_abort && !mbar_wait(bar_done, 0, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
+  __syncthreads();
+  tc_fence_after();
+
+  // ---------------- epilogue: TMEM -> registers -> bf16 -> global
+  // TMEM loads are warp-collective: every lane of a warp whose tile rows start
+  // inside the problem executes them; only the stores depend on the lane's row.
+  const long long r = m0 + warp * 32 + lane;
+  const bool row_ok = r < a.rows;
+  if (!s_abort && m0 + warp * 32 < a.rows) {
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    long long dst_row = -1;     // kPROJ: token
+    long long slab_win = 0;     // kQKV: chunk-relative window
+    int slot = 0;
+    if (MODE == kQKV) {
+      slab_win = r / g.N;
+      slot = (int)(r % g.N);
+    } else if (row_ok) {
+      const long long gr = a.win0 * g.N + r;
+      dst_row = slot_source(g, gr / g.N, (int)(gr % g.N));
+    }
+    for (int c = 0; c < BN / 16; ++c) {
+      uint32_t u[16];
+      tmem_ld16(trow + c * 16, u);
+      tmem_wait_ld();
+      const int col = n0 + c * 16;
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(u[k]) + __bfloat162float(a.bias[col + k]);
+      uint4 w0, w1;
+      if (MODE == kQKV && row_ok) {
+        const int which = col / g.C;
+        const int hh = (col % g.C) >> 5;
+        const int jj = col & 31;  // 0 or 16
+        const float sc = which == 0 ? a.qscale : 1.0f;
+        w0 = make_uint4(pack_bf16x2(v[0] * sc, v[1] * sc), pack_bf16x2(v[2] * sc, v[3] * sc),
+                        pack_bf16x2(v[4] * sc, v[5] * sc), pack_bf16x2(v[6] * sc, v[7] * sc));
+        w1 = make_uint4(pack_bf16x2(v[8] * sc, v[9] * sc), pack_bf16x2(v[10] * sc, v[11] * sc),
+                        pack_bf16x2(v[12] * sc, v[13] * sc), pack_bf16x2(v[14] * sc, v[15] * sc));
+        __nv_bfloat16* slab =
+            a.dst + (((size_t)slab_win * g.heads + hh) * 3 + which) * (size_t)g.Npad * 32;
+        __nv_bfloat16* e = slab + (slot >> 3) * 256 + (jj >> 3) * 64 + (slot & 7) * 8;
+        *reinterpret_cast<uint4*>(e) = w0;
+        *reinterpret_cast<uint4*>(e + 64) = w1;
+      } else if (dst_row >= 0) {
+        w0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                        pack_bf16x2(v[6], v[7]));
+        w1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                        pack_bf16x2(v[14], v[15]));
+        __nv_bfloat16* e = a.dst + dst_row * g.C + col;
+        *reinterpret_cast<uint4*>(e) = w0;
+        *reinterpret_cast<uint4*>(e + 8) = w1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, tcols);
+}
+
+// ============================================================================ attention
+constexpr int kAttnThreads = 128;
+constexpr int kD = 32;                 // head width of this path
+constexpr int kSlabRowBytes = kD * 2;  // 64
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kOCol = 160;        // O accumulators at columns 160, 192, 224
+
+template <int P_, int MH_, int MW_>
+struct Win {
+  static constexpr int P = P_, MH = MH_, MW = MW_;
+  static constexpr int N = P * MH * MW;
+  static constexpr int NPAD = (N + 15) / 16 * 16;
+  static constexpr int NB0 = NPAD < 144 ? NPAD : 144;
+  static constexpr int NB1 = (NPAD - NB0) < 128 ? (NPAD - NB0) : 128;
+  static constexpr int NB2 = NPAD - NB0 - NB1;
+  static constexpr int NBLK = NB2 > 0 ? 3 : (NB1 > 0 ? 2 : 1);
+  static constexpr int WS = 2 * MW - 1;   // table stride of dh
+  static constexpr int TS = (2 * MH - 1) * WS;  // table stride of dt
+  static constexpr int TABLE = (2 * P - 1) * TS;
+  static constexpr int QTILES = (N + 127) / 128;
+  static constexpr int QROWS = QTILES * 128 > NPAD ? QTILES * 128 : NPAD;
+  // shared memory map (bytes)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QROWS * kSlabRowBytes;
+  static constexpr int OFF_V = OFF_K + NPAD * kSlabRowBytes;
+  static constexpr int OFF_T = OFF_V + NPAD * kSlabRowBytes;
+  static constexpr int OFF_BAR = OFF_T + (TABLE * 4 + 15) / 16 * 16;
+  static constexpr int SMEM = OFF_BAR + 64;
+  static_assert(NB2 <= 128, "window too large for this path");
+  static_assert(NPAD <= 400, "window too large for this path");
+};
+
+struct AttnArgs {
+  Geom g;
+  KernelCtx ctx;
+  const __nv_bfloat16* qkv;    // slabs [nwin][heads][3][NPAD*32]
+  const __nv_bfloat16* table;  // [rows][heads]
+  __nv_bfloat16* o;            // [nwin][N][C]
+  long long win0, nwin;
+};
+
+// Per-thread row context for one query tile.
+template <class Wn>
+struct RowCtx {
+  const float* tb;  // table row base: tb_smem + c(i); key j reads tb[-e(j)]
+  bool okt[Wn::P], okh[Wn::MH], okw[Wn::MW];
+};
+
+// Softmax of one key block for the thread's query row: S (TMEM, log2 units,
+// already scaled) + bias (log2 units) [+ mask] -> P (bf16, TMEM), row max m
+// and row sum l of the block.
+template <class Wn, int KB0, int NB, bool MASKED>
+__device__ __forceinline__ void softmax_block(uint32_t trow, const RowCtx<Wn>& rc, float& m_out,
+                                              float& l_out) {
+  float t[NB];
+#pragma unroll
+  for (int c = 0; c < NB / 16; ++c) {
+    uint32_t u[16];
+    tmem_ld16(trow + c * 16, u);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) t[c * 16 + k] = __uint_as_float(u[k]);
+  }
+  tmem_wait_ld();
+  float m = -INFINITY;
+#pragma unroll
+  for (int jj = 0; jj < NB; ++jj) {
+    const int j = KB0 + jj;
+    if (j < Wn::N) {
+      const int pt = j / (Wn::MH * Wn::MW), ph = (j / Wn::MW) % Wn::MH, pw = j % Wn::MW;
+      float v = t[jj] + rc.tb[-(pt * Wn::TS + ph * Wn::WS + pw)];
+      if (MASKED) v = (rc.okt[pt] && rc.okh[ph] && rc.okw[pw]) ? v : -INFINITY;
+      t[jj] = v;
+      m = fmaxf(m, v);
+    } else {
+      t[jj] = -INFINITY;
+    }
+  }
+  const float mm = (m == -INFINITY) ? 0.f : m;
+  float l0 = 0.f, l1 = 0.f;
+  uint32_t pk[NB / 2];
+#pragma unroll
+  for (int jj = 0; jj < NB; jj += 2) {
+    const float p0 = ex2_approx(t[jj] - mm);
+    const float p1 = ex2_approx(t[jj + 1] - mm);
+    l0 += p0;
+    l1 += p1;
+    pk[jj / 2] = pack_bf16x2(p0, p1);
+  }
+#pragma unroll
+  for (int c = 0; c < NB / 16; ++c) tmem_st8(trow + c * 8, &pk[c * 8]);
+  m_out = m;
+  l_out = l0 + l1;
+}
+
+template <class Wn, bool MASKED>
+__device__ __forceinline__ void softmax_all_blocks(int b, uint32_t trow, const RowCtx<Wn>& rc, float* m,
+                                                   float* l) {
+  if (b == 0) softmax_block<Wn, 0, Wn::NB0, MASKED>(trow, rc, m[0], l[0]);
+  if constexpr (Wn::NBLK > 1)
+    if (b == 1) softmax_block<Wn, Wn::NB0, Wn::NB1, MASKED>(trow, rc, m[1], l[1]);
+  if constexpr (Wn::NBLK > 2)
+    if (b == 2) softmax_block<Wn, Wn::NB0 + Wn::NB1, Wn::NB2, MASKED>(trow, rc, m[2], l[2]);
+}
+
+template <class Wn>
+__device__ __forceinline__ int block_start(int b) {
+  return b == 0 ? 0 : (b == 1 ? Wn::NB0 : Wn::NB0 + Wn::NB1);
+}
+template <class Wn>
+__device__ __forceinline__ int block_width(int b) {
+  return b == 0 ? Wn::NB0 : (b == 1 ? Wn::NB1 : Wn::NB2);
+}
+
+template <class Wn>
+__global__ void __launch_bounds__(kAttnThreads, 2) attention_kernel(AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sQ = smem + Wn::OFF_Q;
+  uint8_t* sK = smem + Wn::OFF_K;
+  uint8_t* sV = smem + Wn::OFF_V;
+  float* sT = reinterpret_cast<float*>(smem + Wn::OFF_T);
+  uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + Wn::OFF_BAR);
+  uint64_t* bar_s = bar_ld + 1;
+  uint64_t* bar_o = bar_ld + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_ld + 3);
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Geom& g = a.g;
+  const long long nitems = a.nwin * g.heads;
+  const uint32_t slab_bytes = Wn::NPAD * kSlabRowBytes;
+
+  if (tid == 0) {
+    mbar_init(bar_ld, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  // Rows of the last query tile past the slab are never loaded: keep them zero.
+  for (int k = Wn::NPAD * kSlabRowBytes / 16 + tid; k < Wn::QROWS * kSlabRowBytes / 16; k += kAttnThreads)
+    reinterpret_cast<uint4*>(sQ)[k] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+
+  uint32_t ph_ld = 0, ph_s = 0, ph_o = 0;
+  int cur_head = -1;
+  const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
+
+#pragma unroll 1
+  for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int h = (int)(item / a.nwin);
+    const long long wl = item % a.nwin;
+    const long long win = a.win0 + wl;
+    if (tid == 0) {
+      const __nv_bfloat16* base = a.qkv + ((size_t)wl * g.heads + h) * 3 * (size_t)Wn::NPAD * kD;
+      mbar_arrive_expect_tx(bar_ld, 3 * slab_bytes);
+      bulk_g2s(sQ, base, slab_bytes, bar_ld);
+      bulk_g2s(sK, base + (size_t)Wn::NPAD * kD, slab_bytes, bar_ld);
+      bulk_g2s(sV, base + 2 * (size_t)Wn::NPAD * kD, slab_bytes, bar_ld);
+    }
+    if (h != cur_head) {
+      for (int k = tid; k < Wn::TABLE; k += kAttnThreads)
+        sT[k] = __bfloat162float(a.table[(size_t)k * g.heads + h]) * kLog2e;
+      cur_head = h;
+    }
+    if (!mbar_wait(bar_ld, ph_ld, a.ctx.err, kErrWaitLoad, a.ctx.wait_limit)) s_abort = 1;
+    ph_ld ^= 1;
+    // Key slots past N are padding of the operand tile: zero them.
+    for (int k = tid; k < (Wn::NPAD - Wn::N) * kSlabRowBytes / 16; k += kAttnThreads) {
+      reinterpret_cast<uint4*>(sK + Wn::N * kSlabRowBytes)[k] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(sV + Wn::N * kSlabRowBytes)[k] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (s_abort) break;
+
+    const int split = window_split_bits(g, (int)(win % g.nW));
+    const bool masked = split != 0;
+
+#pragma unroll 1
+    for (int qt = 0; qt < Wn::QTILES; ++qt) {
+      // per-row context
+      const int i = qt * 128 + warp * 32 + lane;
+      const bool warp_active = qt * 128 + warp * 32 < Wn::N;
+      const int ie = i < Wn::N ? i : Wn::N - 1;
+      const int pt_i = ie / (Wn::MH * Wn::MW), ph_i = (ie / Wn::MW) % Wn::MH, pw_i = ie % Wn::MW;
+      RowCtx<Wn> rc;
+      rc.tb = sT + (pt_i + Wn::P - 1) * Wn::TS + (ph_i + Wn::MH - 1) * Wn::WS + (pw_i + Wn::MW - 1);
+      {
+        const int cut_t = Wn::P - g.sh[0], cut_h = Wn::MH - g.sh[1], cut_w = Wn::MW - g.sh[2];
+        const bool rt = pt_i >= cut_t, rh = ph_i >= cut_h, rw = pw_i >= cut_w;
+#pragma unroll
+        for (int k = 0; k < Wn::P; ++k) rc.okt[k] = !(split & 1) || ((k >= cut_t) == rt);
+#pragma unroll
+        for (int k = 0; k < Wn::MH; ++k) rc.okh[k] = !(split & 2) || ((k >= cut_h) == rh);
+#pragma unroll
+        for (int k = 0; k < Wn::MW; ++k) rc.okw[k] = !(split & 4) || ((k >= cut_w) == rw);
+      }
+      float mrow[3] = {-INFINITY, -INFINITY, -INFINITY}, lrow[3] = {0.f, 0.f, 0.f};
+
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          umma_ss(tmem, smem_desc(qaddr + qt * 8192 + ks * 256, 128, 512),
+                  smem_desc(kaddr + ks * 256, 128, 512), idesc_bf16(128, Wn::NB0, 0, 0), ks);
+        umma_commit(bar_s);
+      }
+#pragma unroll 1
+      for (int b = 0; b < Wn::NBLK; ++b) {
+        if (!mbar_wait(bar_s, ph_s, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
+        ph_s ^= 1;
+        __syncthreads();
+        tc_fence_after();
+        if (warp_active && !s_abort) {
+          if (masked)
+            softmax_all_blocks<Wn, true>(b, trow, rc, mrow, lrow);
+          else
+            softmax_all_blocks<Wn, false>(b, trow, rc, mrow, lrow);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && !s_abort) {
+          tc_fence_after();
+          const int kb0 = block_start<Wn>(b), nb = block_width<Wn>(b);
+          for (int ks = 0; ks < nb / 16; ++ks)
+            umma_ts(tmem + kOCol + 32 * b, tmem + 8 * ks,
+                    smem_desc(vaddr + ((kb0 + 16 * ks) >> 3) * 512, 512, 128), idesc_bf16(128, kD, 0, 1),
+                    ks > 0);
+          if (b + 1 < Wn::NBLK) {
+            const int nk0 = block_start<Wn>(b + 1), nnb = block_width<Wn>(b + 1);
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+              umma_ss(tmem, smem_desc(qaddr + qt * 8192 + ks * 256, 128, 512),
+                      smem_desc(kaddr + (nk0 >> 3) * 512 + ks * 256, 128, 512), idesc_bf16(128, nnb, 0, 0),
+                      ks);
+            umma_commit(bar_s);
+          } else {
+            umma_commit(bar_o);
+          }
+        }
+        if (s_abort) break;
+      }
+      if (s_abort) break;
+      if (!mbar_wait(bar_o, ph_o, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
+      ph_o ^= 1;
+      __syncthreads();
+      tc_fence_after();
+      if (warp_active && !s_abort) {
+        float M = mrow[0];
+#pragma unroll
+        for (int b = 1; b < Wn::NBLK; ++b) M = fmaxf(M, mrow[b]);
+        float alpha[3], L = 0.f;
+#pragma unroll
+        for (int b = 0; b < Wn::NBLK; ++b) {
+          alpha[b] = mrow[b] == -INFINITY ? 0.f : ex2_approx(mrow[b] - M);
+          L += alpha[b] * lrow[b];
+        }
+        const float inv = 1.0f / L;
+        float o[kD];
+#pragma unroll
+        for (int k = 0; k < kD; ++k) o[k] = 0.f;
+#pragma unroll
+        for (int b = 0; b < Wn::NBLK; ++b) {
+          uint32_t u0[16], u1[16];
+          tmem_ld16(trow + kOCol + 32 * b, u0);
+          tmem_ld16(trow + kOCol + 32 * b + 16, u1);
+          tmem_wait_ld();
+          const float f = alpha[b] * inv;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            o[k] = fmaf(__uint_as_float(u0[k]), f, o[k]);
+            o[16 + k] = fmaf(__uint_as_float(u1[k]), f, o[16 + k]);
+          }
+        }
+        if (i < Wn::N) {
+          __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            reinterpret_cast<uint4*>(dst)[q] =
+                make_uint4(pack_bf16x2(o[8 * q + 0], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                           pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s_abort) break;
+    }
+    if (s_abort) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <class Wn>
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t e = cudaFuncSetAttribute(attention_kernel<Wn>, cudaFuncAttributeMaxDynamicSharedMemorySize, Wn::SMEM);
+  if (e != cudaSuccess) return e;
+  const long long items = a.nwin * a.g.heads;
+  long long grid = 2LL * sms;
+  if (grid > items) grid = items;
+  attention_kernel<Wn><<<(unsigned)grid, kAttnThreads, Wn::SMEM, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+int pick_bn(int n) {
+  if (n <= kMaxBN && n % 16 == 0) return n;
+  for (int bn = kMaxBN; bn >= 16; bn -= 16)
+    if (n % bn == 0) return bn;
+  return 0;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
+  cudaError_t e =
+      cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes());
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((a.rows + kBM - 1) / kBM), (unsigned)(a.Ntot / a.BN));
+  gemm_kernel<MODE><<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bf16_window_supported(const Geom& g) {
+  const int P = g.win[0], MH = g.win[1], MW = g.win[2];
+  return (P == 8 && MH == 7 && MW == 7) || (P == 4 && MH == 7 && MW == 7) || (P == 2 && MH == 7 && MW == 7) ||
+         (P == 1 && MH == 7 && MW == 7) || (P == 4 && MH == 4 && MW == 4) || (P == 2 && MH == 2 && MW == 2) ||
+         (P == 1 && MH == 1 && MW == 1);
+}
+
+size_t bf16_scratch_bytes(const Geom& g, long long nwin) {
+  const size_t qkv = (size_t)nwin * g.heads * 3 * g.Npad * kD * 2;
+  const size_t o = (size_t)nwin * g.N * g.C * 2;
+  return qkv + o;
+}
+
+cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
+                              const void* bqkv, const void* Wproj, const void* bproj, const void* table,
+                              void* out, void* scratch, long long win0, long long nwin, cudaStream_t st) {
+  __nv_bfloat16* qkv = static_cast<__nv_bfloat16*>(scratch);
+  __nv_bfloat16* o = qkv + (size_t)nwin * g.heads * 3 * g.Npad * kD;
+
+  GemmArgs ga{};
+  ga.g = g;
+  ga.ctx = ctx;
+  ga.A = static_cast<const __nv_bfloat16*>(x);
+  ga.Wt = static_cast<const __nv_bfloat16*>(Wqkv);
+  ga.bias = static_cast<const __nv_bfloat16*>(bqkv);
+  ga.dst = qkv;
+  ga.win0 = win0;
+  ga.rows = nwin * g.N;
+  ga.K = g.C;
+  ga.Ntot = 3 * g.C;
+  ga.BN = pick_bn(3 * g.C);
+  ga.qscale = kLog2e / sqrtf((float)kD);
+  cudaError_t e = launch_gemm<kQKV>(ga, st);
+  if (e != cudaSuccess) return e;
+
+  AttnArgs aa{};
+  aa.g = g;
+  aa.ctx = ctx;
+  aa.qkv = qkv;
+  aa.table = static_cast<const __nv_bfloat16*>(table);
+  aa.o = o;
+  aa.win0 = win0;
+  aa.nwin = nwin;
+  const int P = g.win[0], MH = g.win[1], MW = g.win[2];
+  if (P == 8 && MH == 7 && MW == 7) e = launch_attention<Win<8, 7, 7>>(aa, st);
+  else if (P == 4 && MH == 7 && MW == 7) e = launch_attention<Win<4, 7, 7>>(aa, st);
+  else if (P == 2 && MH == 7 && MW == 7) e = launch_attention<Win<2, 7, 7>>(aa, st);
+  else if (P == 1 && MH == 7 && MW == 7) e = launch_attention<Win<1, 7, 7>>(aa, st);
+  else if (P == 4 && MH == 4 && MW == 4) e = launch_attention<Win<4, 4, 4>>(aa, st);
+  else if (P == 2 && MH == 2 && MW == 2) e = launch_attention<Win<2, 2, 2>>(aa, st);
+  else if (P == 1 && MH == 1 && MW == 1) e = launch_attention<Win<1, 1, 1>>(aa, st);
+  else return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+
+  GemmArgs gp = ga;
+  gp.A = o;
+  gp.Wt = static_cast<const __nv_bfloat16*>(Wproj);
+  gp.bias = static_cast<const __nv_bfloat16*>(bproj);
+  gp.dst = static_cast<__nv_bfloat16*>(out);
+  gp.Ntot = g.C;
+  gp.BN = pick_bn(g.C);
+  gp.qscale = 1.0f;
+  return launch_gemm<kPROJ>(gp, st);
+}
+
+}  // namespace vswin

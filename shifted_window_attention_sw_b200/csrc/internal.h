@@ -1,0 +1,43 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "geometry.cuh"
+
+namespace vswin {
+
+// Per-launch context: the device error word and the wait limit.
+struct KernelCtx {
+  int* err;                       // device error word (0 = fine)
+  unsigned long long wait_limit;  // ns
+};
+
+// Device-side error codes written to the error word.
+enum : int {
+  kErrWaitLoad = 0x101,
+  kErrWaitMma = 0x102,
+  kErrWaitSelftest = 0x1FF,
+};
+
+void count_launch(int n = 1);
+
+// fp32 path (simt_path.cu)
+cudaError_t launch_f32_forward(const Geom& g, const float* x, const float* Wqkv, const float* bqkv,
+                               const float* Wproj, const float* bproj, const float* table, float* out,
+                               float* scratch_qkv, float* scratch_o, cudaStream_t st);
+size_t f32_scratch_floats(const Geom& g, size_t* qkv_floats, size_t* o_floats);
+
+cudaError_t launch_index_maps(const Geom& g, int* win_src, int* region, int* bias_idx, cudaStream_t st);
+
+cudaError_t launch_selftest_timeout(const KernelCtx& ctx, cudaStream_t st);
+
+// bf16 path (bf16_path.cu)
+bool bf16_window_supported(const Geom& g);
+// Scratch for `nwin` windows: QKV slabs then the attention output.
+size_t bf16_scratch_bytes(const Geom& g, long long nwin);
+cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
+                              const void* bqkv, const void* Wproj, const void* bproj, const void* table,
+                              void* out, void* scratch, long long win0, long long nwin, cudaStream_t st);
+
+}  // namespace vswin

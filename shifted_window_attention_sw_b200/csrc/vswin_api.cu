@@ -1,0 +1,332 @@
+// C ABI of the library: argument validation, error reporting, scratch
+// management and dispatch to the fp32 and bf16 paths. See include/vswin.h.
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/vswin.h"
+#include "internal.h"
+
+namespace vswin {
+
+__device__ int g_error_word;
+
+namespace {
+
+thread_local std::string t_last_error;
+std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned long long> g_wait_limit_ns{1000000000ULL};
+std::mutex g_mu;
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return status;
+}
+
+int fail_cuda(cudaError_t e, const char* what) {
+  return fail(VSWIN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+// Device address of the error word for the current device (looked up once per
+// device, with that device current).
+int error_word(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VSWIN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_error_word);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(error word)");
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return VSWIN_OK;
+}
+
+int make_ctx(KernelCtx* ctx) {
+  int* err = nullptr;
+  const int st = error_word(&err);
+  if (st != VSWIN_OK) return st;
+  ctx->err = err;
+  ctx->wait_limit = g_wait_limit_ns.load();
+  return VSWIN_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+int build_geom(int B, int T, int H, int W, int C, int heads, const int* window, const int* shift, Geom* g) {
+  if (!window || !shift) return fail(VSWIN_ERR_INVALID_ARG, "window and shift must be non-NULL host arrays of 3");
+  if (B <= 0 || T <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0)
+    return fail(VSWIN_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d H=%d W=%d C=%d heads=%d)", B, T, H, W,
+                C, heads);
+  if (C % heads != 0) return fail(VSWIN_ERR_INVALID_ARG, "C=%d is not a multiple of heads=%d", C, heads);
+  std::memset(g, 0, sizeof(*g));
+  g->B = B;
+  g->T = T;
+  g->H = H;
+  g->W = W;
+  g->C = C;
+  g->heads = heads;
+  g->d = C / heads;
+  g->L[0] = T;
+  g->L[1] = H;
+  g->L[2] = W;
+  long long nW = 1, N = 1;
+  for (int a = 0; a < 3; ++a) {
+    if (window[a] < 1) return fail(VSWIN_ERR_INVALID_ARG, "window[%d]=%d must be >= 1", a, window[a]);
+    if (shift[a] < 0 || shift[a] >= window[a])
+      return fail(VSWIN_ERR_INVALID_ARG, "shift[%d]=%d must lie in [0, window[%d]=%d)", a, shift[a], a, window[a]);
+    g->win[a] = window[a];
+    g->sh[a] = shift[a];
+    const long long Lp = ((long long)g->L[a] + window[a] - 1) / window[a] * window[a];
+    if (Lp > (1 << 30)) return fail(VSWIN_ERR_INVALID_ARG, "extent too large");
+    g->Lp[a] = (int)Lp;
+    g->nw[a] = (int)(Lp / window[a]);
+    nW *= g->nw[a];
+    N *= window[a];
+  }
+  if (N > (1 << 20) || nW > (1LL << 30)) return fail(VSWIN_ERR_UNSUPPORTED, "window or grid too large");
+  g->nW = (int)nW;
+  g->N = (int)N;
+  g->Npad = ceil_to(g->N, 16);
+  g->table_rows = (2 * window[0] - 1) * (2 * window[1] - 1) * (2 * window[2] - 1);
+  g->windows = (long long)B * nW;
+  g->tokens = (long long)B * T * H * W;
+  if (g->windows * g->N > (1LL << 31) - 1) return fail(VSWIN_ERR_UNSUPPORTED, "B * windows * N exceeds 2^31");
+  return VSWIN_OK;
+}
+
+int check_layer_ptrs(const void* x, const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                     const void* table, const void* out, const Geom& g, size_t elem, size_t align) {
+  const void* ptrs[] = {x, Wqkv, bqkv, Wproj, bproj, table, out};
+  const char* names[] = {"x", "Wqkv", "bqkv", "Wproj", "bproj", "bias_table", "out"};
+  for (int k = 0; k < 7; ++k)
+    if (!ptrs[k]) return fail(VSWIN_ERR_INVALID_ARG, "%s is NULL", names[k]);
+  const void* big[] = {x, Wqkv, Wproj, out};
+  const char* bign[] = {"x", "Wqkv", "Wproj", "out"};
+  for (int k = 0; k < 4; ++k)
+    if (!aligned(big[k], align)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not %zu-byte aligned", bign[k], align);
+  const void* small[] = {bqkv, bproj, table};
+  const char* smalln[] = {"bqkv", "bproj", "bias_table"};
+  for (int k = 0; k < 3; ++k)
+    if (!aligned(small[k], elem)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not %zu-byte aligned", smalln[k], elem);
+  const size_t act = (size_t)g.tokens * g.C * elem;
+  if (overlap(x, act, out, act)) return fail(VSWIN_ERR_INVALID_ARG, "x and out overlap");
+  return VSWIN_OK;
+}
+
+long long chunk_windows(const Geom& g) {
+  static long long budget = [] {
+    const char* s = std::getenv("VSWIN_CHUNK_MB");
+    long long mb = s ? std::atoll(s) : 64;
+    if (mb < 1) mb = 1;
+    return mb << 20;
+  }();
+  const long long per = (long long)bf16_scratch_bytes(g, 1);
+  long long cap = budget / per;
+  if (cap < 1) cap = 1;
+  if (cap >= g.windows) return g.windows;
+  const long long nchunks = (g.windows + cap - 1) / cap;
+  return (g.windows + nchunks - 1) / nchunks;
+}
+
+int forward_bf16_device(const void* x, const Geom& g, const void* Wqkv, const void* bqkv, const void* Wproj,
+                        const void* bproj, const void* table, void* out, cudaStream_t st) {
+  if (g.d != 32) return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path needs head width 32 (C/heads = %d)", g.d);
+  if (!bf16_window_supported(g))
+    return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path has no kernel for window (%d,%d,%d)", g.win[0], g.win[1],
+                g.win[2]);
+  KernelCtx ctx;
+  int status = make_ctx(&ctx);
+  if (status != VSWIN_OK) return status;
+  const long long per_chunk = chunk_windows(g);
+  const size_t bytes = bf16_scratch_bytes(g, per_chunk);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, bytes, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(VSWIN_ERR_NO_MEMORY, "cudaMallocAsync(%zu bytes): %s", bytes, cudaGetErrorString(e));
+  }
+  for (long long w0 = 0; w0 < g.windows; w0 += per_chunk) {
+    const long long n = (g.windows - w0) < per_chunk ? (g.windows - w0) : per_chunk;
+    e = launch_bf16_chunk(g, ctx, x, Wqkv, bqkv, Wproj, bproj, table, out, scratch, w0, n, st);
+    if (e != cudaSuccess) {
+      cudaFreeAsync(scratch, st);
+      return fail_cuda(e, "bf16 kernel launch");
+    }
+  }
+  e = cudaFreeAsync(scratch, st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaFreeAsync");
+  return VSWIN_OK;
+}
+
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
+
+}  // namespace vswin
+
+using namespace vswin;
+
+extern "C" {
+
+int vswin_version(void) { return 100; }
+
+const char* vswin_last_error(void) { return t_last_error.c_str(); }
+
+unsigned long long vswin_launch_count(void) { return g_launches.load(); }
+
+void vswin_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns ? ns : 1); }
+
+int vswin_clamp_window(int T, int H, int W, const int* window_in, const int* shift_in, int* window_out,
+                       int* shift_out) {
+  if (!window_in || !shift_in || !window_out || !shift_out)
+    return fail(VSWIN_ERR_INVALID_ARG, "NULL argument to vswin_clamp_window");
+  const int L[3] = {T, H, W};
+  for (int a = 0; a < 3; ++a) {
+    if (L[a] <= 0 || window_in[a] < 1 || shift_in[a] < 0)
+      return fail(VSWIN_ERR_INVALID_ARG, "invalid extent, window or shift on axis %d", a);
+    if (L[a] <= window_in[a]) {
+      window_out[a] = L[a];
+      shift_out[a] = 0;
+    } else {
+      window_out[a] = window_in[a];
+      shift_out[a] = shift_in[a];
+    }
+  }
+  return VSWIN_OK;
+}
+
+int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                       const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                       const void* bias_table, void* out, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  st = check_layer_ptrs(x, Wqkv, bqkv, Wproj, bproj, bias_table, out, g, 2, 16);
+  if (st != VSWIN_OK) return st;
+  return forward_bf16_device(x, g, Wqkv, bqkv, Wproj, bproj, bias_table, out, static_cast<cudaStream_t>(stream));
+}
+
+int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                           const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
+                           const void* bproj, const void* bias_table, void* out, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  st = check_layer_ptrs(x, Wqkv, bqkv, Wproj, bproj, bias_table, out, g, 4, 4);
+  if (st != VSWIN_OK) return st;
+  if (g.N > 4096) return fail(VSWIN_ERR_UNSUPPORTED, "fp32 path supports N <= 4096 (N = %d)", g.N);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  size_t nq = 0, no = 0;
+  f32_scratch_floats(g, &nq, &no);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, (nq + no) * sizeof(float), s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(VSWIN_ERR_NO_MEMORY, "cudaMallocAsync: %s", cudaGetErrorString(e));
+  }
+  float* sq = static_cast<float*>(scratch);
+  e = launch_f32_forward(g, static_cast<const float*>(x), static_cast<const float*>(Wqkv),
+                         static_cast<const float*>(bqkv), static_cast<const float*>(Wproj),
+                         static_cast<const float*>(bproj), static_cast<const float*>(bias_table),
+                         static_cast<float*>(out), sq, sq + nq, s);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) return fail_cuda(e, "fp32 kernel launch");
+  if (e2 != cudaSuccess) return fail_cuda(e2, "cudaFreeAsync");
+  return VSWIN_OK;
+}
+
+int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads, const int* window,
+                            const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
+                            const void* bproj, const void* bias_table, void* out_host, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  if (!x_host || !out_host) return fail(VSWIN_ERR_INVALID_ARG, "x_host and out_host must be non-NULL");
+  const size_t act = (size_t)g.tokens * g.C * 2;
+  if (overlap(x_host, act, out_host, act)) return fail(VSWIN_ERR_INVALID_ARG, "x_host and out_host overlap");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* buf = nullptr;
+  const size_t act_pad = (act + 255) / 256 * 256;
+  cudaError_t e = cudaMallocAsync(&buf, 2 * act_pad, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(VSWIN_ERR_NO_MEMORY, "cudaMallocAsync: %s", cudaGetErrorString(e));
+  }
+  void* xd = buf;
+  void* od = static_cast<uint8_t*>(buf) + act_pad;
+  e = cudaMemcpyAsync(xd, x_host, act, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) {
+    st = check_layer_ptrs(xd, Wqkv, bqkv, Wproj, bproj, bias_table, od, g, 2, 16);
+    if (st == VSWIN_OK) st = forward_bf16_device(xd, g, Wqkv, bqkv, Wproj, bproj, bias_table, od, s);
+    if (st == VSWIN_OK) {
+      e = cudaMemcpyAsync(out_host, od, act, cudaMemcpyDeviceToHost, s);
+      if (e != cudaSuccess) st = fail_cuda(e, "cudaMemcpyAsync(out)");
+    }
+  } else {
+    st = fail_cuda(e, "cudaMemcpyAsync(x)");
+  }
+  cudaFreeAsync(buf, s);
+  e = cudaStreamSynchronize(s);
+  if (st == VSWIN_OK && e != cudaSuccess) st = fail_cuda(e, "cudaStreamSynchronize");
+  return st;
+}
+
+int vswin_wmsa_index_maps(int B, int T, int H, int W, const int* window, const int* shift, int* win_src,
+                          int* region, int* bias_idx, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, 1, 1, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  if (!win_src && !region && !bias_idx) return VSWIN_OK;
+  if ((long long)g.N * g.N > (1LL << 31) - 1) return fail(VSWIN_ERR_UNSUPPORTED, "N*N exceeds 2^31");
+  cudaError_t e = launch_index_maps(g, win_src, region, bias_idx, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "index map kernel launch");
+  return VSWIN_OK;
+}
+
+int vswin_poll_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "cudaStreamSynchronize");
+  int* err = nullptr;
+  int st = error_word(&err);
+  if (st != VSWIN_OK) return st;
+  int word = 0;
+  e = cudaMemcpy(&word, err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e, "reading the error word");
+  if (word == 0) return VSWIN_OK;
+  const int zero = 0;
+  e = cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return fail_cuda(e, "clearing the error word");
+  return fail(VSWIN_ERR_TIMEOUT, "a kernel wait gave up (code 0x%x)", word);
+}
+
+int vswin_selftest_timeout(void* stream) {
+  KernelCtx ctx;
+  int st = make_ctx(&ctx);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = launch_selftest_timeout(ctx, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "self-test launch");
+  return VSWIN_OK;
+}
+
+}  // extern "C"

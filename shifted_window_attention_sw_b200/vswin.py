@@ -1,0 +1,187 @@
+"""ctypes binding of ``libvswin.so`` (``include/vswin.h``): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; PyTorch only owns
+device memory and streams. There is no fallback: if the library is missing
+or a call fails, a ``VswinError`` is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvswin.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_MEMORY = range(6)
+
+# Every symbol include/vswin.h declares.
+EXPORTS = (
+    "vswin_wmsa_forward",
+    "vswin_wmsa_forward_f32",
+    "vswin_wmsa_forward_host",
+    "vswin_wmsa_index_maps",
+    "vswin_clamp_window",
+    "vswin_last_error",
+    "vswin_poll_error",
+    "vswin_launch_count",
+    "vswin_set_wait_limit_ns",
+    "vswin_selftest_timeout",
+    "vswin_version",
+)
+
+
+class VswinError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"vswin status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_IP = ctypes.POINTER(ctypes.c_int)
+
+
+def lib():
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise VswinError(-1, f"{LIB_PATH} is missing: build it with "
+                                 "`python -m shifted_window_attention_sw_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        layer = [_P, _I, _I, _I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P, _P, _P, _P]
+        for name in ("vswin_wmsa_forward", "vswin_wmsa_forward_f32", "vswin_wmsa_forward_host"):
+            fn = getattr(L, name)
+            fn.argtypes = layer
+            fn.restype = _I
+        L.vswin_wmsa_index_maps.argtypes = [_I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P]
+        L.vswin_wmsa_index_maps.restype = _I
+        L.vswin_clamp_window.argtypes = [_I, _I, _I, _IP, _IP, _IP, _IP]
+        L.vswin_clamp_window.restype = _I
+        L.vswin_last_error.argtypes = []
+        L.vswin_last_error.restype = ctypes.c_char_p
+        L.vswin_poll_error.argtypes = [_P]
+        L.vswin_poll_error.restype = _I
+        L.vswin_launch_count.argtypes = []
+        L.vswin_launch_count.restype = ctypes.c_ulonglong
+        L.vswin_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.vswin_set_wait_limit_ns.restype = None
+        L.vswin_selftest_timeout.argtypes = [_P]
+        L.vswin_selftest_timeout.restype = _I
+        L.vswin_version.argtypes = []
+        L.vswin_version.restype = _I
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().vswin_last_error().decode()
+
+
+def _check(status):
+    if status != OK:
+        raise VswinError(status, last_error())
+
+
+def _i3(v):
+    v = tuple(int(a) for a in v)
+    if len(v) != 3:
+        raise ValueError("window and shift need 3 entries")
+    return (ctypes.c_int * 3)(*v)
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _layer_call(fn, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out, stream):
+    B, T, H, W, C = x.shape
+    _check(fn(_ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv),
+              _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out), _stream_handle(stream)))
+    return out
+
+
+def _prep(x, tensors, dtype):
+    for name, t in tensors.items():
+        if t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def wmsa_forward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):
+    """bf16 layer forward on the GPU (tcgen05 path). All tensors bf16 on one CUDA device."""
+    if out is None:
+        out = torch.empty_like(x)
+    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.bfloat16)
+    return _layer_call(lib().vswin_wmsa_forward, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out,
+                       stream)
+
+
+def wmsa_forward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):
+    """fp32 layer forward on the GPU (FP32 FMA path). All tensors float32 on one CUDA device."""
+    if out is None:
+        out = torch.empty_like(x)
+    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.float32)
+    return _layer_call(lib().vswin_wmsa_forward_f32, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads,
+                       out, stream)
+
+
+def wmsa_forward_host(x_host, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out_host, stream=None):
+    """bf16 forward with x and out in host memory (copies inside the call; synchronises)."""
+    _prep(x_host, dict(x_host=x_host, out_host=out_host), torch.bfloat16)
+    return _layer_call(lib().vswin_wmsa_forward_host, x_host, window, shift, Wqkv, bqkv, Wproj, bproj, table,
+                       heads, out_host, stream)
+
+
+def index_maps(B, T, H, W, window, shift, device="cuda", stream=None):
+    """(win_src, region, bias_idx) as int32 device tensors."""
+    nW = 1
+    N = 1
+    for L, w in zip((T, H, W), window):
+        nW *= -(-L // w)
+        N *= w
+    win_src = torch.empty(B * nW * N, dtype=torch.int32, device=device)
+    region = torch.empty(nW * N, dtype=torch.int32, device=device)
+    bias_idx = torch.empty(N * N, dtype=torch.int32, device=device)
+    _check(lib().vswin_wmsa_index_maps(B, T, H, W, _i3(window), _i3(shift), _ptr(win_src), _ptr(region),
+                                       _ptr(bias_idx), _stream_handle(stream)))
+    return win_src, region, bias_idx
+
+
+def clamp_window(T, H, W, window, shift):
+    wo = (ctypes.c_int * 3)()
+    so = (ctypes.c_int * 3)()
+    _check(lib().vswin_clamp_window(T, H, W, _i3(window), _i3(shift), wo, so))
+    return tuple(wo), tuple(so)
+
+
+def poll_error(stream=None) -> int:
+    """Synchronise and return the device error status (0 = OK, 4 = a kernel wait gave up)."""
+    return int(lib().vswin_poll_error(_stream_handle(stream)))
+
+
+def launch_count() -> int:
+    return int(lib().vswin_launch_count())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().vswin_set_wait_limit_ns(int(ns))
+
+
+def selftest_timeout(stream=None) -> None:
+    _check(lib().vswin_selftest_timeout(_stream_handle(stream)))
+
+
+def version() -> int:
+    return int(lib().vswin_version())

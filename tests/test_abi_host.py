@@ -1,0 +1,105 @@
+"""The C ABI on the host: the library loads, exports every symbol the header
+declares, and rejects bad arguments before launching anything. CPU only."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from shifted_window_attention_sw_b200 import build as build_mod
+from shifted_window_attention_sw_b200 import vswin
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vswin.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return vswin.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vswin_\w+)\s*\(", text)))
+
+
+def test_header_declares_binding_exports():
+    assert sorted(vswin.EXPORTS) == _declared()
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert vswin.version() >= 100
+
+
+# fake device pointers: never dereferenced, because validation fails first
+A16 = 1 << 20
+
+
+def _call(fn, x=A16, B=1, T=8, H=14, W=14, C=96, heads=3, window=(8, 7, 7), shift=(4, 3, 3),
+          Wqkv=A16 * 2, bqkv=A16 * 3, Wproj=A16 * 4, bproj=A16 * 5, table=A16 * 6, out=A16 * 64):
+    w = (ctypes.c_int * 3)(*window) if window is not None else None
+    s = (ctypes.c_int * 3)(*shift) if shift is not None else None
+    p = lambda v: ctypes.c_void_p(v) if v else None  # noqa: E731
+    return fn(p(x), B, T, H, W, C, heads, w, s, p(Wqkv), p(bqkv), p(Wproj), p(bproj), p(table), p(out), None)
+
+
+@pytest.mark.parametrize("name", ["vswin_wmsa_forward", "vswin_wmsa_forward_f32"])
+@pytest.mark.parametrize(
+    "kw",
+    [
+        dict(B=0), dict(T=-1), dict(C=0), dict(heads=0),
+        dict(C=96, heads=5),                      # C % heads != 0
+        dict(shift=(8, 3, 3)),                    # shift >= window
+        dict(shift=(-1, 0, 0)),
+        dict(window=(0, 7, 7)),
+        dict(window=None),
+        dict(x=0), dict(out=0), dict(Wqkv=0), dict(bqkv=0), dict(Wproj=0), dict(bproj=0), dict(table=0),
+        dict(x=A16 + 2),                          # misaligned
+        dict(out=A16 + 8),                        # overlaps x
+    ],
+)
+def test_invalid_arguments_launch_nothing(L, name, kw):
+    before = vswin.launch_count()
+    rc = _call(getattr(L, name), **kw)
+    assert rc == vswin.ERR_INVALID_ARG, (rc, vswin.last_error())
+    assert vswin.last_error()
+    assert vswin.launch_count() == before
+
+
+@pytest.mark.parametrize(
+    "kw",
+    [dict(C=128, heads=2),                          # head width 64
+     dict(window=(3, 7, 7), shift=(1, 3, 3)),      # no kernel compiled for this window
+     dict(window=(16, 7, 7), shift=(8, 3, 3))],    # N = 784 > 400
+)
+def test_bf16_unsupported_shapes(L, kw):
+    before = vswin.launch_count()
+    rc = _call(L.vswin_wmsa_forward, **kw)
+    assert rc == vswin.ERR_UNSUPPORTED, (rc, vswin.last_error())
+    assert vswin.launch_count() == before
+
+
+def test_index_maps_rejects_bad_window(L):
+    w = (ctypes.c_int * 3)(8, 7, 7)
+    s = (ctypes.c_int * 3)(8, 0, 0)
+    rc = L.vswin_wmsa_index_maps(1, 8, 7, 7, w, s, None, None, None, None)
+    assert rc == vswin.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize(
+    "dims,window,shift,ew,es",
+    [
+        ((16, 56, 56), (8, 7, 7), (4, 3, 3), (8, 7, 7), (4, 3, 3)),
+        ((8, 14, 14), (8, 7, 7), (4, 3, 3), (8, 7, 7), (0, 3, 3)),   # T == P: window = 8, shift 0
+        ((16, 7, 7), (8, 7, 7), (4, 3, 3), (8, 7, 7), (4, 0, 0)),    # Swin-B stage 4
+        ((4, 5, 9), (8, 7, 7), (4, 3, 3), (4, 5, 7), (0, 0, 3)),
+    ],
+)
+def test_clamp_window(L, dims, window, shift, ew, es):
+    w, s = vswin.clamp_window(*dims, window, shift)
+    assert w == ew and s == es
