@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the bf16 (shifted-)window attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl vswin|reference]
+
+A step is one pass of the whole layer path over one batch: for the headline
+workload (Swin-T stage 1, 32x224^2 clips, batch 8) the W-MSA layer and the
+SW-MSA layer of a block pair, each on the (8, 16, 56, 56, 96) token tensor.
+Inputs are synthetic and seeded, resident in HBM before timing; L2 is flushed
+by a 512 MB write before every timed step (outside the step's events).
+
+One JSON line is printed by rank 0. ``value`` is layer-tokens per second for
+the whole job (every token passes through both layers of the pair), timed with
+CUDA events, the slowest rank's time over the sum of all ranks' tokens. With
+``--impl reference`` the double-precision CPU oracle is timed instead, on a
+bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from shifted_window_attention_sw_b200 import replicas  # noqa: E402
+from shifted_window_attention_sw_b200.accounting import layer_work  # noqa: E402
+from shifted_window_attention_sw_b200.inputs import workload_layer_inputs  # noqa: E402
+from shifted_window_attention_sw_b200.workloads import HEADLINE, WORKLOADS  # noqa: E402
+
+METRIC = "SW-MSA layer tokens/s and TFLOP/s (frac of bf16 peak), Swin-T stage1 32×224² b8"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def workload_config(wl):
+    layers = []
+    for ly in wl.layers:
+        layers.append({"B": ly.B, "T": ly.T, "H": ly.H, "W": ly.W, "C": ly.C, "heads": ly.heads,
+                       "window": list(ly.window), "shift": list(ly.shift)})
+    return {"workload": wl.name, "description": wl.description, "layers": layers,
+            "tokens_per_layer": wl.layers[0].B * wl.layers[0].T * wl.layers[0].H * wl.layers[0].W,
+            "l2": "flushed by a 512 MB write before every timed step", "parallelism": "replicas"}
+
+
+def step_work(wl):
+    tot = {"tokens": 0, "flops": 0, "attn_flops": 0, "gemm_flops": 0, "bytes": 0, "exps": 0,
+           "unmasked_pairs": 0, "pairs": 0}
+    for ly in wl.layers:
+        w = layer_work(ly.B, ly.T, ly.H, ly.W, ly.C, ly.heads, ly.window, ly.shift, 2)
+        for k in tot:
+            tot[k] += w[k]
+    return tot
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+        "gpu_idle": "nvmlClocksEventReasonGpuIdle",
+    }
+
+    def __init__(self, device, period_s=0.01):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.nv = None
+        self.handle = None
+        try:
+            import pynvml as nv
+
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            self.nv = nv
+        except Exception as e:  # noqa: BLE001 -- clocks are reported as unavailable
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, const in self.REASONS.items():
+                    if bits & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(wl, target_s, nthreads=0, layers=None):
+    """Time the CPU oracle on a bounded sample of the workload: whole windows of each
+    layer (forward_windows), as many as fit in about target_s seconds."""
+    import oracle
+
+    oracle.build()
+    cores = oracle.max_threads(nthreads)
+    layers = layers if layers is not None else wl.layers
+    inputs = [workload_layer_inputs(wl, ly, scale="baseline").as_f64() for ly in layers]
+
+    def run(nwin_per_layer):
+        tokens = 0
+        t0 = time.perf_counter()
+        for ly, a in zip(layers, inputs):
+            g = oracle.geometry(ly.T, ly.H, ly.W, ly.window, ly.shift)
+            total = ly.B * g["nW"]
+            wins = np.linspace(0, total - 1, num=min(nwin_per_layer, total)).astype(np.int64)
+            oracle.forward_windows(a["x"], ly.window, ly.shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"],
+                                   a["table"], ly.heads, wins, nthreads=nthreads)
+            src, _, _ = oracle.index_maps(ly.B, ly.T, ly.H, ly.W, ly.window, ly.shift)
+            N = g["N"]
+            tokens += int(sum((src[w * N:(w + 1) * N] >= 0).sum() for w in wins))
+        return tokens, time.perf_counter() - t0
+
+    tok, dt = run(cores)  # calibration: one window per thread and layer
+    n = max(1, int(cores * target_s / max(dt, 1e-6)))
+    if n > cores:
+        tok, dt = run(n)
+    else:
+        n = cores
+    return {"tokens": tok, "seconds": dt, "cores": cores, "windows_per_layer": n}
+
+
+def run_reference(args):
+    rank, world, _ = replicas.env_rank()
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    import oracle
+
+    oracle.build()
+    cores = oracle.max_threads(0)
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    # calibrate the per-step sample so the whole run stays within a few minutes
+    cal = oracle_sample(wl, budget)
+    nwin = cal["windows_per_layer"]
+    times, toks = [], 0
+    for k in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        s = _oracle_fixed(wl, nwin)
+        dt = time.perf_counter() - t0
+        if k >= args.warmup:
+            times.append(dt)
+            toks += s
+    total = sum(times)
+    value = toks / total
+    work = step_work(wl)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "tflops": value * work["flops"] / work["tokens"] / 1e12,
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": "tokens/s", "cores": cores,
+                         "sample": f"{nwin} whole windows of each layer per step (evenly spaced), "
+                                   f"double precision, OpenMP over windows"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+_ORACLE_CACHE = {}
+
+
+def _oracle_fixed(wl, nwin):
+    import oracle
+
+    key = wl.name
+    if key not in _ORACLE_CACHE:
+        _ORACLE_CACHE[key] = [workload_layer_inputs(wl, ly, scale="baseline").as_f64() for ly in wl.layers]
+    tokens = 0
+    for ly, a in zip(wl.layers, _ORACLE_CACHE[key]):
+        g = oracle.geometry(ly.T, ly.H, ly.W, ly.window, ly.shift)
+        total = ly.B * g["nW"]
+        wins = np.linspace(0, total - 1, num=min(nwin, total)).astype(np.int64)
+        oracle.forward_windows(a["x"], ly.window, ly.shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"],
+                               a["table"], ly.heads, wins)
+        src, _, _ = oracle.index_maps(ly.B, ly.T, ly.H, ly.W, ly.window, ly.shift)
+        N = g["N"]
+        tokens += int(sum((src[w * N:(w + 1) * N] >= 0).sum() for w in wins))
+    return tokens
+
+
+# ------------------------------------------------------------------ GPU arm
+def traffic_record(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the kernel
+    source has not changed since the counters were taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = rec.get(kernel)
+    if not entry:
+        return None
+    src = os.path.join(ROOT, "shifted_window_attention_sw_b200", "csrc", entry.get("source", ""))
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if digest != entry.get("sha256"):
+        return None
+    return entry
+
+
+def run_gpu(args):
+    from shifted_window_attention_sw_b200 import build as build_mod
+    from shifted_window_attention_sw_b200 import vswin
+
+    rank, world = replicas.init("nccl")
+    _, _, local = replicas.env_rank()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if rank == 0:
+        build_mod.build()
+    replicas.barrier(device)
+    vswin.lib()
+    wl = WORKLOADS[args.workload]
+    layers = wl.layers
+    ins = [workload_layer_inputs(wl, ly, scale="baseline").to(device) for ly in layers]
+    outs = [torch.empty_like(i.x) for i in ins]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for ly, i, o in zip(layers, ins, outs):
+            vswin.wmsa_forward(i.x, ly.window, ly.shift, i.Wqkv, i.bqkv, i.Wproj, i.bproj, i.table, ly.heads,
+                               out=o, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    if vswin.poll_error(stream) != vswin.OK:
+        raise RuntimeError("kernel error during warm-up: " + vswin.last_error())
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(device)
+    replicas.barrier(device)
+    torch.cuda.synchronize(device)
+    launches0 = vswin.launch_count()
+    vswin.profile_enable(True)
+    sampler.start()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    replicas.barrier(device)
+    vswin.profile_enable(False)
+    prof = vswin.profile_collect()
+    launches = vswin.launch_count() - launches0
+    status = vswin.poll_error(stream)
+    if status != vswin.OK:
+        raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_s = sum(step_ms) / 1e3
+    work = step_work(wl)
+    max_s, tokens, nranks = replicas.combine(total_s, work["tokens"] * args.steps, device)
+    value = tokens / max_s
+    tflops = nranks * work["flops"] * args.steps / max_s / 1e12
+
+    # end to end through the host-buffer entry point: H2D of x and D2H of out inside the timing
+    e2e = None
+    if not args.no_e2e:
+        xh = [i.x.cpu().pin_memory() for i in ins]
+        oh = [torch.empty_like(x).pin_memory() for x in xh]
+        n_e2e = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            for ly, i, x, o in zip(layers, ins, xh, oh):
+                vswin.wmsa_forward_host(x, ly.window, ly.shift, i.Wqkv, i.bqkv, i.Wproj, i.bproj, i.table,
+                                        ly.heads, o, stream=stream)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        replicas.barrier(device)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e_s = e0.elapsed_time(e1) / 1e3
+        e_max, e_tok, _ = replicas.combine(e_s, work["tokens"] * n_e2e, device)
+        e2e = {"value": e_tok / e_max, "unit": "tokens/s",
+               "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in xh)),
+               "d2h_bytes_per_step": int(sum(o.numel() * o.element_size() for o in oh)),
+               "steps": n_e2e, "api": "vswin_wmsa_forward_host (pinned host buffers)"}
+
+    if rank != 0:
+        replicas.shutdown()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    # dominant kernel by device time
+    dom = max(("qkv_gemm", "attention", "proj_gemm"), key=lambda k: prof[k][0])
+    dom_ms, dom_launches = prof[dom]
+    if dom == "attention":
+        dom_work, unit, bound = work["attn_flops"] * args.steps, "TFLOP/s", "tensor"
+        achieved = dom_work / dom_launches / (dom_ms / dom_launches / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        traffic_kernel = "attention_kernel"
+    else:
+        dom_work, unit, bound = work["gemm_flops"] * args.steps, "TFLOP/s", "tensor"
+        achieved = dom_work / (dom_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        traffic_kernel = "gemm_kernel"
+    tr = traffic_record(traffic_kernel)
+    roofline = {
+        "kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+        "frac": achieved / peak, "peak_source": f"{peak_src} bf16 dense (burst)",
+        "avg_launch_us": 1e3 * dom_ms / max(1, dom_launches), "launches": dom_launches,
+        "traffic": tr["bytes_per_launch"] if tr else None,
+        "units_per_launch": "windows x heads of one chunk; FLOPs 4*windows*N^2*C per layer",
+    }
+    kernel_ms = {k: v[0] / args.steps for k, v in prof.items() if v[1]}
+    step_flops_time = work["flops"] / (float(peaks["bf16_tflops"]) * 1e12)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": nranks, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl),
+        "tflops": tflops,
+        "tflops_frac_of_peak": tflops / nranks / float(peaks["bf16_tflops"]),
+        "step_roofline_us": 1e6 * max(step_flops_time, work["bytes"] / (float(peaks["hbm_gbs"]) * 1e9)),
+        "roofline": roofline,
+        "kernel_ms_per_step": kernel_ms,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        s = oracle_sample(wl, args.cpu_sample_s)
+        line["cpu_baseline"] = {
+            "value": s["tokens"] / s["seconds"], "unit": "tokens/s", "cores": s["cores"], "kind": "oracle",
+            "sample": f"{s['windows_per_layer']} evenly spaced whole windows of each layer of the pair "
+                      f"({s['tokens']} layer-tokens, {s['seconds']:.1f} s), double precision",
+        }
+    print(json.dumps(line), flush=True)
+    replicas.shutdown()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["vswin", "reference"], default="vswin")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

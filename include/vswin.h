@@ -148,6 +148,23 @@ void vswin_set_wait_limit_ns(unsigned long long ns);
  */
 int vswin_selftest_timeout(void* stream);
 
+/*
+ * Per-kernel timing for benchmarks. While enabled, every kernel launch of the
+ * library is bracketed by two CUDA events recorded on its launch stream.
+ * vswin_profile_collect waits for the recorded events, adds their elapsed
+ * times per kernel kind into ms[kind] and launch counts into launches[kind]
+ * (arrays of nkinds entries, kinds VSWIN_KERNEL_*), then forgets them.
+ */
+enum {
+  VSWIN_KERNEL_QKV_GEMM = 0,   /* gather + QKV projection (bf16) */
+  VSWIN_KERNEL_ATTENTION = 1,  /* window attention (bf16) */
+  VSWIN_KERNEL_PROJ_GEMM = 2,  /* output projection + scatter (bf16) */
+  VSWIN_KERNEL_OTHER = 3,      /* fp32 path, index maps, self-test */
+  VSWIN_KERNEL_KINDS = 4
+};
+int vswin_profile_enable(int on);
+int vswin_profile_collect(double* ms, unsigned long long* launches, int nkinds);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int vswin_version(void);
 

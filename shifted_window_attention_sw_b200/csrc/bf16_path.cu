@@ -266,7 +266,8 @@ struct Win {
   static constexpr int OFF_V = OFF_K + NPAD * kSlabRowBytes;
   static constexpr int OFF_T = OFF_V + NPAD * kSlabRowBytes;
   static constexpr int OFF_BAR = OFF_T + (TABLE * 4 + 15) / 16 * 16;
-  static constexpr int SMEM = OFF_BAR + 64;
+  // At least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share an SM.
+  static constexpr int SMEM = (OFF_BAR + 64) < 81920 ? 81920 : (OFF_BAR + 64);
   static_assert(NB2 <= 128, "window too large for this path");
   static_assert(NPAD <= 400, "window too large for this path");
 };
@@ -414,10 +415,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attention_kernel(AttnArgs a) 
     }
     if (!mbar_wait(bar_ld, ph_ld, a.ctx.err, kErrWaitLoad, a.ctx.wait_limit)) s_abort = 1;
     ph_ld ^= 1;
-    // Key slots past N are padding of the operand tile: zero them.
-    for (int k = tid; k < (Wn::NPAD - Wn::N) * kSlabRowBytes / 16; k += kAttnThreads) {
-      reinterpret_cast<uint4*>(sK + Wn::N * kSlabRowBytes)[k] = make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(sV + Wn::N * kSlabRowBytes)[k] = make_uint4(0, 0, 0, 0);
+    // Key slots past N are padding of the operand tile: zero them. A slab row
+    // n is spread over four 16-byte pieces at (n/8)*512 + chunk*128 + (n%8)*16.
+    for (int k = tid; k < (Wn::NPAD - Wn::N) * 4; k += kAttnThreads) {
+      const int n = Wn::N + (k >> 2), chunk = k & 3;
+      const int off = (n >> 3) * 512 + chunk * 128 + (n & 7) * 16;
+      *reinterpret_cast<uint4*>(sK + off) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sV + off) = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -553,7 +557,9 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   const long long items = a.nwin * a.g.heads;
   long long grid = 2LL * sms;
   if (grid > items) grid = items;
+  prof_begin(kKindAttn, st);
   attention_kernel<Wn><<<(unsigned)grid, kAttnThreads, Wn::SMEM, st>>>(a);
+  prof_end(kKindAttn, st);
   count_launch();
   return cudaGetLastError();
 }
@@ -571,7 +577,9 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
       cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes());
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((a.rows + kBM - 1) / kBM), (unsigned)(a.Ntot / a.BN));
+  prof_begin(MODE == kQKV ? kKindQkv : kKindProj, st);
   gemm_kernel<MODE><<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(a);
+  prof_end(MODE == kQKV ? kKindQkv : kKindProj, st);
   count_launch();
   return cudaGetLastError();
 }

@@ -22,6 +22,11 @@ enum : int {
 
 void count_launch(int n = 1);
 
+// Optional per-kernel CUDA-event timing (vswin_profile_enable).
+void prof_begin(int kind, cudaStream_t st);
+void prof_end(int kind, cudaStream_t st);
+enum { kKindQkv = 0, kKindAttn = 1, kKindProj = 2, kKindOther = 3, kKinds = 4 };
+
 // fp32 path (simt_path.cu)
 cudaError_t launch_f32_forward(const Geom& g, const float* x, const float* Wqkv, const float* bqkv,
                                const float* Wproj, const float* bproj, const float* table, float* out,

@@ -160,17 +160,23 @@ cudaError_t launch_f32_forward(const Geom& g, const float* x, const float* Wqkv,
   const long long rows = g.windows * g.N;
   if (rows > 2147483647LL) return cudaErrorInvalidConfiguration;
   dim3 g1((unsigned)rows, (3 * g.C + kThreads - 1) / kThreads);
+  prof_begin(kKindOther, st);
   f32_qkv_kernel<<<g1, kThreads, g.C * sizeof(float), st>>>(g, x, Wqkv, bqkv, scratch_qkv);
+  prof_end(kKindOther, st);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2((unsigned)g.windows, g.N, g.heads);
+  prof_begin(kKindOther, st);
   f32_attention_kernel<<<g2, kThreads, (g.N + g.d) * sizeof(float), st>>>(g, scratch_qkv, table, scratch_o);
+  prof_end(kKindOther, st);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g3((unsigned)rows, (g.C + kThreads - 1) / kThreads);
+  prof_begin(kKindOther, st);
   f32_proj_kernel<<<g3, kThreads, g.C * sizeof(float), st>>>(g, scratch_o, Wproj, bproj, out);
+  prof_end(kKindOther, st);
   count_launch();
   return cudaGetLastError();
 }
@@ -180,13 +186,17 @@ cudaError_t launch_index_maps(const Geom& g, int* win_src, int* region, int* bia
   if ((long long)g.N * g.N > work) work = (long long)g.N * g.N;
   long long blocks = (work + 255) / 256;
   if (blocks > 4096) blocks = 4096;
+  prof_begin(kKindOther, st);
   index_maps_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win_src, region, bias_idx);
+  prof_end(kKindOther, st);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_selftest_timeout(const KernelCtx& ctx, cudaStream_t st) {
+  prof_begin(kKindOther, st);
   selftest_timeout_kernel<<<1, 32, 0, st>>>(ctx);
+  prof_end(kKindOther, st);
   count_launch();
   return cudaGetLastError();
 }

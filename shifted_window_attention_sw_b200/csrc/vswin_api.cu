@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/vswin.h"
 #include "internal.h"
@@ -183,6 +184,50 @@ int forward_bf16_device(const void* x, const Geom& g, const void* Wqkv, const vo
 
 void count_launch(int n) { g_launches.fetch_add((unsigned long long)n); }
 
+namespace {
+struct ProfRecord {
+  int kind;
+  cudaEvent_t start, end;
+};
+std::atomic<int> g_prof_on{0};
+std::mutex g_prof_mu;
+std::vector<ProfRecord> g_prof_records;
+std::vector<cudaEvent_t> g_prof_pool;
+cudaEvent_t g_prof_open[kKinds] = {nullptr, nullptr, nullptr, nullptr};
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
+void prof_begin(int kind, cudaStream_t st) {
+  if (!g_prof_on.load()) return;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  cudaEvent_t e = prof_event();
+  if (!e) return;
+  cudaEventRecord(e, st);
+  g_prof_open[kind] = e;
+}
+
+void prof_end(int kind, cudaStream_t st) {
+  if (!g_prof_on.load()) return;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  cudaEvent_t s = g_prof_open[kind];
+  if (!s) return;
+  cudaEvent_t e = prof_event();
+  if (!e) return;
+  cudaEventRecord(e, st);
+  g_prof_records.push_back({kind, s, e});
+  g_prof_open[kind] = nullptr;
+}
+
 }  // namespace vswin
 
 using namespace vswin;
@@ -318,6 +363,35 @@ int vswin_poll_error(void* stream) {
   e = cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return fail_cuda(e, "clearing the error word");
   return fail(VSWIN_ERR_TIMEOUT, "a kernel wait gave up (code 0x%x)", word);
+}
+
+int vswin_profile_enable(int on) {
+  g_prof_on.store(on ? 1 : 0);
+  return VSWIN_OK;
+}
+
+int vswin_profile_collect(double* ms, unsigned long long* launches, int nkinds) {
+  if (!ms || !launches || nkinds < 0) return fail(VSWIN_ERR_INVALID_ARG, "NULL argument to vswin_profile_collect");
+  for (int k = 0; k < nkinds; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  int status = VSWIN_OK;
+  for (const ProfRecord& r : g_prof_records) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.end);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.start, r.end);
+    if (e != cudaSuccess && status == VSWIN_OK) status = fail_cuda(e, "profile events");
+    if (r.kind < nkinds) {
+      ms[r.kind] += t;
+      launches[r.kind] += 1;
+    }
+    g_prof_pool.push_back(r.start);
+    g_prof_pool.push_back(r.end);
+  }
+  g_prof_records.clear();
+  return status;
 }
 
 int vswin_selftest_timeout(void* stream) {

@@ -30,7 +30,11 @@ EXPORTS = (
     "vswin_set_wait_limit_ns",
     "vswin_selftest_timeout",
     "vswin_version",
+    "vswin_profile_enable",
+    "vswin_profile_collect",
 )
+
+KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other")
 
 
 class VswinError(RuntimeError):
@@ -72,6 +76,10 @@ def lib():
         L.vswin_set_wait_limit_ns.restype = None
         L.vswin_selftest_timeout.argtypes = [_P]
         L.vswin_selftest_timeout.restype = _I
+        L.vswin_profile_enable.argtypes = [_I]
+        L.vswin_profile_enable.restype = _I
+        L.vswin_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_ulonglong), _I]
+        L.vswin_profile_collect.restype = _I
         L.vswin_version.argtypes = []
         L.vswin_version.restype = _I
         _lib = L
@@ -181,6 +189,19 @@ def set_wait_limit_ns(ns: int) -> None:
 
 def selftest_timeout(stream=None) -> None:
     _check(lib().vswin_selftest_timeout(_stream_handle(stream)))
+
+
+def profile_enable(on: bool) -> None:
+    _check(lib().vswin_profile_enable(1 if on else 0))
+
+
+def profile_collect():
+    """{kind: (total ms, launches)} for the launches recorded since the last collect."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_ulonglong * n)()
+    _check(lib().vswin_profile_collect(ms, cnt, n))
+    return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
 
 
 def version() -> int:
