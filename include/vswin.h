@@ -105,6 +105,35 @@ int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int 
                             const void* bias_table, void* out_host, void* stream);
 
 /*
+ * bf16 layer forward that allocates nothing. No passage of the method's pages
+ * corresponds to this: it is an interface for callers that cannot allocate
+ * device memory while they run the layer -- hosts that must stay inside
+ * memory they reserved beforehand, code that must not risk the device-wide
+ * synchronisation an allocation can cause, or processes whose device memory
+ * belongs to another allocator. Arguments, layouts, requirements and results
+ * are those of vswin_wmsa_forward; only the scratch differs.
+ *   * Scratch is one statically sized 32 MiB device array inside this library
+ *     (every GPU that loads the library holds it until the process exits).
+ *     Windows pass through it in equal chunks, so any batch size works; a
+ *     layer whose single window needs more than 32 MiB of scratch is refused
+ *     with VSWIN_ERR_UNSUPPORTED and a message giving both sizes (the layers
+ *     in this repository need 0.3 MB to 3.3 MB per window).
+ *   * No cudaMalloc / cudaMallocAsync / cudaFree or other allocating call is
+ *     made. The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   * All calls share the one array and it keeps the last call's contents.
+ *     Calls whose kernels overlap on the GPU (different streams, or different
+ *     host threads without ordering) race on it and give wrong results: order
+ *     them on one stream or synchronise between them. Nothing in the array
+ *     needs to start at zero.
+ */
+int vswin_wmsa_forward_noalloc(const void* x, int B, int T, int H, int W, int C, int heads,
+                               const int* window, const int* shift,
+                               const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                               const void* bias_table, void* out, void* stream);
+
+/*
  * Index maps of the layer, written to caller-allocated device int32 buffers
  * (any of them may be NULL to skip it):
  *   win_src [B*nW*N]  flat source token b*T*H*W + (t*H + h)*W + w of each

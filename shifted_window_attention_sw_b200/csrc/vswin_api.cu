@@ -230,6 +230,44 @@ void prof_end(int kind, cudaStream_t st) {
 
 }  // namespace vswin
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for vswin_wmsa_forward_noalloc.
+//
+// Some callers cannot allocate device memory on the call path: a plugin or
+// real-time host that must stay within memory it reserved up front, code that
+// may not synchronise the device (cudaMalloc can), or a process whose
+// allocator is owned by another framework. For them the bf16 layer can run
+// out of this statically sized array instead of stream-ordered scratch.
+// Every GPU that loads this library holds the array until the process exits.
+static constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace vswin {
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name only stands in for the symbol; its address on a device comes
+// from cudaGetSymbolAddress, looked up once per device with that device
+// current (the first call on each device does this).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VSWIN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return VSWIN_OK;
+}
+}  // namespace
+}  // namespace vswin
+
 using namespace vswin;
 
 extern "C" {
@@ -400,6 +438,44 @@ int vswin_selftest_timeout(void* stream) {
   if (st != VSWIN_OK) return st;
   cudaError_t e = launch_selftest_timeout(ctx, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "self-test launch");
+  return VSWIN_OK;
+}
+
+int vswin_wmsa_forward_noalloc(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                               const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
+                               const void* bproj, const void* bias_table, void* out, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  st = check_layer_ptrs(x, Wqkv, bqkv, Wproj, bproj, bias_table, out, g, 2, 16);
+  if (st != VSWIN_OK) return st;
+  if (g.d != 32) return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path needs head width 32 (C/heads = %d)", g.d);
+  if (!bf16_window_supported(g))
+    return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path has no kernel for window (%d,%d,%d)", g.win[0], g.win[1],
+                g.win[2]);
+  const size_t per_window = bf16_scratch_bytes(g, 1);
+  if (per_window > kNoAllocScratchBytes)
+    return fail(VSWIN_ERR_UNSUPPORTED,
+                "one window of this layer needs %zu bytes of scratch; the no-allocation entry point has %zu",
+                per_window, kNoAllocScratchBytes);
+  KernelCtx ctx;
+  st = make_ctx(&ctx);
+  if (st != VSWIN_OK) return st;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != VSWIN_OK) return st;
+  // Windows go through the fixed array in equal chunks. Nothing in it needs to
+  // start at zero: every byte a kernel uses is first written by this call.
+  long long cap = (long long)(kNoAllocScratchBytes / per_window);
+  if (cap > g.windows) cap = g.windows;
+  const long long nchunks = (g.windows + cap - 1) / cap;
+  const long long per_chunk = (g.windows + nchunks - 1) / nchunks;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (long long w0 = 0; w0 < g.windows; w0 += per_chunk) {
+    const long long n = (g.windows - w0) < per_chunk ? (g.windows - w0) : per_chunk;
+    cudaError_t e = launch_bf16_chunk(g, ctx, x, Wqkv, bqkv, Wproj, bproj, bias_table, out, scratch, w0, n, s);
+    if (e != cudaSuccess) return fail_cuda(e, "bf16 kernel launch (no-allocation entry)");
+  }
   return VSWIN_OK;
 }
 

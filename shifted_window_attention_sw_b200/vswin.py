@@ -32,6 +32,7 @@ EXPORTS = (
     "vswin_version",
     "vswin_profile_enable",
     "vswin_profile_collect",
+    "vswin_wmsa_forward_noalloc",
 )
 
 KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other")
@@ -58,7 +59,8 @@ def lib():
                                  "`python -m shifted_window_attention_sw_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         layer = [_P, _I, _I, _I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P, _P, _P, _P]
-        for name in ("vswin_wmsa_forward", "vswin_wmsa_forward_f32", "vswin_wmsa_forward_host"):
+        for name in ("vswin_wmsa_forward", "vswin_wmsa_forward_f32", "vswin_wmsa_forward_host",
+                     "vswin_wmsa_forward_noalloc"):
             fn = getattr(L, name)
             fn.argtypes = layer
             fn.restype = _I
@@ -134,6 +136,17 @@ def wmsa_forward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=N
     _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.bfloat16)
     return _layer_call(lib().vswin_wmsa_forward, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out,
                        stream)
+
+
+def wmsa_forward_noalloc(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):
+    """bf16 layer forward that allocates no device memory: the library's fixed
+    32 MiB scratch array is used instead (see include/vswin.h). ``out`` should be
+    passed in by callers that cannot allocate; if it is None a tensor is created."""
+    if out is None:
+        out = torch.empty_like(x)
+    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.bfloat16)
+    return _layer_call(lib().vswin_wmsa_forward_noalloc, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads,
+                       out, stream)
 
 
 def wmsa_forward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):
