@@ -75,64 +75,52 @@ def step_work(wl):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+    """Samples SM clock and throttle reasons DURING the timed region with nvidia-smi in a
+    separate process (-lms period), so nothing runs inside the benchmark process."""
 
-    REASONS = {
-        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
-        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
-        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
-        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
-        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
-        "gpu_idle": "nvmlClocksEventReasonGpuIdle",
-    }
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, device, period_s=0.01):
-        self.samples = []
-        self.reasons = set()
-        self.max_mhz = None
-        self.period = period_s
-        self._stop = threading.Event()
-        self._thread = None
-        self.nv = None
-        self.handle = None
-        try:
-            import pynvml as nv
-
-            nv.nvmlInit()
-            props = torch.cuda.get_device_properties(device)
-            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-            self.handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
-            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
-            self.nv = nv
-        except Exception as e:  # noqa: BLE001 -- clocks are reported as unavailable
-            self.error = repr(e)
-
-    def _run(self):
-        nv = self.nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
-                for name, const in self.REASONS.items():
-                    if bits & getattr(nv, const, 0):
-                        self.reasons.add(name)
-            except Exception:  # noqa: BLE001
-                pass
-            time.sleep(self.period)
+    def __init__(self, device, period_ms=50):
+        self.proc = None
+        self.period_ms = period_ms
+        props = torch.cuda.get_device_properties(device)
+        self.bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
 
     def start(self):
-        if self.nv is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
+        import subprocess
+
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.bus}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={self.period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)  # let the first sample land before the timed region starts
+        except OSError:
+            self.proc = None
 
     def stop(self):
-        if self._thread is not None:
-            self._stop.set()
-            self._thread.join()
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 6:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, f[2:6]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
 
 
 # ------------------------------------------------------------------ CPU oracle sample
@@ -307,6 +295,7 @@ def run_gpu(args):
         raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_s = sum(step_ms) / 1e3
+    step_stats = {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}
     work = step_work(wl)
     max_s, tokens, nranks = replicas.combine(total_s, work["tokens"] * args.steps, device)
     value = tokens / max_s
@@ -378,6 +367,7 @@ def run_gpu(args):
         "step_roofline_us": 1e6 * max(step_flops_time, work["bytes"] / (float(peaks["hbm_gbs"]) * 1e9)),
         "roofline": roofline,
         "kernel_ms_per_step": kernel_ms,
+        "step_ms": step_stats,
         "gpu_launches": int(launches),
         "clocks": clocks,
     }

@@ -38,6 +38,32 @@ constexpr int kBStageMaxBytes = kBK * kMaxBN * 2;  // 16 KB
 
 enum { kQKV = 0, kPROJ = 1 };
 
+// Where q, k and v of one (window, head) live in the chunk scratch: a q slab of
+// `qrows` rows (slot order) then k and v slabs of `kvrows` rows, each row 32
+// bf16 in the no-swizzle operand layout ((row/8)*512 + (col/8)*128 +
+// (row%8)*16 bytes). For (P,7,7) windows the keys are stored as P*7 rows of 8:
+// slot n goes to row (n/7)*8 + n%7, the eighth row of each group is padding,
+// so that the softmax walks keys in 8-column groups of one (pt, ph) line.
+struct SlabLayout {
+  int qrows, kvrows, kv8;
+  __host__ __device__ int kv_row(int n) const { return kv8 ? (n / 7) * 8 + n % 7 : n; }
+  __host__ __device__ size_t head_elems() const { return (size_t)(qrows + 2 * kvrows) * 32; }
+};
+
+__host__ __device__ inline bool window_is_p77(const Geom& g) {
+  const int P = g.win[0];
+  return g.win[1] == 7 && g.win[2] == 7 && (P == 1 || P == 2 || P == 4 || P == 8);
+}
+
+__host__ __device__ inline SlabLayout slab_layout(const Geom& g) {
+  SlabLayout L;
+  L.qrows = g.Npad;
+  L.kv8 = window_is_p77(g) ? 1 : 0;
+  // 8-wide key lines, rounded up to a multiple of 32 columns (4 lines)
+  L.kvrows = L.kv8 ? ((g.win[0] * 7 * 8 + 31) / 32) * 32 : g.Npad;
+  return L;
+}
+
 struct GemmArgs {
   Geom g;
   KernelCtx ctx;
@@ -49,6 +75,7 @@ struct GemmArgs {
   long long rows;             // nwin * N
   int K, Ntot, BN;
   float qscale;
+  SlabLayout slab;
 };
 
 __host__ __device__ constexpr int gemm_smem_bytes() {
@@ -218,9 +245,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
                         pack_bf16x2(v[4] * sc, v[5] * sc), pack_bf16x2(v[6] * sc, v[7] * sc));
         w1 = make_uint4(pack_bf16x2(v[8] * sc, v[9] * sc), pack_bf16x2(v[10] * sc, v[11] * sc),
                         pack_bf16x2(v[12] * sc, v[13] * sc), pack_bf16x2(v[14] * sc, v[15] * sc));
-        __nv_bfloat16* slab =
-            a.dst + (((size_t)slab_win * g.heads + hh) * 3 + which) * (size_t)g.Npad * 32;
-        __nv_bfloat16* e = slab + (slot >> 3) * 256 + (jj >> 3) * 64 + (slot & 7) * 8;
+        const SlabLayout& L = a.slab;
+        __nv_bfloat16* slab = a.dst + ((size_t)slab_win * g.heads + hh) * L.head_elems() +
+                              (which == 0 ? 0 : ((size_t)L.qrows + (size_t)(which - 1) * L.kvrows) * 32);
+        const int row = which == 0 ? slot : L.kv_row(slot);
+        __nv_bfloat16* e = slab + (row >> 3) * 256 + (jj >> 3) * 64 + (row & 7) * 8;
         *reinterpret_cast<uint4*>(e) = w0;
         *reinterpret_cast<uint4*>(e + 64) = w1;
       } else if (dst_row >= 0) {
@@ -275,7 +304,8 @@ struct Win {
 struct AttnArgs {
   Geom g;
   KernelCtx ctx;
-  const __nv_bfloat16* qkv;    // slabs [nwin][heads][3][NPAD*32]
+  SlabLayout slab;
+  const __nv_bfloat16* qkv;    // per (window, head): q | k | v slabs
   const __nv_bfloat16* table;  // [rows][heads]
   __nv_bfloat16* o;            // [nwin][N][C]
   long long win0, nwin;
@@ -402,7 +432,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attention_kernel(AttnArgs a) 
     const long long wl = item % a.nwin;
     const long long win = a.win0 + wl;
     if (tid == 0) {
-      const __nv_bfloat16* base = a.qkv + ((size_t)wl * g.heads + h) * 3 * (size_t)Wn::NPAD * kD;
+      const __nv_bfloat16* base = a.qkv + ((size_t)wl * g.heads + h) * a.slab.head_elems();
       mbar_arrive_expect_tx(bar_ld, 3 * slab_bytes);
       bulk_g2s(sQ, base, slab_bytes, bar_ld);
       bulk_g2s(sK, base + (size_t)Wn::NPAD * kD, slab_bytes, bar_ld);
@@ -564,6 +594,374 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ============================================================================ attention, (P,7,7) windows
+//
+// 256 threads: warps w and w+4 share TMEM lane quarter w%4 (query rows
+// 32*(w%4) .. +31 of the tile) and split each key block into two halves of
+// 8-column key lines. Per block, pass 1 takes the row max of the raw scores
+// (exchanged between the two halves); the block max used for the exponentials
+// is that plus the head's largest bias, an upper bound of the true maximum of
+// score + bias that exceeds it by at most the bias range, so nothing overflows
+// and nothing that matters underflows. Pass 2 streams score + bias -> exp2 ->
+// row sum -> bf16 P. Each half writes its P into its own S columns (already
+// read), and O = P V runs as two K ranges, one per half.
+constexpr int kAttn7Threads = 256;
+
+template <int P_>
+struct W7 {
+  static constexpr int P = P_;
+  static constexpr int N = P * 49;
+  static constexpr int QSLAB = (N + 15) / 16 * 16;             // q slab rows
+  static constexpr int KLINES = P * 7;                         // key lines of 7 real keys
+  static constexpr int KCOLS = (KLINES * 8 + 31) / 32 * 32;    // k/v slab rows (padded key columns)
+  static constexpr int LINES = KCOLS / 8;                      // multiple of 4
+  static constexpr int NBLK = (LINES + 19) / 20;
+  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 3) / 4 * 4;  // lines per block but the last
+  static constexpr int LAST = LINES - (NBLK - 1) * BL;
+  static constexpr int TABLE = (2 * P - 1) * 169;
+  static constexpr int QTILES = (N + 127) / 128;
+  static constexpr int QROWS = QTILES * 128 > QSLAB ? QTILES * 128 : QSLAB;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QROWS * kSlabRowBytes;
+  static constexpr int OFF_V = OFF_K + KCOLS * kSlabRowBytes;
+  static constexpr int OFF_T = OFF_V + KCOLS * kSlabRowBytes;
+  static constexpr int OFF_X = OFF_T + (TABLE * 4 + 15) / 16 * 16;  // exchange: max[2][128], sum[2][3][128]
+  static constexpr int OFF_BAR = OFF_X + (2 * 128 + 6 * 128) * 4;
+  static constexpr int SMEM = (OFF_BAR + 64) < 81920 ? 81920 : (OFF_BAR + 64);
+  static_assert(NBLK <= 3 && BL <= 20 && LAST > 0 && LAST % 4 == 0, "key blocks must fit 160 TMEM columns");
+  static_assert(SMEM <= 110 * 1024, "two CTAs per SM");
+};
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+template <class Wn>
+__device__ __forceinline__ int w7_block_lines(int b) {
+  return b < Wn::NBLK - 1 ? Wn::BL : Wn::LAST;
+}
+
+// Pass 1 over this thread's lines of one block: max of the allowed raw scores.
+template <class Wn, bool MASKED>
+__device__ __forceinline__ float w7_pass1(uint32_t tcol, int l0, int l1, uint32_t okt, uint32_t okh,
+                                          uint32_t okw) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll 1
+  for (int l = l0; l < l1; l += 2) {
+    uint32_t u[16];
+    tmem_ld16(tcol + (l - l0) * 8, u);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int line = l + c;
+      if (line < Wn::KLINES) {
+        const int pt = line / 7, ph = line - 7 * (line / 7);
+        const uint32_t lm = ((okt >> pt) & (okh >> ph) & 1u) ? okw : 0u;  // allowed pw of this line
+#pragma unroll
+        for (int pw = 0; pw < 7; ++pw) {
+          const float v = __uint_as_float(u[c * 8 + pw]);
+          const bool ok = !MASKED || ((lm >> pw) & 1u);
+          if (pw & 1)
+            m1 = ok ? fmaxf(m1, v) : m1;
+          else
+            m0 = ok ? fmaxf(m0, v) : m0;
+        }
+      }
+    }
+  }
+  return fmaxf(m0, m1);
+}
+
+// Pass 2: p = exp2(score + bias - mm) on allowed keys (0 elsewhere), row sum,
+// bf16 P written to TMEM at this half's P columns.
+template <class Wn, bool MASKED>
+__device__ __forceinline__ float w7_pass2(uint32_t tcol, int l0, int l1, const float* tb_row, float mm,
+                                          uint32_t okt, uint32_t okh, uint32_t okw) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll 1
+  for (int l = l0; l < l1; l += 2) {
+    uint32_t u[16];
+    tmem_ld16(tcol + (l - l0) * 8, u);
+    tmem_wait_ld();
+    uint32_t pk[8];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int line = l + c;
+      float p[8];
+      if (line < Wn::KLINES) {
+        const int pt = line / 7, ph = line - 7 * (line / 7);
+        const uint32_t lm = ((okt >> pt) & (okh >> ph) & 1u) ? okw : 0u;
+        const float* tbr = tb_row - (pt * 169 + ph * 13);
+#pragma unroll
+        for (int pw = 0; pw < 7; ++pw) {
+          const bool ok = !MASKED || ((lm >> pw) & 1u);
+          const float t = __uint_as_float(u[c * 8 + pw]) + tbr[-pw] - mm;
+          p[pw] = ok ? ex2_approx(t) : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int pw = 0; pw < 7; ++pw) p[pw] = 0.f;
+      }
+      p[7] = 0.f;
+      s0 += (p[0] + p[2]) + (p[4] + p[6]);
+      s1 += (p[1] + p[3]) + p[5];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pk[c * 4 + k] = pack_bf16x2(p[2 * k], p[2 * k + 1]);
+    }
+    // P of lines l, l+1 -> 8 columns at 4 per line from the half's first column
+    tmem_st8(tcol + (l - l0) * 4, pk);
+  }
+  return s0 + s1;
+}
+
+template <class Wn>
+__global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sQ = smem + Wn::OFF_Q;
+  uint8_t* sK = smem + Wn::OFF_K;
+  uint8_t* sV = smem + Wn::OFF_V;
+  float* sT = reinterpret_cast<float*>(smem + Wn::OFF_T);
+  float* xmax = reinterpret_cast<float*>(smem + Wn::OFF_X);  // [2][128]
+  float* xsum = xmax + 2 * 128;                              // [2][3][128]
+  uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + Wn::OFF_BAR);
+  uint64_t* bar_s = bar_ld + 1;
+  uint64_t* bar_o = bar_ld + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_ld + 3);
+  __shared__ int s_abort;
+  __shared__ float s_part[kAttn7Threads / 32];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int rt = quarter * 32 + lane;  // row within the query tile = TMEM lane
+  const Geom& g = a.g;
+  const long long nitems = a.nwin * g.heads;
+  const uint32_t qbytes = Wn::QSLAB * kSlabRowBytes, kvbytes = Wn::KCOLS * kSlabRowBytes;
+
+  if (tid == 0) {
+    mbar_init(bar_ld, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  for (int k = Wn::QSLAB * kSlabRowBytes / 16 + tid; k < Wn::QROWS * kSlabRowBytes / 16; k += kAttn7Threads)
+    reinterpret_cast<uint4*>(sQ)[k] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+  const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
+
+  uint32_t ph_ld = 0, ph_s = 0, ph_o = 0;
+  int cur_head = -1;
+  float bmax = 0.f;
+
+#pragma unroll 1
+  for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int h = (int)(item / a.nwin);
+    const long long wl = item % a.nwin;
+    const long long win = a.win0 + wl;
+    if (tid == 0) {
+      const __nv_bfloat16* base = a.qkv + ((size_t)wl * g.heads + h) * a.slab.head_elems();
+      mbar_arrive_expect_tx(bar_ld, qbytes + 2 * kvbytes);
+      bulk_g2s(sQ, base, qbytes, bar_ld);
+      bulk_g2s(sK, base + (size_t)Wn::QSLAB * kD, kvbytes, bar_ld);
+      bulk_g2s(sV, base + (size_t)(Wn::QSLAB + Wn::KCOLS) * kD, kvbytes, bar_ld);
+    }
+    if (h != cur_head) {
+      float mx = -INFINITY;
+      for (int k = tid; k < Wn::TABLE; k += kAttn7Threads) {
+        const float v = __bfloat162float(a.table[(size_t)k * g.heads + h]) * kLog2e;
+        sT[k] = v;
+        mx = fmaxf(mx, v);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      if (lane == 0) s_part[warp] = mx;
+      cur_head = h;
+    }
+    if (!mbar_wait(bar_ld, ph_ld, a.ctx.err, kErrWaitLoad, a.ctx.wait_limit)) s_abort = 1;
+    ph_ld ^= 1;
+    // Padding rows of the v slab (8th key of each line, whole padding lines) must be
+    // finite for O = P V: zero them (four 16-byte pieces per row).
+    {
+      constexpr int ndummy = Wn::KLINES + (Wn::LINES - Wn::KLINES) * 8;
+      for (int k = tid; k < ndummy * 4; k += kAttn7Threads) {
+        const int d = k >> 2, chunk = k & 3;
+        const int n = d < Wn::KLINES ? d * 8 + 7 : Wn::KLINES * 8 + (d - Wn::KLINES);
+        *reinterpret_cast<uint4*>(sV + (n >> 3) * 512 + chunk * 128 + (n & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (s_abort) break;
+    {
+      float mx = s_part[0];
+#pragma unroll
+      for (int k = 1; k < kAttn7Threads / 32; ++k) mx = fmaxf(mx, s_part[k]);
+      bmax = mx;
+    }
+    const int split = window_split_bits(g, (int)(win % g.nW));
+
+#pragma unroll 1
+    for (int qt = 0; qt < Wn::QTILES; ++qt) {
+      const int i = qt * 128 + rt;
+      const bool active = qt * 128 + quarter * 32 < Wn::N;
+      const int ie = i < Wn::N ? i : Wn::N - 1;
+      const int pt_i = ie / 49, ph_i = (ie / 7) % 7, pw_i = ie % 7;
+      const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
+      uint32_t okt = 0xFFFFFFFFu, okh = 0xFFFFFFFFu, okw = 0x7Fu;
+      {
+        const int cut_t = Wn::P - g.sh[0], cut_h = 7 - g.sh[1], cut_w = 7 - g.sh[2];
+        const bool rt_ = pt_i >= cut_t, rh_ = ph_i >= cut_h, rw_ = pw_i >= cut_w;
+        if (split & 1) {
+          okt = 0;
+          for (int k = 0; k < Wn::P; ++k) okt |= (uint32_t)((k >= cut_t) == rt_) << k;
+        }
+        if (split & 2) {
+          okh = 0;
+          for (int k = 0; k < 7; ++k) okh |= (uint32_t)((k >= cut_h) == rh_) << k;
+        }
+        if (split & 4) {
+          okw = 0;
+          for (int k = 0; k < 7; ++k) okw |= (uint32_t)((k >= cut_w) == rw_) << k;
+        }
+      }
+      float mrow[3] = {-INFINITY, -INFINITY, -INFINITY}, lrow[3] = {0.f, 0.f, 0.f};
+
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          umma_ss(tmem, smem_desc(qaddr + qt * 8192 + ks * 256, 128, 512), smem_desc(kaddr + ks * 256, 128, 512),
+                  idesc_bf16(128, w7_block_lines<Wn>(0) * 8, 0, 0), ks);
+        umma_commit(bar_s);
+      }
+#pragma unroll 1
+      for (int b = 0; b < Wn::NBLK; ++b) {
+        const int nl = w7_block_lines<Wn>(b);
+        const int l0 = b * Wn::BL + half * (nl / 2), l1 = l0 + nl / 2;
+        const uint32_t tcol = trow + half * (nl / 2) * 8;
+        if (!mbar_wait(bar_s, ph_s, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
+        ph_s ^= 1;
+        __syncthreads();
+        tc_fence_after();
+        if (active && !s_abort) {
+          const float mp = split ? w7_pass1<Wn, true>(tcol, l0, l1, okt, okh, okw)
+                                 : w7_pass1<Wn, false>(tcol, l0, l1, okt, okh, okw);
+          xmax[half * 128 + rt] = mp;
+          named_bar(1 + quarter, 64);
+          const float ms = fmaxf(xmax[rt], xmax[128 + rt]);
+          const float mb = ms == -INFINITY ? -INFINITY : ms + bmax;
+          const float mm = mb == -INFINITY ? 0.f : mb;
+          lrow[b] = split ? w7_pass2<Wn, true>(tcol, l0, l1, tb_row, mm, okt, okh, okw)
+                          : w7_pass2<Wn, false>(tcol, l0, l1, tb_row, mm, okt, okh, okw);
+          mrow[b] = mb;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && !s_abort) {
+          tc_fence_after();
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int key0 = (b * Wn::BL + hf * (nl / 2)) * 8;
+            for (int ks = 0; ks < nl / 4; ++ks)
+              umma_ts(tmem + kOCol + 32 * b, tmem + hf * (nl / 2) * 8 + 8 * ks,
+                      smem_desc(vaddr + ((key0 + 16 * ks) >> 3) * 512, 512, 128), idesc_bf16(128, kD, 0, 1),
+                      (hf | ks) != 0);
+          }
+          if (b + 1 < Wn::NBLK) {
+            const int nkey0 = (b + 1) * Wn::BL * 8;
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+              umma_ss(tmem, smem_desc(qaddr + qt * 8192 + ks * 256, 128, 512),
+                      smem_desc(kaddr + (nkey0 >> 3) * 512 + ks * 256, 128, 512),
+                      idesc_bf16(128, w7_block_lines<Wn>(b + 1) * 8, 0, 0), ks);
+            umma_commit(bar_s);
+          } else {
+            umma_commit(bar_o);
+          }
+        }
+        if (s_abort) break;
+      }
+      if (s_abort) break;
+      if (!mbar_wait(bar_o, ph_o, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
+      ph_o ^= 1;
+      __syncthreads();
+      tc_fence_after();
+      if (active && !s_abort) {
+#pragma unroll
+        for (int b = 0; b < Wn::NBLK; ++b) xsum[(half * 3 + b) * 128 + rt] = lrow[b];
+        named_bar(1 + quarter, 64);
+        float M = mrow[0];
+#pragma unroll
+        for (int b = 1; b < Wn::NBLK; ++b) M = fmaxf(M, mrow[b]);
+        float alpha[3], L = 0.f;
+#pragma unroll
+        for (int b = 0; b < Wn::NBLK; ++b) {
+          alpha[b] = mrow[b] == -INFINITY ? 0.f : ex2_approx(mrow[b] - M);
+          L += alpha[b] * (xsum[b * 128 + rt] + xsum[(3 + b) * 128 + rt]);
+        }
+        const float inv = 1.0f / L;
+        float o[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) o[k] = 0.f;
+#pragma unroll
+        for (int b = 0; b < Wn::NBLK; ++b) {
+          uint32_t u[16];
+          tmem_ld16(trow + kOCol + 32 * b + 16 * half, u);
+          tmem_wait_ld();
+          const float f = alpha[b] * inv;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[k] = fmaf(__uint_as_float(u[k]), f, o[k]);
+        }
+        if (i < Wn::N) {
+          __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD + 16 * half;
+          reinterpret_cast<uint4*>(dst)[0] =
+              make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                         pack_bf16x2(o[6], o[7]));
+          reinterpret_cast<uint4*>(dst)[1] =
+              make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
+                         pack_bf16x2(o[14], o[15]));
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (s_abort) break;
+    }
+    if (s_abort) break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <class Wn>
+cudaError_t launch_attention7(const AttnArgs& a, cudaStream_t st) {
+  if (a.slab.qrows != Wn::QSLAB || a.slab.kvrows != Wn::KCOLS || !a.slab.kv8) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t e =
+      cudaFuncSetAttribute(attention7_kernel<Wn>, cudaFuncAttributeMaxDynamicSharedMemorySize, Wn::SMEM);
+  if (e != cudaSuccess) return e;
+  const long long items = a.nwin * a.g.heads;
+  long long grid = 2LL * sms;
+  if (grid > items) grid = items;
+  prof_begin(kKindAttn, st);
+  attention7_kernel<Wn><<<(unsigned)grid, kAttn7Threads, Wn::SMEM, st>>>(a);
+  prof_end(kKindAttn, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
 int pick_bn(int n) {
   if (n <= kMaxBN && n % 16 == 0) return n;
   for (int bn = kMaxBN; bn >= 16; bn -= 16)
@@ -594,7 +992,7 @@ bool bf16_window_supported(const Geom& g) {
 }
 
 size_t bf16_scratch_bytes(const Geom& g, long long nwin) {
-  const size_t qkv = (size_t)nwin * g.heads * 3 * g.Npad * kD * 2;
+  const size_t qkv = (size_t)nwin * g.heads * slab_layout(g).head_elems() * 2;
   const size_t o = (size_t)nwin * g.N * g.C * 2;
   return qkv + o;
 }
@@ -603,7 +1001,8 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
                               const void* bqkv, const void* Wproj, const void* bproj, const void* table,
                               void* out, void* scratch, long long win0, long long nwin, cudaStream_t st) {
   __nv_bfloat16* qkv = static_cast<__nv_bfloat16*>(scratch);
-  __nv_bfloat16* o = qkv + (size_t)nwin * g.heads * 3 * g.Npad * kD;
+  const SlabLayout L = slab_layout(g);
+  __nv_bfloat16* o = qkv + (size_t)nwin * g.heads * L.head_elems();
 
   GemmArgs ga{};
   ga.g = g;
@@ -618,6 +1017,7 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   ga.Ntot = 3 * g.C;
   ga.BN = pick_bn(3 * g.C);
   ga.qscale = kLog2e / sqrtf((float)kD);
+  ga.slab = L;
   cudaError_t e = launch_gemm<kQKV>(ga, st);
   if (e != cudaSuccess) return e;
 
@@ -629,11 +1029,12 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   aa.o = o;
   aa.win0 = win0;
   aa.nwin = nwin;
+  aa.slab = L;
   const int P = g.win[0], MH = g.win[1], MW = g.win[2];
-  if (P == 8 && MH == 7 && MW == 7) e = launch_attention<Win<8, 7, 7>>(aa, st);
-  else if (P == 4 && MH == 7 && MW == 7) e = launch_attention<Win<4, 7, 7>>(aa, st);
-  else if (P == 2 && MH == 7 && MW == 7) e = launch_attention<Win<2, 7, 7>>(aa, st);
-  else if (P == 1 && MH == 7 && MW == 7) e = launch_attention<Win<1, 7, 7>>(aa, st);
+  if (P == 8 && MH == 7 && MW == 7) e = launch_attention7<W7<8>>(aa, st);
+  else if (P == 4 && MH == 7 && MW == 7) e = launch_attention7<W7<4>>(aa, st);
+  else if (P == 2 && MH == 7 && MW == 7) e = launch_attention7<W7<2>>(aa, st);
+  else if (P == 1 && MH == 7 && MW == 7) e = launch_attention7<W7<1>>(aa, st);
   else if (P == 4 && MH == 4 && MW == 4) e = launch_attention<Win<4, 4, 4>>(aa, st);
   else if (P == 2 && MH == 2 && MW == 2) e = launch_attention<Win<2, 2, 2>>(aa, st);
   else if (P == 1 && MH == 1 && MW == 1) e = launch_attention<Win<1, 1, 1>>(aa, st);
