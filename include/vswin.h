@@ -73,8 +73,8 @@ typedef enum {
  * (1,1,1); otherwise VSWIN_ERR_UNSUPPORTED. Pointers must be 16-byte aligned
  * and x must not overlap out.
  * Scratch: stream-ordered cudaMallocAsync / cudaFreeAsync on `stream`
- * (about 135 KB per window of 392 slots at C = 96, processed in chunks of at
- * most 64 MB).
+ * (about 324 KB per window of 392 slots at C = 96; windows are processed in
+ * chunks of at most 1 GiB of scratch, i.e. one chunk for the layers here).
  */
 int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int heads,
                        const int* window, const int* shift,

@@ -135,10 +135,14 @@ int check_layer_ptrs(const void* x, const void* Wqkv, const void* bqkv, const vo
   return VSWIN_OK;
 }
 
+// Windows per launch chunk. One chunk per layer is fastest on B200 (more
+// (window, head) items per persistent CTA, less wave quantisation) even though
+// the scratch then spills from L2 to HBM; the budget (default 1 GiB,
+// VSWIN_CHUNK_MB overrides) only bounds memory for very large layers.
 long long chunk_windows(const Geom& g) {
   static long long budget = [] {
     const char* s = std::getenv("VSWIN_CHUNK_MB");
-    long long mb = s ? std::atoll(s) : 64;
+    long long mb = s ? std::atoll(s) : 1024;
     if (mb < 1) mb = 1;
     return mb << 20;
   }();
