@@ -72,9 +72,11 @@ typedef enum {
  * compiled shapes (8,7,7), (4,7,7), (2,7,7), (1,7,7), (4,4,4), (2,2,2),
  * (1,1,1); otherwise VSWIN_ERR_UNSUPPORTED. Pointers must be 16-byte aligned
  * and x must not overlap out.
- * Scratch: stream-ordered cudaMallocAsync / cudaFreeAsync on `stream`
- * (about 324 KB per window of 392 slots at C = 96; windows are processed in
- * chunks of at most 1 GiB of scratch, i.e. one chunk for the layers here).
+ * Scratch: stream-ordered allocation on `stream` from a memory pool the
+ * library creates per device and keeps (freed scratch is reused by the next
+ * call; the pool grows to the largest call's need and is held until exit):
+ * about 324 KB per window of 392 slots at C = 96, in chunks of at most 1 GiB
+ * (one chunk for the layers here).
  */
 int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int heads,
                        const int* window, const int* shift,
@@ -84,7 +86,7 @@ int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int hea
 /*
  * fp32 layer forward (plain FP32 FMA arithmetic, no tensor cores): every
  * tensor is float. Any d; N <= 4096. Pointers 4-byte aligned; x must not
- * overlap out. Scratch: cudaMallocAsync on `stream`.
+ * overlap out. Scratch: stream-ordered, from the library's pool (see above).
  */
 int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads,
                            const int* window, const int* shift,
@@ -97,7 +99,7 @@ int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int
  * synchronises `stream`. Weights, biases and table are device pointers (they
  * stay resident between calls). Page-locked host buffers give asynchronous
  * copies; pageable ones work but are slower. Device buffers for x and out
- * come from cudaMallocAsync on `stream`.
+ * come from the library's stream-ordered pool (see vswin_wmsa_forward).
  */
 int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads,
                             const int* window, const int* shift,

@@ -76,6 +76,7 @@ struct GemmArgs {
   int K, Ntot, BN;
   float qscale;
   SlabLayout slab;
+  const int* rowsrc;          // [rows] source token of each chunk row (-1 = padding), or null
 };
 
 __host__ __device__ constexpr int gemm_smem_bytes() {
@@ -87,6 +88,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -266,6 +271,238 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, tcols);
+}
+
+// ============================================================================ persistent GEMM
+//
+// Warp-specialised persistent version of the two GEMMs for layers whose
+// per-CTA weight slice (K x BN bf16) fits in shared memory: warp 0 gathers
+// 128-row A tiles with cp.async (two stages), warp 1 issues tcgen05.mma into
+// two TMEM accumulators (BN columns each), warps 2..9 drain an accumulator
+// (two warps per TMEM lane quarter, half of the columns each) while the next
+// tile is multiplied. CTA c keeps N-tile c % NT and walks the M-tiles
+// c / NT, c / NT + G / NT, ... (G = grid size, a multiple of NT).
+constexpr int kWsProdWarps = 4;
+constexpr int kWsEpiWarps = 8;
+constexpr int kWsMmaWarp = kWsProdWarps;
+constexpr int kWsEpi0 = kWsProdWarps + 1;
+constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
+constexpr int kWsMaxBBytes = 96 * 1024;
+
+__host__ __device__ inline int ws_a_bytes(int K) { return kBM * K * 2; }
+__host__ __device__ inline int ws_smem_bytes(int K, int BN) { return K * BN * 2 + 2 * ws_a_bytes(K) + BN * 4 + 256; }
+
+// Row sources of one chunk: token index (x row) of each window slot, -1 for
+// padding. Consumed by the QKV gather and the projection scatter.
+__global__ void row_source_kernel(Geom g, long long win0, long long rows, int* __restrict__ out) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < rows; r += stride) {
+    const long long gr = win0 * g.N + r;
+    out[r] = (int)slot_source(g, gr / g.N, (int)(gr % g.N));
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int K = a.K, BN = a.BN;
+  uint8_t* sB = smem;                                     // K x BN, MN-major operand layout
+  uint8_t* sA = sB + K * BN * 2;                          // 2 stages of 128 x K, K-major
+  float* sBias = reinterpret_cast<float*>(sA + 2 * ws_a_bytes(K));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBias + BN);
+  uint64_t* b_full = bars;          // B resident
+  uint64_t* a_full = bars + 1;      // [2]
+  uint64_t* a_free = bars + 3;      // [2]
+  uint64_t* acc_full = bars + 5;    // [2]
+  uint64_t* acc_free = bars + 7;    // [2]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 9);
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Geom& g = a.g;
+  const int NT = a.Ntot / BN;
+  const int nt = blockIdx.x % NT;
+  const int n0 = nt * BN;
+  const long long mtiles = (a.rows + kBM - 1) / kBM;
+  const long long m_first = blockIdx.x / NT, m_step = gridDim.x / NT;
+  const uint64_t lim = a.ctx.wait_limit;
+  const uint32_t lboB = (uint32_t)(BN / 8) * 128u;  // B: K-group stride
+  const uint32_t sboA = (uint32_t)(K / 8) * 128u;   // A: 8-row group stride
+  const uint32_t tcols = BN <= 64 ? 128 : BN <= 128 ? 256 : 512;
+  constexpr int kProdThreads = kWsProdWarps * 32;
+
+  if (tid == 0) {
+    mbar_init(b_full, kProdThreads);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&a_full[k], kProdThreads);
+      mbar_init(&a_free[k], 1);
+      mbar_init(&acc_full[k], 1);
+      mbar_init(&acc_free[k], kWsEpiWarps);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  for (int c = tid; c < BN; c += kWsThreads) sBias[c] = __bfloat162float(a.bias[n0 + c]);
+  if (warp == kWsMmaWarp) {
+    tmem_alloc(s_tmem, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp < kWsProdWarps) {
+    // ---------------------------------------------------------------- producers
+    // resident B slice
+    for (int c = tid; c < K * (BN / 8); c += kProdThreads) {
+      const int kk = c / (BN / 8), nc = c % (BN / 8);
+      cp_async_16(sB + (kk >> 3) * lboB + nc * 128 + (kk & 7) * 16, a.Wt + (size_t)kk * a.Ntot + n0 + nc * 8, 16u);
+    }
+    cp_async_commit();
+    // A gather: warp w fills rows [32w, 32w + 32) in groups of 8 rows; 4 lanes per
+    // row, lane l moving chunks l%4, l%4 + 4, ... (64 contiguous bytes per row and
+    // instruction).
+    const int sub = lane >> 2, cq = lane & 3;
+    long long t = 0;
+    for (long long m = m_first; m < mtiles; m += m_step, ++t) {
+      const int s = (int)(t & 1);
+      if (t >= 2 && !s_abort && !mbar_wait(&a_free[s], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+        s_abort = 1;
+      uint8_t* dA = sA + s * ws_a_bytes(K);
+#pragma unroll 1
+      for (int grp = 0; grp < 4; ++grp) {
+        const int row = warp * 32 + grp * 8 + sub;
+        const long long r = m * kBM + row;
+        long long src = -1;
+        if (r < a.rows) {
+          if (MODE == kQKV) {
+            const int tok = a.rowsrc[r];
+            src = tok < 0 ? -1 : (long long)tok * g.C;
+          } else {
+            src = r * (long long)g.C;
+          }
+        }
+        uint8_t* drow = dA + (row >> 3) * sboA + (row & 7) * 16;
+        for (int kc = cq; kc < K / 8; kc += 4)
+          cp_async_16(drow + kc * 128, a.A + (src < 0 ? 0 : src + kc * 8), src < 0 ? 0u : 16u);
+      }
+      cp_async_commit();
+      cp_async_wait<1>();  // the previous group (B, or the previous tile) has landed
+      fence_proxy_async_smem();
+      if (t == 0) mbar_arrive(b_full);
+      else mbar_arrive(&a_full[(t - 1) & 1]);
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (t == 0) mbar_arrive(b_full);
+    else mbar_arrive(&a_full[(t - 1) & 1]);
+  } else if (warp == kWsMmaWarp) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      if (!mbar_wait(b_full, 0, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      const uint32_t idesc = idesc_bf16(kBM, BN, 0, 1);
+      const uint32_t baddr = smem_u32(sB);
+      long long t = 0;
+      for (long long m = m_first; m < mtiles; m += m_step, ++t) {
+        const int s = (int)(t & 1), buf = (int)(t & 1);
+        if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        if (t >= 2 && !s_abort &&
+            !mbar_wait(&acc_free[buf], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+          s_abort = 1;
+        tc_fence_after();
+        if (!s_abort) {
+          const uint32_t aaddr = smem_u32(sA + s * ws_a_bytes(K));
+          for (int ks = 0; ks < K / 16; ++ks)
+            umma_ss(tmem + buf * BN, smem_desc(aaddr + ks * 256, 128, sboA),
+                    smem_desc(baddr + ks * 2 * lboB, lboB, 128), idesc, ks > 0);
+          umma_commit(&a_free[s]);
+          umma_commit(&acc_full[buf]);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31; the eight epilogue
+    // warps cover each quarter twice, the first four taking the low column half.
+    const int q = warp & 3, hf = (warp - kWsEpi0) >> 2;
+    const int cw = BN / 2;  // columns of this warp (multiple of 8)
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    long long t = 0;
+    for (long long m = m_first; m < mtiles; m += m_step, ++t) {
+      const int buf = (int)(t & 1);
+      const long long r = m * kBM + q * 32 + lane;
+      const bool row_ok = r < a.rows;
+      long long dst_row = -1;
+      int slot = 0;
+      long long slab_win = 0;
+      if (row_ok) {
+        if (MODE == kQKV) {
+          const int ri = (int)r;  // rows < 2^31 (checked by the caller)
+          slab_win = ri / g.N;
+          slot = ri - (int)slab_win * g.N;
+        } else {
+          dst_row = a.rowsrc[r];
+        }
+      }
+      if (!s_abort && !mbar_wait(&acc_full[buf], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      tc_fence_after();
+      if (!s_abort && m * kBM + q * 32 < a.rows) {
+        for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += 32) {
+          const int n = (hf + 1) * cw - c0 < 32 ? (hf + 1) * cw - c0 : 32;  // 8, 16, 24 or 32
+          uint32_t u[32];
+          const uint32_t ta = tmem + lane_base + buf * BN + c0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (j * 8 < n)
+              asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                           : "=r"(u[8 * j + 0]), "=r"(u[8 * j + 1]), "=r"(u[8 * j + 2]), "=r"(u[8 * j + 3]),
+                             "=r"(u[8 * j + 4]), "=r"(u[8 * j + 5]), "=r"(u[8 * j + 6]), "=r"(u[8 * j + 7])
+                           : "r"(ta + 8 * j));
+          tmem_wait_ld();
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            if (g8 * 8 >= n) break;
+            const int cc = c0 + g8 * 8;
+            const int col = n0 + cc;
+            const float4 b0 = *reinterpret_cast<const float4*>(sBias + cc);
+            const float4 b1 = *reinterpret_cast<const float4*>(sBias + cc + 4);
+            float v[8] = {__uint_as_float(u[g8 * 8 + 0]) + b0.x, __uint_as_float(u[g8 * 8 + 1]) + b0.y,
+                          __uint_as_float(u[g8 * 8 + 2]) + b0.z, __uint_as_float(u[g8 * 8 + 3]) + b0.w,
+                          __uint_as_float(u[g8 * 8 + 4]) + b1.x, __uint_as_float(u[g8 * 8 + 5]) + b1.y,
+                          __uint_as_float(u[g8 * 8 + 6]) + b1.z, __uint_as_float(u[g8 * 8 + 7]) + b1.w};
+            if (MODE == kQKV) {
+              if (row_ok) {
+                const int which = col / g.C;
+                const int hh = (col % g.C) >> 5;
+                const int jj = col & 31;
+                const float sc = which == 0 ? a.qscale : 1.0f;
+                const SlabLayout& L = a.slab;
+                __nv_bfloat16* slab = a.dst + ((size_t)slab_win * g.heads + hh) * L.head_elems() +
+                                      (which == 0 ? 0 : ((size_t)L.qrows + (size_t)(which - 1) * L.kvrows) * 32);
+                const int row = which == 0 ? slot : L.kv_row(slot);
+                __nv_bfloat16* dst = slab + (row >> 3) * 256 + (jj >> 3) * 64 + (row & 7) * 8;
+                *reinterpret_cast<uint4*>(dst) =
+                    make_uint4(pack_bf16x2(v[0] * sc, v[1] * sc), pack_bf16x2(v[2] * sc, v[3] * sc),
+                               pack_bf16x2(v[4] * sc, v[5] * sc), pack_bf16x2(v[6] * sc, v[7] * sc));
+              }
+            } else if (dst_row >= 0) {
+              *reinterpret_cast<uint4*>(a.dst + dst_row * g.C + col) =
+                  make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                             pack_bf16x2(v[6], v[7]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWsMmaWarp) tmem_dealloc(tmem, tcols);
 }
 
 // ============================================================================ attention
@@ -971,6 +1208,25 @@ int pick_bn(int n) {
 
 template <int MODE>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
+  if (a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int NT = a.Ntot / a.BN;
+    const long long mtiles = (a.rows + kBM - 1) / kBM;
+    long long per_nt = sms / NT;
+    if (per_nt < 1) per_nt = 1;
+    if (per_nt > mtiles) per_nt = mtiles;
+    // at least 116 KB so that one CTA (up to 512 TMEM columns) owns each SM
+    const int smem_ws = ws_smem_bytes(a.K, a.BN) > 116 * 1024 ? ws_smem_bytes(a.K, a.BN) : 116 * 1024;
+    cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_ws);
+    if (e != cudaSuccess) return e;
+    prof_begin(MODE == kQKV ? kKindQkv : kKindProj, st);
+    gemm_ws_kernel<MODE><<<(unsigned)(per_nt * NT), kWsThreads, smem_ws, st>>>(a);
+    prof_end(MODE == kQKV ? kKindQkv : kKindProj, st);
+    count_launch();
+    return cudaGetLastError();
+  }
   cudaError_t e =
       cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes());
   if (e != cudaSuccess) return e;
@@ -994,7 +1250,8 @@ bool bf16_window_supported(const Geom& g) {
 size_t bf16_scratch_bytes(const Geom& g, long long nwin) {
   const size_t qkv = (size_t)nwin * g.heads * slab_layout(g).head_elems() * 2;
   const size_t o = (size_t)nwin * g.N * g.C * 2;
-  return qkv + o;
+  const size_t rows = ((size_t)nwin * g.N * 4 + 255) / 256 * 256;
+  return qkv + o + rows;
 }
 
 cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
@@ -1003,6 +1260,19 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   __nv_bfloat16* qkv = static_cast<__nv_bfloat16*>(scratch);
   const SlabLayout L = slab_layout(g);
   __nv_bfloat16* o = qkv + (size_t)nwin * g.heads * L.head_elems();
+  int* rowsrc = reinterpret_cast<int*>(o + (size_t)nwin * g.N * g.C);
+
+  {
+    const long long rows = nwin * g.N;
+    long long blocks = (rows + 255) / 256;
+    if (blocks > 2048) blocks = 2048;
+    prof_begin(kKindOther, st);
+    row_source_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, rowsrc);
+    prof_end(kKindOther, st);
+    count_launch();
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
+  }
 
   GemmArgs ga{};
   ga.g = g;
@@ -1018,6 +1288,7 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   ga.BN = pick_bn(3 * g.C);
   ga.qscale = kLog2e / sqrtf((float)kD);
   ga.slab = L;
+  ga.rowsrc = rowsrc;
   cudaError_t e = launch_gemm<kQKV>(ga, st);
   if (e != cudaSuccess) return e;
 

@@ -67,6 +67,47 @@ int make_ctx(KernelCtx* ctx) {
   return VSWIN_OK;
 }
 
+// Stream-ordered scratch comes from one library-owned memory pool per device
+// whose release threshold keeps freed blocks for the next call: without it
+// every synchronisation hands the scratch back to the driver and the next call
+// maps it again (hundreds of MB per layer).
+cudaMemPool_t g_pool[kMaxDevices] = {nullptr};
+
+int scratch_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VSWIN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemPoolSetAttribute");
+    g_pool[dev] = pool;
+  }
+  *out = g_pool[dev];
+  return VSWIN_OK;
+}
+
+int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
+  cudaMemPool_t pool = nullptr;
+  const int status = scratch_pool(&pool);
+  if (status != VSWIN_OK) return status;
+  cudaError_t e = cudaMallocFromPoolAsync(p, bytes, pool, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(VSWIN_ERR_NO_MEMORY, "scratch allocation of %zu bytes: %s", bytes, cudaGetErrorString(e));
+  }
+  return VSWIN_OK;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
@@ -166,11 +207,9 @@ int forward_bf16_device(const void* x, const Geom& g, const void* Wqkv, const vo
   const long long per_chunk = chunk_windows(g);
   const size_t bytes = bf16_scratch_bytes(g, per_chunk);
   void* scratch = nullptr;
-  cudaError_t e = cudaMallocAsync(&scratch, bytes, st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(VSWIN_ERR_NO_MEMORY, "cudaMallocAsync(%zu bytes): %s", bytes, cudaGetErrorString(e));
-  }
+  status = scratch_alloc(&scratch, bytes, st);
+  if (status != VSWIN_OK) return status;
+  cudaError_t e = cudaSuccess;
   for (long long w0 = 0; w0 < g.windows; w0 += per_chunk) {
     const long long n = (g.windows - w0) < per_chunk ? (g.windows - w0) : per_chunk;
     e = launch_bf16_chunk(g, ctx, x, Wqkv, bqkv, Wproj, bproj, table, out, scratch, w0, n, st);
@@ -327,13 +366,10 @@ int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int
   size_t nq = 0, no = 0;
   f32_scratch_floats(g, &nq, &no);
   void* scratch = nullptr;
-  cudaError_t e = cudaMallocAsync(&scratch, (nq + no) * sizeof(float), s);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(VSWIN_ERR_NO_MEMORY, "cudaMallocAsync: %s", cudaGetErrorString(e));
-  }
+  st = scratch_alloc(&scratch, (nq + no) * sizeof(float), s);
+  if (st != VSWIN_OK) return st;
   float* sq = static_cast<float*>(scratch);
-  e = launch_f32_forward(g, static_cast<const float*>(x), static_cast<const float*>(Wqkv),
+  cudaError_t e = launch_f32_forward(g, static_cast<const float*>(x), static_cast<const float*>(Wqkv),
                          static_cast<const float*>(bqkv), static_cast<const float*>(Wproj),
                          static_cast<const float*>(bproj), static_cast<const float*>(bias_table),
                          static_cast<float*>(out), sq, sq + nq, s);
@@ -355,11 +391,9 @@ int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* buf = nullptr;
   const size_t act_pad = (act + 255) / 256 * 256;
-  cudaError_t e = cudaMallocAsync(&buf, 2 * act_pad, s);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(VSWIN_ERR_NO_MEMORY, "cudaMallocAsync: %s", cudaGetErrorString(e));
-  }
+  st = scratch_alloc(&buf, 2 * act_pad, s);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = cudaSuccess;
   void* xd = buf;
   void* od = static_cast<uint8_t*>(buf) + act_pad;
   e = cudaMemcpyAsync(xd, x_host, act, cudaMemcpyHostToDevice, s);
