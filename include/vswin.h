@@ -173,6 +173,16 @@ unsigned long long vswin_launch_count(void);
 void vswin_set_wait_limit_ns(unsigned long long ns);
 
 /*
+ * Test hook for the bf16 (P,7,7) attention kernel. Its softmax normally uses
+ * one reference per query row, |q_i| * max_j |k_j| + max(bias) + 1 (an upper
+ * bound of the row's scores), and recomputes a row exactly -- two-pass softmax
+ * on the CUDA cores -- only when the row's sum underflows below 2^-100 (logits
+ * spanning more than ~69 natural-log units). on != 0 sends every row through
+ * that exact path, so that tests can check it; 0 restores the normal rule.
+ */
+void vswin_set_exact_softmax(int on);
+
+/*
  * Self-test of the timeout path: launches one kernel that waits, with the
  * current limit, on a barrier that nothing completes. It must give up and set
  * the error word, so a following vswin_poll_error returns VSWIN_ERR_TIMEOUT.

@@ -364,30 +364,38 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     // row, lane l moving chunks l%4, l%4 + 4, ... (64 contiguous bytes per row and
     // instruction).
     const int sub = lane >> 2, cq = lane & 3;
+    // Source offsets of this lane's 4 rows, fetched one tile ahead so that the
+    // table reads overlap the previous tile's copies.
+    auto row_src = [&](long long m, int grp) -> long long {
+      const long long r = m * kBM + warp * 32 + grp * 8 + sub;
+      if (r >= a.rows) return -1;
+      if (MODE == kQKV) {
+        const int tok = a.rowsrc[r];
+        return tok < 0 ? -1 : (long long)tok * g.C;
+      }
+      return r * (long long)g.C;
+    };
+    long long src[4];
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp) src[grp] = m_first < mtiles ? row_src(m_first, grp) : -1;
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += m_step, ++t) {
       const int s = (int)(t & 1);
       if (t >= 2 && !s_abort && !mbar_wait(&a_free[s], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
         s_abort = 1;
       uint8_t* dA = sA + s * ws_a_bytes(K);
-#pragma unroll 1
+#pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
         const int row = warp * 32 + grp * 8 + sub;
-        const long long r = m * kBM + row;
-        long long src = -1;
-        if (r < a.rows) {
-          if (MODE == kQKV) {
-            const int tok = a.rowsrc[r];
-            src = tok < 0 ? -1 : (long long)tok * g.C;
-          } else {
-            src = r * (long long)g.C;
-          }
-        }
         uint8_t* drow = dA + (row >> 3) * sboA + (row & 7) * 16;
+        const long long sg = src[grp];
         for (int kc = cq; kc < K / 8; kc += 4)
-          cp_async_16(drow + kc * 128, a.A + (src < 0 ? 0 : src + kc * 8), src < 0 ? 0u : 16u);
+          cp_async_16(drow + kc * 128, a.A + (sg < 0 ? 0 : sg + kc * 8), sg < 0 ? 0u : 16u);
       }
       cp_async_commit();
+      const long long mn = m + m_step;
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) src[grp] = mn < mtiles ? row_src(mn, grp) : -1;
       cp_async_wait<1>();  // the previous group (B, or the previous tile) has landed
       fence_proxy_async_smem();
       if (t == 0) mbar_arrive(b_full);
@@ -474,8 +482,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
                           __uint_as_float(u[g8 * 8 + 6]) + b1.z, __uint_as_float(u[g8 * 8 + 7]) + b1.w};
             if (MODE == kQKV) {
               if (row_ok) {
-                const int which = col / g.C;
-                const int hh = (col % g.C) >> 5;
+                const int sidx = col >> 5;  // (which, head) slab: C is a multiple of 32
+                const int which = sidx / g.heads;
+                const int hh = sidx - which * g.heads;
                 const int jj = col & 31;
                 const float sc = which == 0 ? a.qscale : 1.0f;
                 const SlabLayout& L = a.slab;
@@ -542,6 +551,7 @@ struct AttnArgs {
   Geom g;
   KernelCtx ctx;
   SlabLayout slab;
+  float exact_below;           // rows whose softmax sum is below this are recomputed exactly
   const __nv_bfloat16* qkv;    // per (window, head): q | k | v slabs
   const __nv_bfloat16* table;  // [rows][heads]
   __nv_bfloat16* o;            // [nwin][N][C]
@@ -835,13 +845,18 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 //
 // 256 threads: warps w and w+4 share TMEM lane quarter w%4 (query rows
 // 32*(w%4) .. +31 of the tile) and split each key block into two halves of
-// 8-column key lines. Per block, pass 1 takes the row max of the raw scores
-// (exchanged between the two halves); the block max used for the exponentials
-// is that plus the head's largest bias, an upper bound of the true maximum of
-// score + bias that exceeds it by at most the bias range, so nothing overflows
-// and nothing that matters underflows. Pass 2 streams score + bias -> exp2 ->
-// row sum -> bf16 P. Each half writes its P into its own S columns (already
-// read), and O = P V runs as two K ranges, one per half.
+// 8-column key lines; each half streams score + bias -> exp2 -> row sum ->
+// bf16 P, writes its P into its own S columns (already read), and O = P V runs
+// as two K ranges, one per half.
+//
+// Softmax reference. Each query row i uses one reference for all its keys,
+//   m_i = |q_i| * max_j |k_j| + max(bias) + 1   (log2 units, q pre-scaled),
+// an upper bound of every score + bias of the row (Cauchy-Schwarz), so no
+// exponential overflows and no per-block maximum is needed. The bound exceeds
+// the row's true maximum by the slack of the inequality; should that slack be
+// so large that the row sum underflows (below 2^-100: logits spanning more
+// than ~69 natural-log units), the row is recomputed exactly with a two-pass
+// softmax on the CUDA cores (w7_exact_row).
 constexpr int kAttn7Threads = 256;
 
 template <int P_>
@@ -951,6 +966,67 @@ __device__ __forceinline__ float w7_pass2(uint32_t tcol, int l0, int l1, const f
   return s0 + s1;
 }
 
+// Exact recomputation of one query row (rare path, see the reference rule
+// above the kernel): two-pass softmax over the allowed keys on the CUDA cores,
+// operands read from shared memory; writes the row's 32 normalised outputs.
+template <class Wn>
+__device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, const uint8_t* sV, const float* tb_row,
+                                          int i, uint32_t okt, uint32_t okh, uint32_t okw, float* o) {
+  float q[32];
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4*>(sQ + (i >> 3) * 512 + c * 128 + (i & 7) * 16);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(h2[k]);
+      q[c * 8 + 2 * k] = f.x;
+      q[c * 8 + 2 * k + 1] = f.y;
+    }
+  }
+  auto score = [&](int n) {  // q . k of slab row n
+    float acc = 0.f;
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = *reinterpret_cast<const uint4*>(sK + (n >> 3) * 512 + c * 128 + (n & 7) * 16);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(h2[k]);
+        acc = fmaf(q[c * 8 + 2 * k], f.x, acc);
+        acc = fmaf(q[c * 8 + 2 * k + 1], f.y, acc);
+      }
+    }
+    return acc;
+  };
+  float m = -INFINITY;
+  for (int line = 0; line < Wn::KLINES; ++line) {
+    const int pt = line / 7, ph = line - 7 * pt;
+    const uint32_t lm = ((okt >> pt) & (okh >> ph) & 1u) ? okw : 0u;
+    for (int pw = 0; pw < 7; ++pw)
+      if ((lm >> pw) & 1u) m = fmaxf(m, score(line * 8 + pw) + tb_row[-(pt * 169 + ph * 13 + pw)]);
+  }
+  float l = 0.f;
+  for (int d = 0; d < 32; ++d) o[d] = 0.f;
+  for (int line = 0; line < Wn::KLINES; ++line) {
+    const int pt = line / 7, ph = line - 7 * pt;
+    const uint32_t lm = ((okt >> pt) & (okh >> ph) & 1u) ? okw : 0u;
+    for (int pw = 0; pw < 7; ++pw) {
+      if (!((lm >> pw) & 1u)) continue;
+      const int n = line * 8 + pw;
+      const float pr = exp2f(score(n) + tb_row[-(pt * 169 + ph * 13 + pw)] - m);
+      l += pr;
+      for (int ch = 0; ch < 4; ++ch) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sV + (n >> 3) * 512 + ch * 128 + (n & 7) * 16);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h2[k]);
+          o[ch * 8 + 2 * k] = fmaf(pr, f.x, o[ch * 8 + 2 * k]);
+          o[ch * 8 + 2 * k + 1] = fmaf(pr, f.y, o[ch * 8 + 2 * k + 1]);
+        }
+      }
+    }
+  }
+  const float inv = 1.0f / l;
+  for (int d = 0; d < 32; ++d) o[d] *= inv;
+}
+
 template <class Wn>
 __global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -966,6 +1042,7 @@ __global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_ld + 3);
   __shared__ int s_abort;
   __shared__ float s_part[kAttn7Threads / 32];
+  __shared__ float s_kpart[kAttn7Threads / 32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, half = warp >> 2;
@@ -1035,14 +1112,31 @@ __global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a
         *reinterpret_cast<uint4*>(sV + (n >> 3) * 512 + chunk * 128 + (n & 7) * 16) = make_uint4(0, 0, 0, 0);
       }
     }
+    {
+      float kx = 0.f;
+      for (int n = tid; n < Wn::KLINES * 8; n += kAttn7Threads) {
+        if ((n & 7) == 7) continue;
+        float acc = 0.f;
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sK + (n >> 3) * 512 + c * 128 + (n & 7) * 16);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+          for (int k = 0; k < 4; ++k) { const float2 f = __bfloat1622float2(h2[k]); acc = fmaf(f.x, f.x, fmaf(f.y, f.y, acc)); }
+        }
+        kx = fmaxf(kx, acc);
+      }
+      for (int off = 16; off > 0; off >>= 1) kx = fmaxf(kx, __shfl_xor_sync(0xffffffffu, kx, off));
+      if (lane == 0) s_kpart[warp] = kx;
+    }
     fence_proxy_async_smem();
     __syncthreads();
     if (s_abort) break;
+    float kmax = 0.f;
     {
-      float mx = s_part[0];
+      float mx = s_part[0], kx = s_kpart[0];
 #pragma unroll
-      for (int k = 1; k < kAttn7Threads / 32; ++k) mx = fmaxf(mx, s_part[k]);
+      for (int k = 1; k < kAttn7Threads / 32; ++k) { mx = fmaxf(mx, s_part[k]); kx = fmaxf(kx, s_kpart[k]); }
       bmax = mx;
+      kmax = sqrtf(kx);
     }
     const int split = window_split_bits(g, (int)(win % g.nW));
 
@@ -1071,6 +1165,17 @@ __global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a
         }
       }
       float mrow[3] = {-INFINITY, -INFINITY, -INFINITY}, lrow[3] = {0.f, 0.f, 0.f};
+      float mref = 0.f;
+      {
+        float qq = 0.f;
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sQ + (ie >> 3) * 512 + c * 128 + (ie & 7) * 16);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+          for (int k = 0; k < 4; ++k) { const float2 f = __bfloat1622float2(h2[k]); qq = fmaf(f.x, f.x, fmaf(f.y, f.y, qq)); }
+        }
+        mref = sqrtf(qq) * kmax + bmax + 1.0f;
+        if (!(mref < 3.0e38f)) mref = 0.f;
+      }
 
       if (tid == 0) {
         tc_fence_after();
@@ -1090,13 +1195,8 @@ __global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a
         __syncthreads();
         tc_fence_after();
         if (active && !s_abort) {
-          const float mp = split ? w7_pass1<Wn, true>(tcol, l0, l1, okt, okh, okw)
-                                 : w7_pass1<Wn, false>(tcol, l0, l1, okt, okh, okw);
-          xmax[half * 128 + rt] = mp;
-          named_bar(1 + quarter, 64);
-          const float ms = fmaxf(xmax[rt], xmax[128 + rt]);
-          const float mb = ms == -INFINITY ? -INFINITY : ms + bmax;
-          const float mm = mb == -INFINITY ? 0.f : mb;
+          const float mb = mref;
+          const float mm = mref;
           lrow[b] = split ? w7_pass2<Wn, true>(tcol, l0, l1, tb_row, mm, okt, okh, okw)
                           : w7_pass2<Wn, false>(tcol, l0, l1, tb_row, mm, okt, okh, okw);
           mrow[b] = mb;
@@ -1160,13 +1260,24 @@ __global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a
           for (int k = 0; k < 16; ++k) o[k] = fmaf(__uint_as_float(u[k]), f, o[k]);
         }
         if (i < Wn::N) {
-          __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD + 16 * half;
-          reinterpret_cast<uint4*>(dst)[0] =
-              make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                         pack_bf16x2(o[6], o[7]));
-          reinterpret_cast<uint4*>(dst)[1] =
-              make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
-                         pack_bf16x2(o[14], o[15]));
+          __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD;
+          if (L >= a.exact_below) {  // the common case
+            dst += 16 * half;
+            reinterpret_cast<uint4*>(dst)[0] =
+                make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                           pack_bf16x2(o[6], o[7]));
+            reinterpret_cast<uint4*>(dst)[1] =
+                make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
+                           pack_bf16x2(o[14], o[15]));
+          } else if (half == 0) {  // the reference was too loose for this row: recompute it exactly
+            float oe[32];
+            w7_exact_row<Wn>(sQ, sK, sV, tb_row, i, okt, okh, okw, oe);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd)
+              reinterpret_cast<uint4*>(dst)[qd] =
+                  make_uint4(pack_bf16x2(oe[8 * qd + 0], oe[8 * qd + 1]), pack_bf16x2(oe[8 * qd + 2], oe[8 * qd + 3]),
+                             pack_bf16x2(oe[8 * qd + 4], oe[8 * qd + 5]), pack_bf16x2(oe[8 * qd + 6], oe[8 * qd + 7]));
+          }
         }
       }
       tc_fence_before();
@@ -1301,6 +1412,7 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   aa.win0 = win0;
   aa.nwin = nwin;
   aa.slab = L;
+  aa.exact_below = ctx.force_exact ? INFINITY : 7.8886e-31f;  // 2^-100
   const int P = g.win[0], MH = g.win[1], MW = g.win[2];
   if (P == 8 && MH == 7 && MW == 7) e = launch_attention7<W7<8>>(aa, st);
   else if (P == 4 && MH == 7 && MW == 7) e = launch_attention7<W7<4>>(aa, st);

@@ -11,6 +11,7 @@ namespace vswin {
 struct KernelCtx {
   int* err;                       // device error word (0 = fine)
   unsigned long long wait_limit;  // ns
+  int force_exact;                // test hook: every row through the exact softmax path
 };
 
 // Device-side error codes written to the error word.

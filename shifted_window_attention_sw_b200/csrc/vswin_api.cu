@@ -22,6 +22,7 @@ namespace {
 thread_local std::string t_last_error;
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_wait_limit_ns{1000000000ULL};
+std::atomic<int> g_force_exact{0};
 std::mutex g_mu;
 constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices] = {nullptr};
@@ -64,6 +65,7 @@ int make_ctx(KernelCtx* ctx) {
   if (st != VSWIN_OK) return st;
   ctx->err = err;
   ctx->wait_limit = g_wait_limit_ns.load();
+  ctx->force_exact = g_force_exact.load();
   return VSWIN_OK;
 }
 
@@ -322,6 +324,8 @@ const char* vswin_last_error(void) { return t_last_error.c_str(); }
 unsigned long long vswin_launch_count(void) { return g_launches.load(); }
 
 void vswin_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns ? ns : 1); }
+
+void vswin_set_exact_softmax(int on) { g_force_exact.store(on ? 1 : 0); }
 
 int vswin_clamp_window(int T, int H, int W, const int* window_in, const int* shift_in, int* window_out,
                        int* shift_out) {

@@ -33,6 +33,7 @@ EXPORTS = (
     "vswin_profile_enable",
     "vswin_profile_collect",
     "vswin_wmsa_forward_noalloc",
+    "vswin_set_exact_softmax",
 )
 
 KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other")
@@ -76,6 +77,8 @@ def lib():
         L.vswin_launch_count.restype = ctypes.c_ulonglong
         L.vswin_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.vswin_set_wait_limit_ns.restype = None
+        L.vswin_set_exact_softmax.argtypes = [_I]
+        L.vswin_set_exact_softmax.restype = None
         L.vswin_selftest_timeout.argtypes = [_P]
         L.vswin_selftest_timeout.restype = _I
         L.vswin_profile_enable.argtypes = [_I]
@@ -198,6 +201,11 @@ def launch_count() -> int:
 
 def set_wait_limit_ns(ns: int) -> None:
     lib().vswin_set_wait_limit_ns(int(ns))
+
+
+def set_exact_softmax(on: bool) -> None:
+    """Test hook: route every query row of the bf16 (P,7,7) kernel through its exact softmax path."""
+    lib().vswin_set_exact_softmax(1 if on else 0)
 
 
 def selftest_timeout(stream=None) -> None:

@@ -165,6 +165,35 @@ def test_bf16_separates_plausible_slips(flag):
     assert np.linalg.norm(out - ref) * 10 <= np.linalg.norm(out - mut)
 
 
+@pytest.mark.parametrize("shape,heads,window,shift", [((1, 8, 14, 14, 96), 3, (8, 7, 7), (4, 3, 3)),
+                                                     ((1, 4, 14, 14, 64), 2, (4, 7, 7), (2, 3, 3))])
+def test_bf16_exact_softmax_rows(shape, heads, window, shift):
+    # Every row through the kernel's exact two-pass recomputation (normally taken only
+    # when the per-row reference is too loose): same parity gates as the fast path.
+    inp = make_layer_inputs(shape, heads, window, "bf16", "sensitivity", seed=515)
+    ref = _oracle(inp.as_f64(), window, shift, heads)
+    vswin.set_exact_softmax(True)
+    try:
+        out = _gpu(inp, window, shift, heads, "bf16")
+    finally:
+        vswin.set_exact_softmax(False)
+    _check_bf16(out, ref, True)
+
+
+def test_bf16_large_logits():
+    # Query/key magnitudes 6x the sensitivity scale: logits spread over tens of units,
+    # the regime where the per-row reference is loosest.
+    shape, heads, window, shift = (1, 8, 14, 14, 64), 2, (8, 7, 7), (4, 3, 3)
+    inp = make_layer_inputs(shape, heads, window, "bf16", "sensitivity", seed=616)
+    C = shape[-1]
+    inp.Wqkv[:, :2 * C] = (inp.Wqkv[:, :2 * C].float() * 6.0).to(torch.bfloat16)
+    ref = _oracle(inp.as_f64(), window, shift, heads)
+    out = _gpu(inp, window, shift, heads, "bf16")
+    assert np.isfinite(out).all()
+    s = _stats(out, ref)
+    assert s["rel_l2"] <= 5e-2, s  # peaked softmax: bf16 rounding of q and k moves the weights more
+
+
 def test_bf16_deterministic():
     shape, heads, window, shift = (2, 16, 14, 14, 96), 3, (8, 7, 7), (4, 3, 3)
     d = make_layer_inputs(shape, heads, window, "bf16", "sensitivity", seed=7).to("cuda")
