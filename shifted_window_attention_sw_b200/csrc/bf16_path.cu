@@ -843,132 +843,149 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 
 // ============================================================================ attention, (P,7,7) windows
 //
-// 256 threads: warps w and w+4 share TMEM lane quarter w%4 (query rows
-// 32*(w%4) .. +31 of the tile) and split each key block into two halves of
-// 8-column key lines; each half streams score + bias -> exp2 -> row sum ->
-// bf16 P, writes its P into its own S columns (already read), and O = P V runs
-// as two K ranges, one per half.
+// Persistent, warp-specialised kernel, one CTA per SM, 416 threads:
+//   warps 0-3    preparation of (window, head) items, two in flight: bulk loads
+//                of the q / k / v slabs, the head's bias table in log2 units,
+//                key norms, the extension rows of the score MMA (below), zeroed
+//                v padding;
+//   warp 4       tcgen05.mma issue (one thread), serving the two softmax
+//                groups in turn;
+//   warps 5-8 and 9-12   softmax groups 0 and 1: group g owns this CTA's query
+//                tiles g, g + 2, g + 4, ... (128-row tiles, items in order).
+// Keys are taken in blocks of up to 20 lines of 8 columns (the 7 keys of one
+// (pt, ph) line and a padding column). Per block: S = q k^T into the group's
+// TMEM columns, the group turns S into bf16 P in place, then O += P v and
+// l += P 1 on the tensor core. While one group exponentiates, the tensor core
+// works for the other.
 //
-// Softmax reference. Each query row i uses one reference for all its keys,
+// Softmax reference. Every query row i uses one reference for all its keys,
 //   m_i = |q_i| * max_j |k_j| + max(bias) + 1   (log2 units, q pre-scaled),
-// an upper bound of every score + bias of the row (Cauchy-Schwarz), so no
-// exponential overflows and no per-block maximum is needed. The bound exceeds
-// the row's true maximum by the slack of the inequality; should that slack be
-// so large that the row sum underflows (below 2^-100: logits spanning more
-// than ~69 natural-log units), the row is recomputed exactly with a two-pass
-// softmax on the CUDA cores (w7_exact_row).
-constexpr int kAttn7Threads = 256;
+// an upper bound of every score + bias of the row (Cauchy-Schwarz): no
+// exponential overflows, blocks need no rescaling, and O and l accumulate
+// straight across blocks. Should the bound's slack make the row sum underflow
+// (below 2^-100: logits spanning more than ~69 natural-log units), the row is
+// recomputed exactly by a two-pass softmax on the CUDA cores (w7_exact_row).
+//
+// The reference and the shifted-window mask enter the score MMA as one extra
+// K = 16 step whose two 8-column halves read the same 16-byte rows (descriptor
+// K stride 0):
+//   query row i:  (-m_i/2, 1/2, r_t(i)/2, r_h(i)/2, r_w(i)/2, 0, 0, 0)
+//   key j:        (1, -256 (r_t(j) + r_h(j) + r_w(j)), y_t(j), y_h(j), y_w(j), 0, 0, 0)
+// where r_a is the region bit of a slot on split axis a (0 on other axes) and
+// y_a = -256 (1 - 2 r_a) on split axes. Over both halves the step adds
+// -m_i - 256 * #{axes whose regions differ}: every allowed key of row i gets
+// the same -m_i (identical step inputs), masked keys end at least 257 below
+// the reference and exponentiate to exactly 0. -m_i/2 is rounded towards
+// -inf, so the effective reference is never below m_i.
+constexpr int kA7Threads = 416;
+constexpr int kA7PrepWarps = 4;
+constexpr int kA7MmaWarp = 4;
+constexpr int kA7Soft0 = 5;
+constexpr uint32_t kA7TmemCols = 512;
+constexpr uint32_t kA7GroupCols = 256;  // per group: S / P [0, 160), O [160, 192), l [192, 208)
+constexpr uint32_t kA7OCol = 160;
+constexpr uint32_t kA7LCol = 192;
 
 template <int P_>
 struct W7 {
   static constexpr int P = P_;
   static constexpr int N = P * 49;
-  static constexpr int QSLAB = (N + 15) / 16 * 16;             // q slab rows
-  static constexpr int KLINES = P * 7;                         // key lines of 7 real keys
-  static constexpr int KCOLS = (KLINES * 8 + 31) / 32 * 32;    // k/v slab rows (padded key columns)
-  static constexpr int LINES = KCOLS / 8;                      // multiple of 4
+  static constexpr int QSLAB = (N + 15) / 16 * 16;           // q slab rows
+  static constexpr int KLINES = P * 7;                       // key lines of 7 real keys
+  static constexpr int KCOLS = (KLINES * 8 + 31) / 32 * 32;  // k / v slab rows (padded key columns)
+  static constexpr int LINES = KCOLS / 8;
   static constexpr int NBLK = (LINES + 19) / 20;
-  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 3) / 4 * 4;  // lines per block but the last
+  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 1) / 2 * 2;  // lines per block but the last
   static constexpr int LAST = LINES - (NBLK - 1) * BL;
   static constexpr int TABLE = (2 * P - 1) * 169;
   static constexpr int QTILES = (N + 127) / 128;
-  static constexpr int QROWS = QTILES * 128 > QSLAB ? QTILES * 128 : QSLAB;
+  static constexpr int TAIL = N - (QTILES - 1) * 128;  // rows of the last tile
+  // A last tile of at most 32 rows is placed in lane quarter (item & 3), so that
+  // its work rotates over the four SM sub-partitions.
+  static constexpr bool ROTATE = QTILES > 1 && TAIL <= 32;
+  static constexpr int QXROWS = QTILES * 128;
+  // shared memory, two item buffers of each
+  static constexpr int QB = QSLAB * kSlabRowBytes;
+  static constexpr int KB = KCOLS * kSlabRowBytes;
+  static constexpr int QXB = QXROWS * 16;
+  static constexpr int KXB = KCOLS * 16;
+  static constexpr int TB = (TABLE * 4 + 127) / 128 * 128;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + QROWS * kSlabRowBytes;
-  static constexpr int OFF_V = OFF_K + KCOLS * kSlabRowBytes;
-  static constexpr int OFF_T = OFF_V + KCOLS * kSlabRowBytes;
-  static constexpr int OFF_X = OFF_T + (TABLE * 4 + 15) / 16 * 16;  // exchange: max[2][128], sum[2][3][128]
-  static constexpr int OFF_BAR = OFF_X + (2 * 128 + 6 * 128) * 4;
-  static constexpr int SMEM = (OFF_BAR + 64) < 81920 ? 81920 : (OFF_BAR + 64);
-  static_assert(NBLK <= 3 && BL <= 20 && LAST > 0 && LAST % 4 == 0, "key blocks must fit 160 TMEM columns");
-  static_assert(SMEM <= 110 * 1024, "two CTAs per SM");
+  static constexpr int OFF_K = OFF_Q + 2 * QB;
+  static constexpr int OFF_V = OFF_K + 2 * KB;
+  static constexpr int OFF_QX = OFF_V + 2 * KB;
+  static constexpr int OFF_KX = OFF_QX + 2 * QXB;
+  static constexpr int OFF_T = OFF_KX + 2 * KXB;
+  static constexpr int OFF_ONES = OFF_T + 2 * TB;
+  static constexpr int OFF_BAR = OFF_ONES + 512;
+  static constexpr int SMEM = OFF_BAR + 256;
+  static_assert(NBLK <= 3 && BL <= 20 && LAST > 0 && LAST % 2 == 0, "key blocks must fit 160 TMEM columns");
+  // a tile's operand rows beyond the q slab read the following buffers (their
+  // results land in TMEM lanes that are never used)
+  static_assert(OFF_Q + QB + QXROWS * kSlabRowBytes <= SMEM, "tile rows must stay inside shared memory");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 template <class Wn>
-__device__ __forceinline__ int w7_block_lines(int b) {
-  return b < Wn::NBLK - 1 ? Wn::BL : Wn::LAST;
+__device__ __forceinline__ int w7_tile_row0(int qt, long long jj) {
+  if (Wn::ROTATE && qt == Wn::QTILES - 1) return qt * 128 - 32 * (int)(jj & 3);
+  return qt * 128;
 }
 
-// Pass 1 over this thread's lines of one block: max of the allowed raw scores.
-template <class Wn, bool MASKED>
-__device__ __forceinline__ float w7_pass1(uint32_t tcol, int l0, int l1, uint32_t okt, uint32_t okh,
-                                          uint32_t okw) {
-  float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll 1
-  for (int l = l0; l < l1; l += 2) {
-    uint32_t u[16];
-    tmem_ld16(tcol + (l - l0) * 8, u);
-    tmem_wait_ld();
+// Region bit of slot coordinate c on an axis cut at `cut`, when the axis is split.
+__device__ __forceinline__ int w7_region(int split_bit, int c, int cut) { return (split_bit && c >= cut) ? 1 : 0; }
+
+// Lines l and l + 1 of a block (16 TMEM columns in u): p = 2^(s + bias) for
+// the 7 keys of a real line, 0 for padding columns and padding lines; packed
+// into 8 bf16x2 words.
+template <class Wn>
+__device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], const float* tb_row, uint32_t* pk) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int line = l + c;
-      if (line < Wn::KLINES) {
-        const int pt = line / 7, ph = line - 7 * (line / 7);
-        const uint32_t lm = ((okt >> pt) & (okh >> ph) & 1u) ? okw : 0u;  // allowed pw of this line
+  for (int c = 0; c < 2; ++c) {
+    const int line = l + c;
+    float p[8];
+    if (line < Wn::KLINES) {
+      const float* tbr = tb_row - ((line / 7) * 169 + (line % 7) * 13);
 #pragma unroll
-        for (int pw = 0; pw < 7; ++pw) {
-          const float v = __uint_as_float(u[c * 8 + pw]);
-          const bool ok = !MASKED || ((lm >> pw) & 1u);
-          if (pw & 1)
-            m1 = ok ? fmaxf(m1, v) : m1;
-          else
-            m0 = ok ? fmaxf(m0, v) : m0;
-        }
-      }
+      for (int pw = 0; pw < 7; ++pw) p[pw] = ex2_approx(__uint_as_float(u[c * 8 + pw]) + tbr[-pw]);
+    } else {
+#pragma unroll
+      for (int pw = 0; pw < 7; ++pw) p[pw] = 0.f;
     }
+    p[7] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pk[c * 4 + k] = pack_bf16x2(p[2 * k], p[2 * k + 1]);
   }
-  return fmaxf(m0, m1);
 }
 
-// Pass 2: p = exp2(score + bias - mm) on allowed keys (0 elsewhere), row sum,
-// bf16 P written to TMEM at this half's P columns.
-template <class Wn, bool MASKED>
-__device__ __forceinline__ float w7_pass2(uint32_t tcol, int l0, int l1, const float* tb_row, float mm,
-                                          uint32_t okt, uint32_t okh, uint32_t okw) {
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll 1
-  for (int l = l0; l < l1; l += 2) {
-    uint32_t u[16];
-    tmem_ld16(tcol + (l - l0) * 8, u);
-    tmem_wait_ld();
+// One key block of NL lines starting at line L0 for this thread's query row:
+// S (TMEM columns from tS) -> bf16 P written in place (4 columns per line),
+// the next line pair's load in flight while the current one is processed.
+template <class Wn, int NL>
+__device__ __forceinline__ void w7_block(uint32_t tS, int L0, const float* tb_row) {
+  uint32_t ua[16], ub[16];
+  tmem_ld16(tS, ua);
+  tmem_wait_ld_keep(ua);
+#pragma unroll
+  for (int k = 0; k < NL / 2; ++k) {
     uint32_t pk[8];
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int line = l + c;
-      float p[8];
-      if (line < Wn::KLINES) {
-        const int pt = line / 7, ph = line - 7 * (line / 7);
-        const uint32_t lm = ((okt >> pt) & (okh >> ph) & 1u) ? okw : 0u;
-        const float* tbr = tb_row - (pt * 169 + ph * 13);
-#pragma unroll
-        for (int pw = 0; pw < 7; ++pw) {
-          const bool ok = !MASKED || ((lm >> pw) & 1u);
-          const float t = __uint_as_float(u[c * 8 + pw]) + tbr[-pw] - mm;
-          p[pw] = ok ? ex2_approx(t) : 0.f;
-        }
-      } else {
-#pragma unroll
-        for (int pw = 0; pw < 7; ++pw) p[pw] = 0.f;
-      }
-      p[7] = 0.f;
-      s0 += (p[0] + p[2]) + (p[4] + p[6]);
-      s1 += (p[1] + p[3]) + p[5];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) pk[c * 4 + k] = pack_bf16x2(p[2 * k], p[2 * k + 1]);
+    if ((k & 1) == 0) {
+      if (k + 1 < NL / 2) tmem_ld16(tS + 16 * (k + 1), ub);
+      w7_line_pair<Wn>(L0 + 2 * k, ua, tb_row, pk);
+      tmem_st8(tS + 8 * k, pk);
+      if (k + 1 < NL / 2) tmem_wait_ld_keep(ub);
+    } else {
+      if (k + 1 < NL / 2) tmem_ld16(tS + 16 * (k + 1), ua);
+      w7_line_pair<Wn>(L0 + 2 * k, ub, tb_row, pk);
+      tmem_st8(tS + 8 * k, pk);
+      if (k + 1 < NL / 2) tmem_wait_ld_keep(ua);
     }
-    // P of lines l, l+1 -> 8 columns at 4 per line from the half's first column
-    tmem_st8(tcol + (l - l0) * 4, pk);
   }
-  return s0 + s1;
 }
 
 // Exact recomputation of one query row (rare path, see the reference rule
-// above the kernel): two-pass softmax over the allowed keys on the CUDA cores,
-// operands read from shared memory; writes the row's 32 normalised outputs.
+// above): two-pass softmax over the allowed keys on the CUDA cores, operands
+// read from shared memory; writes the row's 32 normalised outputs.
 template <class Wn>
 __device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, const uint8_t* sV, const float* tb_row,
                                           int i, uint32_t okt, uint32_t okh, uint32_t okw, float* o) {
@@ -1027,268 +1044,364 @@ __device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, 
   for (int d = 0; d < 32; ++d) o[d] *= inv;
 }
 
+__device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 v) { return (uint32_t)__bfloat16_as_ushort(v); }
+
 template <class Wn>
-__global__ void __launch_bounds__(kAttn7Threads, 2) attention7_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sQ = smem + Wn::OFF_Q;
-  uint8_t* sK = smem + Wn::OFF_K;
-  uint8_t* sV = smem + Wn::OFF_V;
-  float* sT = reinterpret_cast<float*>(smem + Wn::OFF_T);
-  float* xmax = reinterpret_cast<float*>(smem + Wn::OFF_X);  // [2][128]
-  float* xsum = xmax + 2 * 128;                              // [2][3][128]
-  uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + Wn::OFF_BAR);
-  uint64_t* bar_s = bar_ld + 1;
-  uint64_t* bar_o = bar_ld + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_ld + 3);
-  __shared__ int s_abort;
-  __shared__ float s_part[kAttn7Threads / 32];
-  __shared__ float s_kpart[kAttn7Threads / 32];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Wn::OFF_BAR);
+  uint64_t* ld_full = bars;        // [buffer] q / k / v bytes landed
+  uint64_t* prep_done = bars + 2;  // [buffer] item prepared (128 arrivals)
+  uint64_t* buf_free = bars + 4;   // [buffer] item finished (MMA commit + 4 warps per tile)
+  uint64_t* s_full = bars + 6;     // [group] S of the group's current block in TMEM
+  uint64_t* p_full = bars + 8;     // [group] P written (128 arrivals)
+  uint64_t* o_full = bars + 10;    // [group] O and l of the group's tile complete
+  uint64_t* prep_sync = bars + 12; // preparation warps' own barrier (128 arrivals)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
+  float* s_red = reinterpret_cast<float*>(smem + Wn::OFF_BAR + 128);  // [buffer][8]
+  __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quarter = warp & 3, half = warp >> 2;
-  const int rt = quarter * 32 + lane;  // row within the query tile = TMEM lane
   const Geom& g = a.g;
   const long long nitems = a.nwin * g.heads;
-  const uint32_t qbytes = Wn::QSLAB * kSlabRowBytes, kvbytes = Wn::KCOLS * kSlabRowBytes;
+  const long long nmine =
+      nitems > (long long)blockIdx.x ? (nitems - (long long)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const long long ntiles = nmine * Wn::QTILES;
+  const uint64_t lim = a.ctx.wait_limit;
+  const int cut_t = Wn::P - g.sh[0], cut_h = 7 - g.sh[1], cut_w = 7 - g.sh[2];
 
   if (tid == 0) {
-    mbar_init(bar_ld, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&ld_full[k], 1);
+      mbar_init(&prep_done[k], kA7PrepWarps * 32);
+      mbar_init(&buf_free[k], 5 * Wn::QTILES);
+      mbar_init(&s_full[k], 1);
+      mbar_init(&p_full[k], 128);
+      mbar_init(&o_full[k], 1);
+    }
+    mbar_init(prep_sync, kA7PrepWarps * 32);
     fence_mbar_init();
     s_abort = 0;
   }
-  for (int k = Wn::QSLAB * kSlabRowBytes / 16 + tid; k < Wn::QROWS * kSlabRowBytes / 16; k += kAttn7Threads)
-    reinterpret_cast<uint4*>(sQ)[k] = make_uint4(0, 0, 0, 0);
+  // Ones operand of l = P 1: 16 keys x 16 columns, MN-major (K-group stride
+  // 256 B, N-group stride 128 B), column 0 = 1.
+  if (tid < 32) {
+    const int ngroup = (tid >> 3) & 1;
+    reinterpret_cast<uint4*>(smem + Wn::OFF_ONES)[tid] = make_uint4(ngroup == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
+  }
   fence_proxy_async_smem();
-  if (warp == 0) {
-    tmem_alloc(s_tmem, kTmemCols);
+  if (warp == kA7MmaWarp) {
+    tmem_alloc(s_tmem, kA7TmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-  const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
 
-  uint32_t ph_ld = 0, ph_s = 0, ph_o = 0;
-  int cur_head = -1;
-  float bmax = 0.f;
-
-#pragma unroll 1
-  for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int h = (int)(item / a.nwin);
-    const long long wl = item % a.nwin;
-    const long long win = a.win0 + wl;
-    if (tid == 0) {
-      const __nv_bfloat16* base = a.qkv + ((size_t)wl * g.heads + h) * a.slab.head_elems();
-      mbar_arrive_expect_tx(bar_ld, qbytes + 2 * kvbytes);
-      bulk_g2s(sQ, base, qbytes, bar_ld);
-      bulk_g2s(sK, base + (size_t)Wn::QSLAB * kD, kvbytes, bar_ld);
-      bulk_g2s(sV, base + (size_t)(Wn::QSLAB + Wn::KCOLS) * kD, kvbytes, bar_ld);
-    }
-    if (h != cur_head) {
-      float mx = -INFINITY;
-      for (int k = tid; k < Wn::TABLE; k += kAttn7Threads) {
-        const float v = __bfloat162float(a.table[(size_t)k * g.heads + h]) * kLog2e;
-        sT[k] = v;
-        mx = fmaxf(mx, v);
+  if (warp < kA7PrepWarps) {
+    // ------------------------------------------------------------ preparation
+    const int pt_ = tid;
+    int tab_head[2] = {-1, -1};
+    float tab_max[2] = {0.f, 0.f};
+    uint32_t ph_sync = 0;
+    long long j = 0;
+    for (long long item = blockIdx.x; item < nitems; item += gridDim.x, ++j) {
+      const int X = (int)(j & 1);
+      const uint32_t use = (uint32_t)(j >> 1);
+      if (j >= 2 && !mbar_wait(&buf_free[X], (use - 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      if (s_abort) break;
+      const int h = (int)(item / a.nwin);
+      const long long wl = item % a.nwin;
+      uint8_t* sQ = smem + Wn::OFF_Q + X * Wn::QB;
+      uint8_t* sK = smem + Wn::OFF_K + X * Wn::KB;
+      uint8_t* sV = smem + Wn::OFF_V + X * Wn::KB;
+      uint8_t* sQX = smem + Wn::OFF_QX + X * Wn::QXB;
+      uint8_t* sKX = smem + Wn::OFF_KX + X * Wn::KXB;
+      float* sT = reinterpret_cast<float*>(smem + Wn::OFF_T + X * Wn::TB);
+      float* red = s_red + X * 8;
+      if (pt_ == 0) {
+        const __nv_bfloat16* base = a.qkv + ((size_t)wl * g.heads + h) * a.slab.head_elems();
+        mbar_arrive_expect_tx(&ld_full[X], (uint32_t)(Wn::QB + 2 * Wn::KB));
+        bulk_g2s(sQ, base, Wn::QB, &ld_full[X]);
+        bulk_g2s(sK, base + (size_t)Wn::QSLAB * kD, Wn::KB, &ld_full[X]);
+        bulk_g2s(sV, base + (size_t)(Wn::QSLAB + Wn::KCOLS) * kD, Wn::KB, &ld_full[X]);
       }
+      const bool new_table = h != tab_head[X];
+      if (new_table) {
+        float mx = -INFINITY;
+        for (int k = pt_; k < Wn::TABLE; k += kA7PrepWarps * 32) {
+          const float v = __bfloat162float(a.table[(size_t)k * g.heads + h]) * kLog2e;
+          sT[k] = v;
+          mx = fmaxf(mx, v);
+        }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      if (lane == 0) s_part[warp] = mx;
-      cur_head = h;
-    }
-    if (!mbar_wait(bar_ld, ph_ld, a.ctx.err, kErrWaitLoad, a.ctx.wait_limit)) s_abort = 1;
-    ph_ld ^= 1;
-    // Padding rows of the v slab (8th key of each line, whole padding lines) must be
-    // finite for O = P V: zero them (four 16-byte pieces per row).
-    {
-      constexpr int ndummy = Wn::KLINES + (Wn::LINES - Wn::KLINES) * 8;
-      for (int k = tid; k < ndummy * 4; k += kAttn7Threads) {
-        const int d = k >> 2, chunk = k & 3;
-        const int n = d < Wn::KLINES ? d * 8 + 7 : Wn::KLINES * 8 + (d - Wn::KLINES);
-        *reinterpret_cast<uint4*>(sV + (n >> 3) * 512 + chunk * 128 + (n & 7) * 16) = make_uint4(0, 0, 0, 0);
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red[warp] = mx;
       }
-    }
-    {
-      float kx = 0.f;
-      for (int n = tid; n < Wn::KLINES * 8; n += kAttn7Threads) {
-        if ((n & 7) == 7) continue;
-        float acc = 0.f;
-        for (int c = 0; c < 4; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(sK + (n >> 3) * 512 + c * 128 + (n & 7) * 16);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
-          for (int k = 0; k < 4; ++k) { const float2 f = __bfloat1622float2(h2[k]); acc = fmaf(f.x, f.x, fmaf(f.y, f.y, acc)); }
+      const int split = window_split_bits(g, (int)((a.win0 + wl) % g.nW));
+      // key extension rows (independent of the loaded data)
+      for (int n = pt_; n < Wn::KCOLS; n += kA7PrepWarps * 32) {
+        const int l = n >> 3, pw = n & 7;
+        int rt = 0, rh = 0, rw = 0;
+        if (l < Wn::KLINES && pw < 7) {
+          rt = w7_region(split & 1, l / 7, cut_t);
+          rh = w7_region(split & 2, l % 7, cut_h);
+          rw = w7_region(split & 4, pw, cut_w);
         }
-        kx = fmaxf(kx, acc);
+        const float yt = (split & 1) ? -256.f * (float)(1 - 2 * rt) : 0.f;
+        const float yh = (split & 2) ? -256.f * (float)(1 - 2 * rh) : 0.f;
+        const float yw = (split & 4) ? -256.f * (float)(1 - 2 * rw) : 0.f;
+        const float z = -256.f * (float)(rt + rh + rw);
+        *reinterpret_cast<uint4*>(sKX + (n >> 3) * 128 + (n & 7) * 16) =
+            make_uint4(pack_bf16x2(1.f, z), pack_bf16x2(yt, yh), pack_bf16x2(yw, 0.f), 0u);
       }
-      for (int off = 16; off > 0; off >>= 1) kx = fmaxf(kx, __shfl_xor_sync(0xffffffffu, kx, off));
-      if (lane == 0) s_kpart[warp] = kx;
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (s_abort) break;
-    float kmax = 0.f;
-    {
-      float mx = s_part[0], kx = s_kpart[0];
+      if (!mbar_wait(&ld_full[X], use & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      if (s_abort) break;
+      // key norms
+      {
+        float kx = 0.f;
+        for (int n = pt_; n < Wn::KLINES * 8; n += kA7PrepWarps * 32) {
+          if ((n & 7) == 7) continue;
+          float acc = 0.f;
 #pragma unroll
-      for (int k = 1; k < kAttn7Threads / 32; ++k) { mx = fmaxf(mx, s_part[k]); kx = fmaxf(kx, s_kpart[k]); }
-      bmax = mx;
-      kmax = sqrtf(kx);
+          for (int c = 0; c < 4; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(sK + (n >> 3) * 512 + c * 128 + (n & 7) * 16);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = __bfloat1622float2(h2[k]);
+              acc = fmaf(f.x, f.x, fmaf(f.y, f.y, acc));
+            }
+          }
+          kx = fmaxf(kx, acc);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kx = fmaxf(kx, __shfl_xor_sync(0xffffffffu, kx, off));
+        if (lane == 0) red[4 + warp] = kx;
+      }
+      mbar_arrive(prep_sync);
+      if (!mbar_wait(prep_sync, ph_sync, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      ph_sync ^= 1;
+      if (s_abort) break;
+      if (new_table) {
+        tab_max[X] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        tab_head[X] = h;
+      }
+      const float kmax = sqrtf(fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+      const float bmax = tab_max[X];
+      // query extension rows
+      for (int i = pt_; i < Wn::QXROWS; i += kA7PrepWarps * 32) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (i < Wn::N) {
+          float qq = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 qv = *reinterpret_cast<const uint4*>(sQ + (i >> 3) * 512 + c * 128 + (i & 7) * 16);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = __bfloat1622float2(h2[k]);
+              qq = fmaf(f.x, f.x, fmaf(f.y, f.y, qq));
+            }
+          }
+          float m = sqrtf(qq) * kmax + bmax + 1.0f;
+          if (!(m < 3.0e38f)) m = 0.f;  // the row sum then fails the range test: exact path
+          const int pt = i / 49, ph = (i / 7) % 7, pw = i % 7;
+          const float rt = 0.5f * (float)w7_region(split & 1, pt, cut_t);
+          const float rh = 0.5f * (float)w7_region(split & 2, ph, cut_h);
+          const float rw = 0.5f * (float)w7_region(split & 4, pw, cut_w);
+          w.x = bf16_bits(__float2bfloat16_rd(-0.5f * m)) | (bf16_bits(__float2bfloat16(0.5f)) << 16);
+          w.y = pack_bf16x2(rt, rh);
+          w.z = pack_bf16x2(rw, 0.f);
+        }
+        *reinterpret_cast<uint4*>(sQX + (i >> 3) * 128 + (i & 7) * 16) = w;
+      }
+      // Padding rows of the v slab (8th key of each line, whole padding lines)
+      // must be finite for O = P V: zero them (four 16-byte pieces per row).
+      {
+        constexpr int ndummy = Wn::KLINES + (Wn::LINES - Wn::KLINES) * 8;
+        for (int k = pt_; k < ndummy * 4; k += kA7PrepWarps * 32) {
+          const int d = k >> 2, chunk = k & 3;
+          const int n = d < Wn::KLINES ? d * 8 + 7 : Wn::KLINES * 8 + (d - Wn::KLINES);
+          *reinterpret_cast<uint4*>(sV + (n >> 3) * 512 + chunk * 128 + (n & 7) * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&prep_done[X]);
     }
-    const int split = window_split_bits(g, (int)(win % g.nW));
-
-#pragma unroll 1
-    for (int qt = 0; qt < Wn::QTILES; ++qt) {
-      const int i = qt * 128 + rt;
-      const bool active = qt * 128 + quarter * 32 < Wn::N;
-      const int ie = i < Wn::N ? i : Wn::N - 1;
-      const int pt_i = ie / 49, ph_i = (ie / 7) % 7, pw_i = ie % 7;
-      const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
-      uint32_t okt = 0xFFFFFFFFu, okh = 0xFFFFFFFFu, okw = 0x7Fu;
-      {
-        const int cut_t = Wn::P - g.sh[0], cut_h = 7 - g.sh[1], cut_w = 7 - g.sh[2];
-        const bool rt_ = pt_i >= cut_t, rh_ = ph_i >= cut_h, rw_ = pw_i >= cut_w;
-        if (split & 1) {
-          okt = 0;
-          for (int k = 0; k < Wn::P; ++k) okt |= (uint32_t)((k >= cut_t) == rt_) << k;
+  } else if (warp == kA7MmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0 && ntiles > 0) {
+      long long tau[2] = {0, 1};
+      int blk[2] = {0, 0};
+      uint32_t ph_p[2] = {0, 0};
+      const uint32_t s_base = smem_u32(smem);
+      auto issue_s = [&](int w) {
+        const long long t = tau[w];
+        const long long jj = t / Wn::QTILES;
+        const int qt = (int)(t % Wn::QTILES);
+        const int X = (int)(jj & 1);
+        const int b = blk[w];
+        if (b == 0 && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) {
+          s_abort = 1;
+          return;
         }
-        if (split & 2) {
-          okh = 0;
-          for (int k = 0; k < 7; ++k) okh |= (uint32_t)((k >= cut_h) == rh_) << k;
-        }
-        if (split & 4) {
-          okw = 0;
-          for (int k = 0; k < 7; ++k) okw |= (uint32_t)((k >= cut_w) == rw_) << k;
-        }
-      }
-      float mrow[3] = {-INFINITY, -INFINITY, -INFINITY}, lrow[3] = {0.f, 0.f, 0.f};
-      float mref = 0.f;
-      {
-        float qq = 0.f;
-        for (int c = 0; c < 4; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(sQ + (ie >> 3) * 512 + c * 128 + (ie & 7) * 16);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
-          for (int k = 0; k < 4; ++k) { const float2 f = __bfloat1622float2(h2[k]); qq = fmaf(f.x, f.x, fmaf(f.y, f.y, qq)); }
-        }
-        mref = sqrtf(qq) * kmax + bmax + 1.0f;
-        if (!(mref < 3.0e38f)) mref = 0.f;
-      }
-
-      if (tid == 0) {
         tc_fence_after();
+        const int row0 = w7_tile_row0<Wn>(qt, jj);
+        const int l0 = b * Wn::BL;
+        const int nl = b < Wn::NBLK - 1 ? Wn::BL : Wn::LAST;
+        const uint32_t idesc = idesc_bf16(128, nl * 8, 0, 0);
+        const uint32_t dS = tmem + (uint32_t)w * kA7GroupCols;
+        const uint32_t qx = s_base + Wn::OFF_QX + X * Wn::QXB + (row0 >> 3) * 128;
+        const uint32_t kx = s_base + Wn::OFF_KX + X * Wn::KXB + l0 * 128;
+        umma_ss(dS, smem_desc(qx, 0, 128), smem_desc(kx, 0, 128), idesc, 0);
+        const uint32_t qa = s_base + Wn::OFF_Q + X * Wn::QB + (row0 >> 3) * 512;
+        const uint32_t ka = s_base + Wn::OFF_K + X * Wn::KB + l0 * 512;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          umma_ss(tmem, smem_desc(qaddr + qt * 8192 + ks * 256, 128, 512), smem_desc(kaddr + ks * 256, 128, 512),
-                  idesc_bf16(128, w7_block_lines<Wn>(0) * 8, 0, 0), ks);
-        umma_commit(bar_s);
-      }
-#pragma unroll 1
-      for (int b = 0; b < Wn::NBLK; ++b) {
-        const int nl = w7_block_lines<Wn>(b);
-        const int l0 = b * Wn::BL + half * (nl / 2), l1 = l0 + nl / 2;
-        const uint32_t tcol = trow + half * (nl / 2) * 8;
-        if (!mbar_wait(bar_s, ph_s, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
-        ph_s ^= 1;
-        __syncthreads();
+          umma_ss(dS, smem_desc(qa + ks * 256, 128, 512), smem_desc(ka + ks * 256, 128, 512), idesc, 1);
+        umma_commit(&s_full[w]);
+      };
+      auto issue_pv = [&](int w) {
+        if (!mbar_wait(&p_full[w], ph_p[w], a.ctx.err, kErrWaitMma, lim)) {
+          s_abort = 1;
+          return;
+        }
+        ph_p[w] ^= 1;
         tc_fence_after();
-        if (active && !s_abort) {
-          const float mb = mref;
-          const float mm = mref;
-          lrow[b] = split ? w7_pass2<Wn, true>(tcol, l0, l1, tb_row, mm, okt, okh, okw)
-                          : w7_pass2<Wn, false>(tcol, l0, l1, tb_row, mm, okt, okh, okw);
-          mrow[b] = mb;
+        const long long t = tau[w];
+        const long long jj = t / Wn::QTILES;
+        const int X = (int)(jj & 1);
+        const int b = blk[w];
+        const int l0 = b * Wn::BL;
+        const int nl = b < Wn::NBLK - 1 ? Wn::BL : Wn::LAST;
+        const uint32_t dS = tmem + (uint32_t)w * kA7GroupCols;
+        const uint32_t vbase = s_base + Wn::OFF_V + X * Wn::KB;
+        const uint64_t ones = smem_desc(s_base + Wn::OFF_ONES, 256, 128);
+        for (int ks = 0; ks < nl / 2; ++ks) {
+          const uint32_t acc = (b > 0 || ks > 0) ? 1u : 0u;
+          umma_ts(dS + kA7OCol, dS + 8 * ks, smem_desc(vbase + (l0 + 2 * ks) * 512, 512, 128),
+                  idesc_bf16(128, kD, 0, 1), acc);
+          umma_ts(dS + kA7LCol, dS + 8 * ks, ones, idesc_bf16(128, 16, 0, 1), acc);
+        }
+        if (b == Wn::NBLK - 1) {
+          umma_commit(&o_full[w]);
+          umma_commit(&buf_free[X]);
+          tau[w] += 2;
+          blk[w] = 0;
+        } else {
+          blk[w] = b + 1;
+        }
+      };
+      issue_s(0);
+      if (ntiles > 1 && !s_abort) issue_s(1);
+      while (!s_abort) {
+        bool any = false;
+        for (int w = 0; w < 2 && !s_abort; ++w) {
+          if (tau[w] >= ntiles) continue;
+          any = true;
+          issue_pv(w);
+          if (!s_abort && tau[w] < ntiles) issue_s(w);
+        }
+        if (!any) break;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax groups
+    const int grp = (warp - kA7Soft0) >> 2;
+    const int qd = warp & 3;  // TMEM lane quarter this warp may access
+    const uint32_t tS = tmem + (uint32_t)grp * kA7GroupCols + ((uint32_t)(qd * 32) << 16);
+    uint32_t ph_s = 0, ph_o = 0;
+    for (long long t = grp; t < ntiles; t += 2) {
+      const long long jj = t / Wn::QTILES;
+      const int qt = (int)(t % Wn::QTILES);
+      const int X = (int)(jj & 1);
+      const long long item = (long long)blockIdx.x + jj * gridDim.x;
+      const int h = (int)(item / a.nwin);
+      const long long wl = item % a.nwin;
+      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      const int row0 = w7_tile_row0<Wn>(qt, jj);
+      const int wrow = row0 + qd * 32;
+      const int i = wrow + lane;
+      const bool active = i >= qt * 128 && i < Wn::N;
+      const bool warp_active = wrow + 31 >= qt * 128 && wrow < Wn::N;
+      const int ie = i < qt * 128 ? qt * 128 : (i < Wn::N ? i : Wn::N - 1);
+      const int pt_i = ie / 49, ph_i = (ie / 7) % 7, pw_i = ie % 7;
+      const float* sT = reinterpret_cast<const float*>(smem + Wn::OFF_T + X * Wn::TB);
+      const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
+#pragma unroll
+      for (int b = 0; b < Wn::NBLK; ++b) {
+        if (!s_abort && !mbar_wait(&s_full[grp], ph_s, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+        ph_s ^= 1;
+        tc_fence_after();
+        if (warp_active && !s_abort) {
+          if (b < Wn::NBLK - 1)
+            w7_block<Wn, Wn::BL>(tS, b * Wn::BL, tb_row);
+          else
+            w7_block<Wn, Wn::LAST>(tS, b * Wn::BL, tb_row);
         }
         tmem_wait_st();
         tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && !s_abort) {
-          tc_fence_after();
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int key0 = (b * Wn::BL + hf * (nl / 2)) * 8;
-            for (int ks = 0; ks < nl / 4; ++ks)
-              umma_ts(tmem + kOCol + 32 * b, tmem + hf * (nl / 2) * 8 + 8 * ks,
-                      smem_desc(vaddr + ((key0 + 16 * ks) >> 3) * 512, 512, 128), idesc_bf16(128, kD, 0, 1),
-                      (hf | ks) != 0);
-          }
-          if (b + 1 < Wn::NBLK) {
-            const int nkey0 = (b + 1) * Wn::BL * 8;
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-              umma_ss(tmem, smem_desc(qaddr + qt * 8192 + ks * 256, 128, 512),
-                      smem_desc(kaddr + (nkey0 >> 3) * 512 + ks * 256, 128, 512),
-                      idesc_bf16(128, w7_block_lines<Wn>(b + 1) * 8, 0, 0), ks);
-            umma_commit(bar_s);
-          } else {
-            umma_commit(bar_o);
-          }
-        }
-        if (s_abort) break;
+        mbar_arrive(&p_full[grp]);
       }
-      if (s_abort) break;
-      if (!mbar_wait(bar_o, ph_o, a.ctx.err, kErrWaitMma, a.ctx.wait_limit)) s_abort = 1;
+      if (!s_abort && !mbar_wait(&o_full[grp], ph_o, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
       ph_o ^= 1;
-      __syncthreads();
       tc_fence_after();
-      if (active && !s_abort) {
-#pragma unroll
-        for (int b = 0; b < Wn::NBLK; ++b) xsum[(half * 3 + b) * 128 + rt] = lrow[b];
-        named_bar(1 + quarter, 64);
-        float M = mrow[0];
-#pragma unroll
-        for (int b = 1; b < Wn::NBLK; ++b) M = fmaxf(M, mrow[b]);
-        float alpha[3], L = 0.f;
-#pragma unroll
-        for (int b = 0; b < Wn::NBLK; ++b) {
-          alpha[b] = mrow[b] == -INFINITY ? 0.f : ex2_approx(mrow[b] - M);
-          L += alpha[b] * (xsum[b * 128 + rt] + xsum[(3 + b) * 128 + rt]);
-        }
-        const float inv = 1.0f / L;
-        float o[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) o[k] = 0.f;
-#pragma unroll
-        for (int b = 0; b < Wn::NBLK; ++b) {
-          uint32_t u[16];
-          tmem_ld16(trow + kOCol + 32 * b + 16 * half, u);
-          tmem_wait_ld();
-          const float f = alpha[b] * inv;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) o[k] = fmaf(__uint_as_float(u[k]), f, o[k]);
-        }
-        if (i < Wn::N) {
+      if (warp_active && !s_abort) {
+        uint32_t o[32];
+        uint32_t lr[1];
+        tmem_ld32(tS + kA7OCol, o);
+        lr[0] = tmem_ld1(tS + kA7LCol);
+        tmem_wait_ld_keep(o);
+        tmem_wait_ld_keep(lr);
+        const float L = __uint_as_float(lr[0]);
+        if (active) {
           __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD;
-          if (L >= a.exact_below) {  // the common case
-            dst += 16 * half;
-            reinterpret_cast<uint4*>(dst)[0] =
-                make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                           pack_bf16x2(o[6], o[7]));
-            reinterpret_cast<uint4*>(dst)[1] =
-                make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
-                           pack_bf16x2(o[14], o[15]));
-          } else if (half == 0) {  // the reference was too loose for this row: recompute it exactly
-            float oe[32];
-            w7_exact_row<Wn>(sQ, sK, sV, tb_row, i, okt, okh, okw, oe);
+          if (L >= a.exact_below && L <= 3.0e38f) {  // the common case
+            const float inv = 1.0f / L;
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd)
-              reinterpret_cast<uint4*>(dst)[qd] =
-                  make_uint4(pack_bf16x2(oe[8 * qd + 0], oe[8 * qd + 1]), pack_bf16x2(oe[8 * qd + 2], oe[8 * qd + 3]),
-                             pack_bf16x2(oe[8 * qd + 4], oe[8 * qd + 5]), pack_bf16x2(oe[8 * qd + 6], oe[8 * qd + 7]));
+            for (int c = 0; c < 4; ++c)
+              reinterpret_cast<uint4*>(dst)[c] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+          } else {  // the reference was too loose for this row (or overflowed): recompute it exactly
+            const int split = window_split_bits(g, (int)((a.win0 + wl) % g.nW));
+            uint32_t okt = 0xFFFFFFFFu, okh = 0xFFFFFFFFu, okw = 0x7Fu;
+            if (split & 1) {
+              okt = 0;
+              for (int k = 0; k < Wn::P; ++k) okt |= (uint32_t)((k >= cut_t) == (pt_i >= cut_t)) << k;
+            }
+            if (split & 2) {
+              okh = 0;
+              for (int k = 0; k < 7; ++k) okh |= (uint32_t)((k >= cut_h) == (ph_i >= cut_h)) << k;
+            }
+            if (split & 4) {
+              okw = 0;
+              for (int k = 0; k < 7; ++k) okw |= (uint32_t)((k >= cut_w) == (pw_i >= cut_w)) << k;
+            }
+            float oe[32];
+            w7_exact_row<Wn>(smem + Wn::OFF_Q + X * Wn::QB, smem + Wn::OFF_K + X * Wn::KB,
+                             smem + Wn::OFF_V + X * Wn::KB, tb_row, i, okt, okh, okw, oe);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              reinterpret_cast<uint4*>(dst)[c] =
+                  make_uint4(pack_bf16x2(oe[8 * c + 0], oe[8 * c + 1]), pack_bf16x2(oe[8 * c + 2], oe[8 * c + 3]),
+                             pack_bf16x2(oe[8 * c + 4], oe[8 * c + 5]), pack_bf16x2(oe[8 * c + 6], oe[8 * c + 7]));
           }
         }
       }
       tc_fence_before();
-      __syncthreads();
-      if (s_abort) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&buf_free[X]);
     }
-    if (s_abort) break;
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kA7MmaWarp) tmem_dealloc(tmem, kA7TmemCols);
 }
 
 template <class Wn>
@@ -1301,10 +1414,10 @@ cudaError_t launch_attention7(const AttnArgs& a, cudaStream_t st) {
       cudaFuncSetAttribute(attention7_kernel<Wn>, cudaFuncAttributeMaxDynamicSharedMemorySize, Wn::SMEM);
   if (e != cudaSuccess) return e;
   const long long items = a.nwin * a.g.heads;
-  long long grid = 2LL * sms;
+  long long grid = sms;
   if (grid > items) grid = items;
   prof_begin(kKindAttn, st);
-  attention7_kernel<Wn><<<(unsigned)grid, kAttn7Threads, Wn::SMEM, st>>>(a);
+  attention7_kernel<Wn><<<(unsigned)grid, kA7Threads, Wn::SMEM, st>>>(a);
   prof_end(kKindAttn, st);
   count_launch();
   return cudaGetLastError();

@@ -114,6 +114,23 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Wait for this thread's TMEM loads, then pass the destination registers
+// through empty volatile statements so that no use of them is scheduled
+// before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_keep(uint32_t (&r)[N]) {
+  tmem_wait_ld();
+#pragma unroll
+  for (int k = 0; k < N; ++k) asm volatile("" : "+r"(r[k]));
+}
+
+// 32 lanes x 1 column.
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns: thread t of the warp receives
