@@ -843,20 +843,20 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 
 // ============================================================================ attention, (P,7,7) windows
 //
-// Persistent, warp-specialised kernel, one CTA per SM, 416 threads:
-//   warps 0-3    preparation of (window, head) items, two in flight: bulk loads
+// Persistent, warp-specialised kernel, one CTA per SM, 384 threads:
+//   warps 0-2    preparation of (window, head) items, two in flight: bulk loads
 //                of the q / k / v slabs, the head's bias table in log2 units,
 //                key norms, the extension rows of the score MMA (below), zeroed
 //                v padding;
-//   warp 4       tcgen05.mma issue (one thread), serving the two softmax
-//                groups in turn;
-//   warps 5-8 and 9-12   softmax groups 0 and 1: group g owns this CTA's query
+//   warp 3       tcgen05.mma issue (one elected lane), serving the two
+//                softmax groups in turn;
+//   warps 4-7 and 8-11   softmax groups 0 and 1: group g owns this CTA's query
 //                tiles g, g + 2, g + 4, ... (128-row tiles, items in order).
 // Keys are taken in blocks of up to 20 lines of 8 columns (the 7 keys of one
 // (pt, ph) line and a padding column). Per block: S = q k^T into the group's
-// TMEM columns, the group turns S into bf16 P in place, then O += P v and
-// l += P 1 on the tensor core. While one group exponentiates, the tensor core
-// works for the other.
+// TMEM columns, the group turns S into bf16 P in place (summing p as it goes),
+// then O += P v on the tensor core. While one group exponentiates, the tensor
+// core works for the other.
 //
 // Softmax reference. Every query row i uses one reference for all its keys,
 //   m_i = |q_i| * max_j |k_j| + max(bias) + 1   (log2 units, q pre-scaled),
@@ -877,14 +877,13 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 // the same -m_i (identical step inputs), masked keys end at least 257 below
 // the reference and exponentiate to exactly 0. -m_i/2 is rounded towards
 // -inf, so the effective reference is never below m_i.
-constexpr int kA7Threads = 416;
-constexpr int kA7PrepWarps = 4;
-constexpr int kA7MmaWarp = 4;
-constexpr int kA7Soft0 = 5;
+constexpr int kA7Threads = 384;
+constexpr int kA7PrepWarps = 3;
+constexpr int kA7MmaWarp = 3;
+constexpr int kA7Soft0 = 4;
 constexpr uint32_t kA7TmemCols = 512;
-constexpr uint32_t kA7GroupCols = 256;  // per group: S / P [0, 160), O [160, 192), l [192, 208)
+constexpr uint32_t kA7GroupCols = 256;  // per group: S / P [0, 160), O [160, 192)
 constexpr uint32_t kA7OCol = 160;
-constexpr uint32_t kA7LCol = 192;
 
 template <int P_>
 struct W7 {
@@ -916,8 +915,7 @@ struct W7 {
   static constexpr int OFF_QX = OFF_V + 2 * KB;
   static constexpr int OFF_KX = OFF_QX + 2 * QXB;
   static constexpr int OFF_T = OFF_KX + 2 * KXB;
-  static constexpr int OFF_ONES = OFF_T + 2 * TB;
-  static constexpr int OFF_BAR = OFF_ONES + 512;
+  static constexpr int OFF_BAR = OFF_T + 2 * TB;
   static constexpr int SMEM = OFF_BAR + 256;
   static_assert(NBLK <= 3 && BL <= 20 && LAST > 0 && LAST % 2 == 0, "key blocks must fit 160 TMEM columns");
   // a tile's operand rows beyond the q slab read the following buffers (their
@@ -939,7 +937,8 @@ __device__ __forceinline__ int w7_region(int split_bit, int c, int cut) { return
 // the 7 keys of a real line, 0 for padding columns and padding lines; packed
 // into 8 bf16x2 words.
 template <class Wn>
-__device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], const float* tb_row, uint32_t* pk) {
+__device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], const float* tb_row, uint32_t* pk,
+                                             float& sum) {
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     const int line = l + c;
@@ -953,6 +952,7 @@ __device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], con
       for (int pw = 0; pw < 7; ++pw) p[pw] = 0.f;
     }
     p[7] = 0.f;
+    sum += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + p[6]);
 #pragma unroll
     for (int k = 0; k < 4; ++k) pk[c * 4 + k] = pack_bf16x2(p[2 * k], p[2 * k + 1]);
   }
@@ -961,8 +961,10 @@ __device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], con
 // One key block of NL lines starting at line L0 for this thread's query row:
 // S (TMEM columns from tS) -> bf16 P written in place (4 columns per line),
 // the next line pair's load in flight while the current one is processed.
+// Returns the block's sum of p.
 template <class Wn, int NL>
-__device__ __forceinline__ void w7_block(uint32_t tS, int L0, const float* tb_row) {
+__device__ __forceinline__ float w7_block(uint32_t tS, int L0, const float* tb_row) {
+  float sum = 0.f;
   uint32_t ua[16], ub[16];
   tmem_ld16(tS, ua);
   tmem_wait_ld_keep(ua);
@@ -971,16 +973,48 @@ __device__ __forceinline__ void w7_block(uint32_t tS, int L0, const float* tb_ro
     uint32_t pk[8];
     if ((k & 1) == 0) {
       if (k + 1 < NL / 2) tmem_ld16(tS + 16 * (k + 1), ub);
-      w7_line_pair<Wn>(L0 + 2 * k, ua, tb_row, pk);
+      w7_line_pair<Wn>(L0 + 2 * k, ua, tb_row, pk, sum);
       tmem_st8(tS + 8 * k, pk);
       if (k + 1 < NL / 2) tmem_wait_ld_keep(ub);
     } else {
       if (k + 1 < NL / 2) tmem_ld16(tS + 16 * (k + 1), ua);
-      w7_line_pair<Wn>(L0 + 2 * k, ub, tb_row, pk);
+      w7_line_pair<Wn>(L0 + 2 * k, ub, tb_row, pk, sum);
       tmem_st8(tS + 8 * k, pk);
       if (k + 1 < NL / 2) tmem_wait_ld_keep(ua);
     }
   }
+  return sum;
+}
+
+// One elected lane of a converged warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Score MMA of one key block of NL lines: the extension step first (it
+// overwrites the accumulator), then the two q . k steps. Descriptors point at
+// the tile's first q row and the block's first key; one K step of 16 columns is
+// 256 bytes (16 in descriptor units).
+template <int NL>
+__device__ __forceinline__ void w7_issue_s(uint32_t dS, uint64_t qxd, uint64_t kxd, uint64_t qd, uint64_t kd) {
+  constexpr uint32_t id = idesc_bf16(128, NL * 8, 0, 0);
+  umma_ss(dS, qxd, kxd, id, 0u);
+  umma_ss(dS, qd, kd, id, 1u);
+  umma_ss(dS, qd + 16, kd + 16, id, 1u);
+}
+
+// O (+)= P v for one key block of NL lines: 16 keys (8 P columns, 1 KB of v)
+// per MMA.
+template <int NL>
+__device__ __forceinline__ void w7_issue_pv(uint32_t dO, uint32_t dP, uint64_t vd, bool first) {
+  constexpr uint32_t id = idesc_bf16(128, kD, 0, 1);
+#pragma unroll
+  for (int ks = 0; ks < NL / 2; ++ks)
+    umma_ts(dO, dP + 8 * ks, vd + (uint64_t)(64 * ks), id, (first && ks == 0) ? 0u : 1u);
 }
 
 // Exact recomputation of one query row (rare path, see the reference rule
@@ -1051,12 +1085,12 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Wn::OFF_BAR);
   uint64_t* ld_full = bars;        // [buffer] q / k / v bytes landed
-  uint64_t* prep_done = bars + 2;  // [buffer] item prepared (128 arrivals)
+  uint64_t* prep_done = bars + 2;  // [buffer] item prepared (one arrival per preparation thread)
   uint64_t* buf_free = bars + 4;   // [buffer] item finished (MMA commit + 4 warps per tile)
   uint64_t* s_full = bars + 6;     // [group] S of the group's current block in TMEM
   uint64_t* p_full = bars + 8;     // [group] P written (128 arrivals)
   uint64_t* o_full = bars + 10;    // [group] O and l of the group's tile complete
-  uint64_t* prep_sync = bars + 12; // preparation warps' own barrier (128 arrivals)
+  uint64_t* prep_sync = bars + 12; // preparation warps' own barrier
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
   float* s_red = reinterpret_cast<float*>(smem + Wn::OFF_BAR + 128);  // [buffer][8]
   __shared__ volatile int s_abort;
@@ -1083,13 +1117,6 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     fence_mbar_init();
     s_abort = 0;
   }
-  // Ones operand of l = P 1: 16 keys x 16 columns, MN-major (K-group stride
-  // 256 B, N-group stride 128 B), column 0 = 1.
-  if (tid < 32) {
-    const int ngroup = (tid >> 3) & 1;
-    reinterpret_cast<uint4*>(smem + Wn::OFF_ONES)[tid] = make_uint4(ngroup == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
-  }
-  fence_proxy_async_smem();
   if (warp == kA7MmaWarp) {
     tmem_alloc(s_tmem, kA7TmemCols);
     tmem_relinquish();
@@ -1102,8 +1129,8 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
   if (warp < kA7PrepWarps) {
     // ------------------------------------------------------------ preparation
     const int pt_ = tid;
-    int tab_head[2] = {-1, -1};
-    float tab_max[2] = {0.f, 0.f};
+    int tab_head0 = -1, tab_head1 = -1;
+    float tab_max0 = 0.f, tab_max1 = 0.f;
     uint32_t ph_sync = 0;
     long long j = 0;
     for (long long item = blockIdx.x; item < nitems; item += gridDim.x, ++j) {
@@ -1127,7 +1154,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
         bulk_g2s(sK, base + (size_t)Wn::QSLAB * kD, Wn::KB, &ld_full[X]);
         bulk_g2s(sV, base + (size_t)(Wn::QSLAB + Wn::KCOLS) * kD, Wn::KB, &ld_full[X]);
       }
-      const bool new_table = h != tab_head[X];
+      const bool new_table = h != (X ? tab_head1 : tab_head0);
       if (new_table) {
         float mx = -INFINITY;
         for (int k = pt_; k < Wn::TABLE; k += kA7PrepWarps * 32) {
@@ -1137,7 +1164,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        if (lane == 0) red[warp] = mx;
+        if (lane == 0) red[warp] = mx;  // red[0 .. kA7PrepWarps)
       }
       const int split = window_split_bits(g, (int)((a.win0 + wl) % g.nW));
       // key extension rows (independent of the loaded data)
@@ -1178,18 +1205,29 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) kx = fmaxf(kx, __shfl_xor_sync(0xffffffffu, kx, off));
-        if (lane == 0) red[4 + warp] = kx;
+        if (lane == 0) red[4 + warp] = kx;  // red[4 .. 4 + kA7PrepWarps)
       }
       mbar_arrive(prep_sync);
       if (!mbar_wait(prep_sync, ph_sync, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
       ph_sync ^= 1;
       if (s_abort) break;
       if (new_table) {
-        tab_max[X] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        tab_head[X] = h;
+        float mx = red[0];
+#pragma unroll
+        for (int k = 1; k < kA7PrepWarps; ++k) mx = fmaxf(mx, red[k]);
+        if (X) {
+          tab_max1 = mx;
+          tab_head1 = h;
+        } else {
+          tab_max0 = mx;
+          tab_head0 = h;
+        }
       }
-      const float kmax = sqrtf(fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
-      const float bmax = tab_max[X];
+      float kx2 = red[4];
+#pragma unroll
+      for (int k = 1; k < kA7PrepWarps; ++k) kx2 = fmaxf(kx2, red[4 + k]);
+      const float kmax = sqrtf(kx2);
+      const float bmax = X ? tab_max1 : tab_max0;
       // query extension rows
       for (int i = pt_; i < Wn::QXROWS; i += kA7PrepWarps * 32) {
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -1232,79 +1270,92 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     }
   } else if (warp == kA7MmaWarp) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0 && ntiles > 0) {
-      long long tau[2] = {0, 1};
-      int blk[2] = {0, 0};
-      uint32_t ph_p[2] = {0, 0};
+    // The whole warp walks the schedule (waits included); one elected lane
+    // issues. Per buffer the operand descriptors are fixed; tiles and blocks
+    // only add offsets (descriptor units of 16 bytes).
+    if (ntiles > 0) {
       const uint32_t s_base = smem_u32(smem);
-      auto issue_s = [&](int w) {
-        const long long t = tau[w];
+      const uint64_t qxd0 = smem_desc(s_base + Wn::OFF_QX, 0, 128);
+      const uint64_t kxd0 = smem_desc(s_base + Wn::OFF_KX, 0, 128);
+      const uint64_t qd0 = smem_desc(s_base + Wn::OFF_Q, 128, 512);
+      const uint64_t kd0 = smem_desc(s_base + Wn::OFF_K, 128, 512);
+      const uint64_t vd0 = smem_desc(s_base + Wn::OFF_V, 512, 128);
+      // buffer X adds X * (buffer bytes) / 16
+      auto issue_s = [&](int w, long long t, int b) {
         const long long jj = t / Wn::QTILES;
         const int qt = (int)(t % Wn::QTILES);
-        const int X = (int)(jj & 1);
-        const int b = blk[w];
+        const uint32_t X = (uint32_t)(jj & 1);
         if (b == 0 && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) {
           s_abort = 1;
           return;
         }
         tc_fence_after();
-        const int row0 = w7_tile_row0<Wn>(qt, jj);
-        const int l0 = b * Wn::BL;
-        const int nl = b < Wn::NBLK - 1 ? Wn::BL : Wn::LAST;
-        const uint32_t idesc = idesc_bf16(128, nl * 8, 0, 0);
+        const uint32_t row0 = (uint32_t)w7_tile_row0<Wn>(qt, jj);
+        const uint32_t l0 = (uint32_t)(b * Wn::BL);
         const uint32_t dS = tmem + (uint32_t)w * kA7GroupCols;
-        const uint32_t qx = s_base + Wn::OFF_QX + X * Wn::QXB + (row0 >> 3) * 128;
-        const uint32_t kx = s_base + Wn::OFF_KX + X * Wn::KXB + l0 * 128;
-        umma_ss(dS, smem_desc(qx, 0, 128), smem_desc(kx, 0, 128), idesc, 0);
-        const uint32_t qa = s_base + Wn::OFF_Q + X * Wn::QB + (row0 >> 3) * 512;
-        const uint32_t ka = s_base + Wn::OFF_K + X * Wn::KB + l0 * 512;
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-          umma_ss(dS, smem_desc(qa + ks * 256, 128, 512), smem_desc(ka + ks * 256, 128, 512), idesc, 1);
-        umma_commit(&s_full[w]);
+        // q row r: 16 B of extension (r units), 64 B of q (4 r units); key line l: 128 B / 512 B
+        const uint64_t ax = qxd0 + X * (Wn::QXB / 16) + row0;
+        const uint64_t aq = qd0 + X * (Wn::QB / 16) + 4 * row0;
+        const uint64_t bx = kxd0 + X * (Wn::KXB / 16) + 8 * l0;
+        const uint64_t bk = kd0 + X * (Wn::KB / 16) + 32 * l0;
+        if (elect_one()) {
+          if (b == Wn::NBLK - 1)
+            w7_issue_s<Wn::LAST>(dS, ax, bx, aq, bk);
+          else
+            w7_issue_s<Wn::BL>(dS, ax, bx, aq, bk);
+          umma_commit(&s_full[w]);
+        }
+        __syncwarp();
       };
-      auto issue_pv = [&](int w) {
-        if (!mbar_wait(&p_full[w], ph_p[w], a.ctx.err, kErrWaitMma, lim)) {
+      // returns true when the tile is complete
+      auto issue_pv = [&](int w, long long t, int b, uint32_t& ph) -> bool {
+        if (!mbar_wait(&p_full[w], ph, a.ctx.err, kErrWaitMma, lim)) {
           s_abort = 1;
-          return;
+          return false;
         }
-        ph_p[w] ^= 1;
+        ph ^= 1;
         tc_fence_after();
-        const long long t = tau[w];
-        const long long jj = t / Wn::QTILES;
-        const int X = (int)(jj & 1);
-        const int b = blk[w];
-        const int l0 = b * Wn::BL;
-        const int nl = b < Wn::NBLK - 1 ? Wn::BL : Wn::LAST;
+        const uint32_t X = (uint32_t)((t / Wn::QTILES) & 1);
         const uint32_t dS = tmem + (uint32_t)w * kA7GroupCols;
-        const uint32_t vbase = s_base + Wn::OFF_V + X * Wn::KB;
-        const uint64_t ones = smem_desc(s_base + Wn::OFF_ONES, 256, 128);
-        for (int ks = 0; ks < nl / 2; ++ks) {
-          const uint32_t acc = (b > 0 || ks > 0) ? 1u : 0u;
-          umma_ts(dS + kA7OCol, dS + 8 * ks, smem_desc(vbase + (l0 + 2 * ks) * 512, 512, 128),
-                  idesc_bf16(128, kD, 0, 1), acc);
-          umma_ts(dS + kA7LCol, dS + 8 * ks, ones, idesc_bf16(128, 16, 0, 1), acc);
+        const uint64_t bv = vd0 + X * (Wn::KB / 16) + 32 * (uint32_t)(b * Wn::BL);
+        const bool last = b == Wn::NBLK - 1;
+        if (elect_one()) {
+          if (last)
+            w7_issue_pv<Wn::LAST>(dS + kA7OCol, dS, bv, b == 0);
+          else
+            w7_issue_pv<Wn::BL>(dS + kA7OCol, dS, bv, b == 0);
+          if (last) {
+            umma_commit(&o_full[w]);
+            umma_commit(&buf_free[X]);
+          }
         }
-        if (b == Wn::NBLK - 1) {
-          umma_commit(&o_full[w]);
-          umma_commit(&buf_free[X]);
-          tau[w] += 2;
-          blk[w] = 0;
-        } else {
-          blk[w] = b + 1;
-        }
+        __syncwarp();
+        return last;
       };
-      issue_s(0);
-      if (ntiles > 1 && !s_abort) issue_s(1);
-      while (!s_abort) {
-        bool any = false;
-        for (int w = 0; w < 2 && !s_abort; ++w) {
-          if (tau[w] >= ntiles) continue;
-          any = true;
-          issue_pv(w);
-          if (!s_abort && tau[w] < ntiles) issue_s(w);
+      long long t0 = 0, t1 = 1;
+      int b0 = 0, b1 = 0;
+      uint32_t ph0 = 0, ph1 = 0;
+      issue_s(0, t0, 0);
+      if (t1 < ntiles && !s_abort) issue_s(1, t1, 0);
+      while (!s_abort && (t0 < ntiles || t1 < ntiles)) {
+        if (t0 < ntiles) {
+          if (issue_pv(0, t0, b0, ph0)) {
+            t0 += 2;
+            b0 = 0;
+          } else {
+            ++b0;
+          }
+          if (!s_abort && t0 < ntiles) issue_s(0, t0, b0);
         }
-        if (!any) break;
+        if (t1 < ntiles && !s_abort) {
+          if (issue_pv(1, t1, b1, ph1)) {
+            t1 += 2;
+            b1 = 0;
+          } else {
+            ++b1;
+          }
+          if (!s_abort && t1 < ntiles) issue_s(1, t1, b1);
+        }
       }
     }
     __syncwarp();
@@ -1331,6 +1382,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       const int pt_i = ie / 49, ph_i = (ie / 7) % 7, pw_i = ie % 7;
       const float* sT = reinterpret_cast<const float*>(smem + Wn::OFF_T + X * Wn::TB);
       const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
+      float L = 0.f;
 #pragma unroll
       for (int b = 0; b < Wn::NBLK; ++b) {
         if (!s_abort && !mbar_wait(&s_full[grp], ph_s, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
@@ -1338,9 +1390,9 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
         tc_fence_after();
         if (warp_active && !s_abort) {
           if (b < Wn::NBLK - 1)
-            w7_block<Wn, Wn::BL>(tS, b * Wn::BL, tb_row);
+            L += w7_block<Wn, Wn::BL>(tS, b * Wn::BL, tb_row);
           else
-            w7_block<Wn, Wn::LAST>(tS, b * Wn::BL, tb_row);
+            L += w7_block<Wn, Wn::LAST>(tS, b * Wn::BL, tb_row);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -1351,12 +1403,8 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       tc_fence_after();
       if (warp_active && !s_abort) {
         uint32_t o[32];
-        uint32_t lr[1];
         tmem_ld32(tS + kA7OCol, o);
-        lr[0] = tmem_ld1(tS + kA7LCol);
         tmem_wait_ld_keep(o);
-        tmem_wait_ld_keep(lr);
-        const float L = __uint_as_float(lr[0]);
         if (active) {
           __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD;
           if (L >= a.exact_below && L <= 3.0e38f) {  // the common case
