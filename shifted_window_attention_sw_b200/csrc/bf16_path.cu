@@ -23,6 +23,25 @@
 
 namespace vswin {
 
+// Optional event trace of the attention kernel, compiled in only with
+// -DVSWIN_TRACE: CTA 0 records (tag, clock64) pairs per role (preparation
+// thread, lane 0 of each softmax warp), read back by
+// vswin_trace_read.
+#ifdef VSWIN_TRACE
+constexpr int kTraceRoles = 17, kTraceCap = 1024;
+__device__ long long g_trace[kTraceRoles][kTraceCap][2];
+__device__ __forceinline__ void trace_event(int role, int& n, int tag) {
+  if (blockIdx.x == 0 && n < kTraceCap) {
+    g_trace[role][n][0] = tag;
+    g_trace[role][n][1] = clock64();
+  }
+  ++n;
+}
+#define VSWIN_TRACE_EVENT(role, n, tag) trace_event(role, n, tag)
+#else
+#define VSWIN_TRACE_EVENT(role, n, tag) ((void)0)
+#endif
+
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -843,20 +862,29 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 
 // ============================================================================ attention, (P,7,7) windows
 //
-// Persistent, warp-specialised kernel, one CTA per SM, 384 threads:
-//   warps 0-2    preparation of (window, head) items, two in flight: bulk loads
+// Persistent, warp-specialised kernel, one CTA per SM, 512 threads:
+//   warps 0-3    preparation of (window, head) items, two in flight: bulk loads
 //                of the q / k / v slabs, the head's bias table in log2 units,
 //                key norms, the extension rows of the score MMA (below), zeroed
 //                v padding;
-//   warp 3       tcgen05.mma issue (one elected lane), serving the two
-//                softmax groups in turn;
-//   warps 4-7 and 8-11   softmax groups 0 and 1: group g owns this CTA's query
-//                tiles g, g + 2, g + 4, ... (128-row tiles, items in order).
-// Keys are taken in blocks of up to 20 lines of 8 columns (the 7 keys of one
+//   warps 4-15   three softmax groups of four warps (one per TMEM lane
+//                quarter); group g owns this CTA's query tiles g, g + 3, ...
+//                (128-row tiles, items in order).
+// Keys are taken in blocks of up to 12 lines of 8 columns (the 7 keys of one
 // (pt, ph) line and a padding column). Per block: S = q k^T into the group's
-// TMEM columns, the group turns S into bf16 P in place (summing p as it goes),
-// then O += P v on the tensor core. While one group exponentiates, the tensor
-// core works for the other.
+// 96 TMEM columns (q from TMEM, where the group copies its tile's q rows and
+// their extension rows, so that only keys are read from shared memory), the
+// group turns S into bf16 P in place (4 columns per line,
+// summing p as it goes), then O += P v on the tensor core. Each group issues
+// its own MMAs: after a block (a named barrier over its 128 threads) one
+// elected lane of the block's issuer warp (the warps take turns) issues the
+// block's P v and the next block's scores into the same columns (the tensor
+// core runs them in order). The softmax is bound by the latency of its
+// instruction chains, so three groups (three softmax warps per SM
+// sub-partition) keep the exponential units busy while a group waits for its
+// next scores. With three or more tiles per item, a tile's epilogue (O / l to
+// memory) runs inside the group's next tile's first block, when its P v has
+// long completed.
 //
 // Softmax reference. Every query row i uses one reference for all its keys,
 //   m_i = |q_i| * max_j |k_j| + max(bias) + 1   (log2 units, q pre-scaled),
@@ -877,13 +905,17 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 // the same -m_i (identical step inputs), masked keys end at least 257 below
 // the reference and exponentiate to exactly 0. -m_i/2 is rounded towards
 // -inf, so the effective reference is never below m_i.
-constexpr int kA7Threads = 384;
-constexpr int kA7PrepWarps = 3;
-constexpr int kA7MmaWarp = 3;
-constexpr int kA7Soft0 = 4;
+constexpr int kA7PrepWarps = 4;
+constexpr int kA7Groups = 3;
+constexpr int kA7Soft0 = kA7PrepWarps;                               // first softmax warp
+constexpr int kA7Threads = (kA7PrepWarps + 4 * kA7Groups) * 32;  // 512
 constexpr uint32_t kA7TmemCols = 512;
-constexpr uint32_t kA7GroupCols = 256;  // per group: S / P [0, 160), O [160, 192)
-constexpr uint32_t kA7OCol = 160;
+// per group: S / P [0, 96), O [96, 128), q of the tile [128, 144), its
+// extension row (twice) [144, 152)
+constexpr uint32_t kA7GroupCols = 160;
+constexpr uint32_t kA7OCol = 96;
+constexpr uint32_t kA7QCol = 128;
+constexpr uint32_t kA7QXCol = 144;
 
 template <int P_>
 struct W7 {
@@ -893,8 +925,8 @@ struct W7 {
   static constexpr int KLINES = P * 7;                       // key lines of 7 real keys
   static constexpr int KCOLS = (KLINES * 8 + 31) / 32 * 32;  // k / v slab rows (padded key columns)
   static constexpr int LINES = KCOLS / 8;
-  static constexpr int NBLK = (LINES + 19) / 20;
-  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 1) / 2 * 2;  // lines per block but the last
+  static constexpr int NBLK = (LINES + 11) / 12;
+  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 3) / 4 * 4;  // lines per block but the last
   static constexpr int LAST = LINES - (NBLK - 1) * BL;
   static constexpr int TABLE = (2 * P - 1) * 169;
   static constexpr int QTILES = (N + 127) / 128;
@@ -917,7 +949,7 @@ struct W7 {
   static constexpr int OFF_T = OFF_KX + 2 * KXB;
   static constexpr int OFF_BAR = OFF_T + 2 * TB;
   static constexpr int SMEM = OFF_BAR + 256;
-  static_assert(NBLK <= 3 && BL <= 20 && LAST > 0 && LAST % 2 == 0, "key blocks must fit 160 TMEM columns");
+  static_assert(BL <= 12 && LAST > 0 && LAST % 4 == 0, "key blocks of 4-line groups must fit 96 TMEM columns");
   // a tile's operand rows beyond the q slab read the following buffers (their
   // results land in TMEM lanes that are never used)
   static_assert(OFF_Q + QB + QXROWS * kSlabRowBytes <= SMEM, "tile rows must stay inside shared memory");
@@ -933,11 +965,29 @@ __device__ __forceinline__ int w7_tile_row0(int qt, long long jj) {
 // Region bit of slot coordinate c on an axis cut at `cut`, when the axis is split.
 __device__ __forceinline__ int w7_region(int split_bit, int c, int cut) { return (split_bit && c >= cut) ? 1 : 0; }
 
+// TMEM helpers for the softmax loop without a memory clobber (TMEM is not
+// generic memory; their order relative to each other and to the fences is
+// kept because all of them are volatile), so that shared-memory loads of the
+// bias may be scheduled across them.
+__device__ __forceinline__ void tmem_st16_reg(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
+}
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[N]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;");
+#pragma unroll
+  for (int k = 0; k < N; ++k) asm volatile("" : "+r"(r[k]));
+}
+
 // Lines l and l + 1 of a block (16 TMEM columns in u): p = 2^(s + bias) for
-// the 7 keys of a real line, 0 for padding columns and padding lines; packed
-// into 8 bf16x2 words.
+// the 7 keys of each real line, 0 for padding columns and padding lines;
+// packed into 8 bf16x2 words; the p are added to `sum`.
 template <class Wn>
-__device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], const float* tb_row, uint32_t* pk,
+__device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], const float* tb_row, uint32_t (&pk)[8],
                                              float& sum) {
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
@@ -958,63 +1008,38 @@ __device__ __forceinline__ void w7_line_pair(int l, const uint32_t (&u)[16], con
   }
 }
 
-// One key block of NL lines starting at line L0 for this thread's query row:
-// S (TMEM columns from tS) -> bf16 P written in place (4 columns per line),
-// the next line pair's load in flight while the current one is processed.
-// Returns the block's sum of p.
+__device__ __forceinline__ void tmem_st8_reg(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
+}
+
+// One key block of NL lines (even) starting at line L0 for this thread's query
+// row: S (TMEM columns from tS) -> bf16 P in place, 2 lines at a time (P of
+// lines 2k, 2k + 1 lands on columns 8k .. 8k + 7, whose scores were read
+// before), the next 2 lines' load in flight while the current ones are
+// processed. Returns the block's sum of p.
 template <class Wn, int NL>
 __device__ __forceinline__ float w7_block(uint32_t tS, int L0, const float* tb_row) {
   float sum = 0.f;
   uint32_t ua[16], ub[16];
   tmem_ld16(tS, ua);
-  tmem_wait_ld_keep(ua);
+  tmem_wait_ld_regs(ua);
 #pragma unroll
   for (int k = 0; k < NL / 2; ++k) {
     uint32_t pk[8];
     if ((k & 1) == 0) {
       if (k + 1 < NL / 2) tmem_ld16(tS + 16 * (k + 1), ub);
       w7_line_pair<Wn>(L0 + 2 * k, ua, tb_row, pk, sum);
-      tmem_st8(tS + 8 * k, pk);
-      if (k + 1 < NL / 2) tmem_wait_ld_keep(ub);
+      tmem_st8_reg(tS + 8 * k, pk);
+      if (k + 1 < NL / 2) tmem_wait_ld_regs(ub);
     } else {
       if (k + 1 < NL / 2) tmem_ld16(tS + 16 * (k + 1), ua);
       w7_line_pair<Wn>(L0 + 2 * k, ub, tb_row, pk, sum);
-      tmem_st8(tS + 8 * k, pk);
-      if (k + 1 < NL / 2) tmem_wait_ld_keep(ua);
+      tmem_st8_reg(tS + 8 * k, pk);
+      if (k + 1 < NL / 2) tmem_wait_ld_regs(ua);
     }
   }
   return sum;
-}
-
-// One elected lane of a converged warp.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
-      : "=r"(pred));
-  return pred != 0;
-}
-
-// Score MMA of one key block of NL lines: the extension step first (it
-// overwrites the accumulator), then the two q . k steps. Descriptors point at
-// the tile's first q row and the block's first key; one K step of 16 columns is
-// 256 bytes (16 in descriptor units).
-template <int NL>
-__device__ __forceinline__ void w7_issue_s(uint32_t dS, uint64_t qxd, uint64_t kxd, uint64_t qd, uint64_t kd) {
-  constexpr uint32_t id = idesc_bf16(128, NL * 8, 0, 0);
-  umma_ss(dS, qxd, kxd, id, 0u);
-  umma_ss(dS, qd, kd, id, 1u);
-  umma_ss(dS, qd + 16, kd + 16, id, 1u);
-}
-
-// O (+)= P v for one key block of NL lines: 16 keys (8 P columns, 1 KB of v)
-// per MMA.
-template <int NL>
-__device__ __forceinline__ void w7_issue_pv(uint32_t dO, uint32_t dP, uint64_t vd, bool first) {
-  constexpr uint32_t id = idesc_bf16(128, kD, 0, 1);
-#pragma unroll
-  for (int ks = 0; ks < NL / 2; ++ks)
-    umma_ts(dO, dP + 8 * ks, vd + (uint64_t)(64 * ks), id, (first && ks == 0) ? 0u : 1u);
 }
 
 // Exact recomputation of one query row (rare path, see the reference rule
@@ -1078,6 +1103,76 @@ __device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, 
   for (int d = 0; d < 32; ++d) o[d] *= inv;
 }
 
+// Named barrier over `nthreads` threads (whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One elected lane of a converged warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Score MMA of one key block of NL lines, q rows from TMEM (tq: 16 columns of
+// q, tqx: 8 columns of the extension row): the extension step first (it
+// overwrites the accumulator), then the two q . k steps. Key descriptors point
+// at the block's first key; one K step of 16 columns is 256 bytes (16 in
+// descriptor units).
+template <int NL>
+__device__ __forceinline__ void w7_issue_s(uint32_t dS, uint32_t tq, uint32_t tqx, uint64_t kxd, uint64_t kd) {
+  constexpr uint32_t id = idesc_bf16(128, NL * 8, 0, 0);
+  umma_ts(dS, tqx, kxd, id, 0u);
+  umma_ts(dS, tq, kd, id, 1u);
+  umma_ts(dS, tq + 8, kd + 16, id, 1u);
+}
+
+// O (+)= P v for one key block of NL lines: 16 keys (8 P columns, 1 KB of v)
+// per MMA.
+template <int NL>
+__device__ __forceinline__ void w7_issue_pv(uint32_t dO, uint32_t dP, uint64_t vd, bool first) {
+  constexpr uint32_t id = idesc_bf16(128, kD, 0, 1);
+#pragma unroll
+  for (int ks = 0; ks < NL / 2; ++ks)
+    umma_ts(dO, dP + 8 * ks, vd + (uint64_t)(64 * ks), id, (first && ks == 0) ? 0u : 1u);
+}
+
+// The exact path for query row i of a tile of item buffer X: mask bits of the
+// row, w7_exact_row, and the row's 32 outputs to dst.
+template <class Wn>
+__device__ __noinline__ void w7_exact_store(const AttnArgs& a, const uint8_t* smem, int X, long long wl, int i,
+                                            __nv_bfloat16* dst) {
+  const Geom& g = a.g;
+  const int pt_i = i / 49, ph_i = (i / 7) % 7, pw_i = i % 7;
+  const int cut_t = Wn::P - g.sh[0], cut_h = 7 - g.sh[1], cut_w = 7 - g.sh[2];
+  const int split = window_split_bits(g, (int)((a.win0 + wl) % g.nW));
+  uint32_t okt = 0xFFFFFFFFu, okh = 0xFFFFFFFFu, okw = 0x7Fu;
+  if (split & 1) {
+    okt = 0;
+    for (int k = 0; k < Wn::P; ++k) okt |= (uint32_t)((k >= cut_t) == (pt_i >= cut_t)) << k;
+  }
+  if (split & 2) {
+    okh = 0;
+    for (int k = 0; k < 7; ++k) okh |= (uint32_t)((k >= cut_h) == (ph_i >= cut_h)) << k;
+  }
+  if (split & 4) {
+    okw = 0;
+    for (int k = 0; k < 7; ++k) okw |= (uint32_t)((k >= cut_w) == (pw_i >= cut_w)) << k;
+  }
+  const float* sT = reinterpret_cast<const float*>(smem + Wn::OFF_T + X * Wn::TB);
+  const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
+  float oe[32];
+  w7_exact_row<Wn>(smem + Wn::OFF_Q + X * Wn::QB, smem + Wn::OFF_K + X * Wn::KB, smem + Wn::OFF_V + X * Wn::KB,
+                   tb_row, i, okt, okh, okw, oe);
+  for (int k = 0; k < 4; ++k)
+    reinterpret_cast<uint4*>(dst)[k] =
+        make_uint4(pack_bf16x2(oe[8 * k + 0], oe[8 * k + 1]), pack_bf16x2(oe[8 * k + 2], oe[8 * k + 3]),
+                   pack_bf16x2(oe[8 * k + 4], oe[8 * k + 5]), pack_bf16x2(oe[8 * k + 6], oe[8 * k + 7]));
+}
+
 __device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 v) { return (uint32_t)__bfloat16_as_ushort(v); }
 
 template <class Wn>
@@ -1087,12 +1182,11 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
   uint64_t* ld_full = bars;        // [buffer] q / k / v bytes landed
   uint64_t* prep_done = bars + 2;  // [buffer] item prepared (one arrival per preparation thread)
   uint64_t* buf_free = bars + 4;   // [buffer] item finished (MMA commit + 4 warps per tile)
-  uint64_t* s_full = bars + 6;     // [group] S of the group's current block in TMEM
-  uint64_t* p_full = bars + 8;     // [group] P written (128 arrivals)
-  uint64_t* o_full = bars + 10;    // [group] O and l of the group's tile complete
-  uint64_t* prep_sync = bars + 12; // preparation warps' own barrier
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
-  float* s_red = reinterpret_cast<float*>(smem + Wn::OFF_BAR + 128);  // [buffer][8]
+  uint64_t* s_full = bars + 6;     // [group] scores of the group's next block in TMEM
+  uint64_t* o_full = bars + 10;    // [group] O of the group's tile complete
+  uint64_t* prep_sync = bars + 14; // preparation warps' own barrier
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 15);
+  float* s_red = reinterpret_cast<float*>(smem + Wn::OFF_BAR + 192);  // [buffer][8]
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1109,15 +1203,16 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       mbar_init(&ld_full[k], 1);
       mbar_init(&prep_done[k], kA7PrepWarps * 32);
       mbar_init(&buf_free[k], 5 * Wn::QTILES);
+    }
+    for (int k = 0; k < kA7Groups; ++k) {
       mbar_init(&s_full[k], 1);
-      mbar_init(&p_full[k], 128);
       mbar_init(&o_full[k], 1);
     }
     mbar_init(prep_sync, kA7PrepWarps * 32);
     fence_mbar_init();
     s_abort = 0;
   }
-  if (warp == kA7MmaWarp) {
+  if (warp == 0) {
     tmem_alloc(s_tmem, kA7TmemCols);
     tmem_relinquish();
   }
@@ -1132,12 +1227,15 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     int tab_head0 = -1, tab_head1 = -1;
     float tab_max0 = 0.f, tab_max1 = 0.f;
     uint32_t ph_sync = 0;
+    int trace_n = 0;
+    (void)trace_n;
     long long j = 0;
     for (long long item = blockIdx.x; item < nitems; item += gridDim.x, ++j) {
       const int X = (int)(j & 1);
       const uint32_t use = (uint32_t)(j >> 1);
       if (j >= 2 && !mbar_wait(&buf_free[X], (use - 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
       if (s_abort) break;
+      if (pt_ == 0) VSWIN_TRACE_EVENT(0, trace_n, 1);
       const int h = (int)(item / a.nwin);
       const long long wl = item % a.nwin;
       uint8_t* sQ = smem + Wn::OFF_Q + X * Wn::QB;
@@ -1185,6 +1283,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       }
       if (!mbar_wait(&ld_full[X], use & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
       if (s_abort) break;
+      if (pt_ == 0) VSWIN_TRACE_EVENT(0, trace_n, 2);
       // key norms
       {
         float kx = 0.f;
@@ -1266,190 +1365,220 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
         }
       }
       fence_proxy_async_smem();
+      if (pt_ == 0) VSWIN_TRACE_EVENT(0, trace_n, 3);
       mbar_arrive(&prep_done[X]);
     }
-  } else if (warp == kA7MmaWarp) {
-    // ------------------------------------------------------------ MMA issue
-    // The whole warp walks the schedule (waits included); one elected lane
-    // issues. Per buffer the operand descriptors are fixed; tiles and blocks
-    // only add offsets (descriptor units of 16 bytes).
-    if (ntiles > 0) {
-      const uint32_t s_base = smem_u32(smem);
-      const uint64_t qxd0 = smem_desc(s_base + Wn::OFF_QX, 0, 128);
-      const uint64_t kxd0 = smem_desc(s_base + Wn::OFF_KX, 0, 128);
-      const uint64_t qd0 = smem_desc(s_base + Wn::OFF_Q, 128, 512);
-      const uint64_t kd0 = smem_desc(s_base + Wn::OFF_K, 128, 512);
-      const uint64_t vd0 = smem_desc(s_base + Wn::OFF_V, 512, 128);
-      // buffer X adds X * (buffer bytes) / 16
-      auto issue_s = [&](int w, long long t, int b) {
-        const long long jj = t / Wn::QTILES;
-        const int qt = (int)(t % Wn::QTILES);
-        const uint32_t X = (uint32_t)(jj & 1);
-        if (b == 0 && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) {
-          s_abort = 1;
-          return;
-        }
-        tc_fence_after();
-        const uint32_t row0 = (uint32_t)w7_tile_row0<Wn>(qt, jj);
-        const uint32_t l0 = (uint32_t)(b * Wn::BL);
-        const uint32_t dS = tmem + (uint32_t)w * kA7GroupCols;
-        // q row r: 16 B of extension (r units), 64 B of q (4 r units); key line l: 128 B / 512 B
-        const uint64_t ax = qxd0 + X * (Wn::QXB / 16) + row0;
-        const uint64_t aq = qd0 + X * (Wn::QB / 16) + 4 * row0;
-        const uint64_t bx = kxd0 + X * (Wn::KXB / 16) + 8 * l0;
-        const uint64_t bk = kd0 + X * (Wn::KB / 16) + 32 * l0;
-        if (elect_one()) {
-          if (b == Wn::NBLK - 1)
-            w7_issue_s<Wn::LAST>(dS, ax, bx, aq, bk);
-          else
-            w7_issue_s<Wn::BL>(dS, ax, bx, aq, bk);
-          umma_commit(&s_full[w]);
-        }
-        __syncwarp();
-      };
-      // returns true when the tile is complete
-      auto issue_pv = [&](int w, long long t, int b, uint32_t& ph) -> bool {
-        if (!mbar_wait(&p_full[w], ph, a.ctx.err, kErrWaitMma, lim)) {
-          s_abort = 1;
-          return false;
-        }
-        ph ^= 1;
-        tc_fence_after();
-        const uint32_t X = (uint32_t)((t / Wn::QTILES) & 1);
-        const uint32_t dS = tmem + (uint32_t)w * kA7GroupCols;
-        const uint64_t bv = vd0 + X * (Wn::KB / 16) + 32 * (uint32_t)(b * Wn::BL);
-        const bool last = b == Wn::NBLK - 1;
-        if (elect_one()) {
-          if (last)
-            w7_issue_pv<Wn::LAST>(dS + kA7OCol, dS, bv, b == 0);
-          else
-            w7_issue_pv<Wn::BL>(dS + kA7OCol, dS, bv, b == 0);
-          if (last) {
-            umma_commit(&o_full[w]);
-            umma_commit(&buf_free[X]);
-          }
-        }
-        __syncwarp();
-        return last;
-      };
-      long long t0 = 0, t1 = 1;
-      int b0 = 0, b1 = 0;
-      uint32_t ph0 = 0, ph1 = 0;
-      issue_s(0, t0, 0);
-      if (t1 < ntiles && !s_abort) issue_s(1, t1, 0);
-      while (!s_abort && (t0 < ntiles || t1 < ntiles)) {
-        if (t0 < ntiles) {
-          if (issue_pv(0, t0, b0, ph0)) {
-            t0 += 2;
-            b0 = 0;
-          } else {
-            ++b0;
-          }
-          if (!s_abort && t0 < ntiles) issue_s(0, t0, b0);
-        }
-        if (t1 < ntiles && !s_abort) {
-          if (issue_pv(1, t1, b1, ph1)) {
-            t1 += 2;
-            b1 = 0;
-          } else {
-            ++b1;
-          }
-          if (!s_abort && t1 < ntiles) issue_s(1, t1, b1);
-        }
-      }
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax groups
     const int grp = (warp - kA7Soft0) >> 2;
     const int qd = warp & 3;  // TMEM lane quarter this warp may access
-    const uint32_t tS = tmem + (uint32_t)grp * kA7GroupCols + ((uint32_t)(qd * 32) << 16);
+    const uint32_t tG = tmem + (uint32_t)grp * kA7GroupCols;  // the group's columns, lane 0
+    const uint32_t tS = tG + ((uint32_t)(qd * 32) << 16);     // ... at this warp's lanes
+    const uint32_t s_base = smem_u32(smem);
     uint32_t ph_s = 0, ph_o = 0;
-    for (long long t = grp; t < ntiles; t += 2) {
+    int turn = 0;  // block counter: the block's issuer warp is the one with qd == turn & 3
+    int trace_n = 0;
+    (void)trace_n;
+    const int trace_role = 1 + warp - kA7Soft0;
+    // Scores of block b of tile t (elected lane). Item buffer X adds
+    // X * (buffer bytes) / 16 to a descriptor; q row r is 16 B of extension
+    // (r units) and 64 B of q (4 r units); key line l is 128 B / 512 B.
+    auto issue_s = [&](long long t, int b) {
+      const uint32_t X = (uint32_t)((t / Wn::QTILES) & 1);
+      const uint32_t l0 = (uint32_t)(b * Wn::BL);
+      const uint64_t bx = smem_desc(s_base + Wn::OFF_KX + X * Wn::KXB + l0 * 128, 0, 128);
+      const uint64_t bk = smem_desc(s_base + Wn::OFF_K + X * Wn::KB + l0 * 512, 128, 512);
+      if (b == Wn::NBLK - 1)
+        w7_issue_s<Wn::LAST>(tG, tG + kA7QCol, tG + kA7QXCol, bx, bk);
+      else
+        w7_issue_s<Wn::BL>(tG, tG + kA7QCol, tG + kA7QXCol, bx, bk);
+      umma_commit(&s_full[grp]);
+    };
+    // q rows and extension rows of tile t (this thread's TMEM lane) into the
+    // group's q columns, once its item is prepared; the extension row fills
+    // both halves of its K step. Every thread of the group stages its lane.
+    auto stage_q = [&](long long t) {
+      const long long jj = t / Wn::QTILES;
+      const int X = (int)(jj & 1);
+      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      const int r = w7_tile_row0<Wn>((int)(t % Wn::QTILES), jj) + qd * 32 + lane;  // < QXROWS
+      const uint8_t* sQ = smem + Wn::OFF_Q + X * Wn::QB;  // rows past the slab read the next buffer
+      const uint8_t* sQX = smem + Wn::OFF_QX + X * Wn::QXB;
+      uint32_t qv[16], xv[8];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sQ + (r >> 3) * 512 + c * 128 + (r & 7) * 16);
+        qv[4 * c + 0] = w.x;
+        qv[4 * c + 1] = w.y;
+        qv[4 * c + 2] = w.z;
+        qv[4 * c + 3] = w.w;
+      }
+      const uint4 x = *reinterpret_cast<const uint4*>(sQX + (r >> 3) * 128 + (r & 7) * 16);
+      xv[0] = xv[4] = x.x;
+      xv[1] = xv[5] = x.y;
+      xv[2] = xv[6] = x.z;
+      xv[3] = xv[7] = x.w;
+      tmem_st16(tS + kA7QCol, qv);
+      tmem_st8(tS + kA7QXCol, xv);
+    };
+    // stage tile t's q with the whole group, then one warp issues its first scores
+    auto start_tile = [&](long long t) {
+      stage_q(t);
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(1 + grp, 128);
+      if (qd == 0) {
+        tc_fence_after();
+        if (!s_abort && elect_one()) issue_s(t, 0);
+        __syncwarp();
+      }
+    };
+    // Per-row context of tile t for this thread.
+    struct TileRow {
+      long long wl;
+      int h, X, i, pt_i, ph_i, pw_i;
+      bool active, warp_active;
+      const float* tb_row;
+    };
+    auto tile_row = [&](long long t) {
+      TileRow c;
       const long long jj = t / Wn::QTILES;
       const int qt = (int)(t % Wn::QTILES);
-      const int X = (int)(jj & 1);
+      c.X = (int)(jj & 1);
       const long long item = (long long)blockIdx.x + jj * gridDim.x;
-      const int h = (int)(item / a.nwin);
-      const long long wl = item % a.nwin;
-      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
-      const int row0 = w7_tile_row0<Wn>(qt, jj);
-      const int wrow = row0 + qd * 32;
-      const int i = wrow + lane;
-      const bool active = i >= qt * 128 && i < Wn::N;
-      const bool warp_active = wrow + 31 >= qt * 128 && wrow < Wn::N;
-      const int ie = i < qt * 128 ? qt * 128 : (i < Wn::N ? i : Wn::N - 1);
-      const int pt_i = ie / 49, ph_i = (ie / 7) % 7, pw_i = ie % 7;
-      const float* sT = reinterpret_cast<const float*>(smem + Wn::OFF_T + X * Wn::TB);
-      const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
+      c.h = (int)(item / a.nwin);
+      c.wl = item % a.nwin;
+      const int wrow = w7_tile_row0<Wn>(qt, jj) + qd * 32;
+      c.i = wrow + lane;
+      c.active = c.i >= qt * 128 && c.i < Wn::N;
+      c.warp_active = wrow + 31 >= qt * 128 && wrow < Wn::N;
+      const int ie = c.i < qt * 128 ? qt * 128 : (c.i < Wn::N ? c.i : Wn::N - 1);
+      c.pt_i = ie / 49;
+      c.ph_i = (ie / 7) % 7;
+      c.pw_i = ie % 7;
+      const float* sT = reinterpret_cast<const float*>(smem + Wn::OFF_T + c.X * Wn::TB);
+      c.tb_row = sT + (c.pt_i + Wn::P - 1) * 169 + (c.ph_i + 6) * 13 + (c.pw_i + 6);
+      return c;
+    };
+    // O / l of finished tile t (row sum L) to memory (or the exact
+    // recomputation of a row), then this warp's share of the item's release.
+    auto epilogue = [&](long long t, float L) {
+      const TileRow c = tile_row(t);
+      if (!s_abort && !mbar_wait(&o_full[grp], ph_o, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      ph_o ^= 1;
+      tc_fence_after();
+      if (c.warp_active && !s_abort) {
+        __nv_bfloat16* dst = a.o + ((size_t)c.wl * Wn::N + c.i) * g.C + c.h * kD;
+        const bool common = L >= a.exact_below && L <= 3.0e38f;
+        const float inv = 1.0f / L;
+#pragma unroll
+        for (int hv = 0; hv < 2; ++hv) {  // two halves of 16 columns
+          uint32_t o[16];
+          tmem_ld16(tS + kA7OCol + 16 * hv, o);
+          tmem_wait_ld_keep(o);
+          if (c.active && common) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+              reinterpret_cast<uint4*>(dst)[2 * hv + k] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv));
+          }
+        }
+        // the reference was too loose for this row (or overflowed): recompute it exactly
+        if (c.active && !common) w7_exact_store<Wn>(a, smem, c.X, c.wl, c.i, dst);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        VSWIN_TRACE_EVENT(trace_role, trace_n, 44);
+        mbar_arrive(&buf_free[c.X]);
+      }
+    };
+    // A group's next tile is three tiles on. With three or more tiles per item it
+    // lies at most one item ahead, whose preparation never waits for this tile:
+    // the epilogue can wait for the next tile's first block, and that tile's
+    // first scores can be issued from the last block of this one. With fewer
+    // tiles per item the next item's preparation may wait for this tile's
+    // epilogue, so the epilogue comes first and then the next tile starts.
+    constexpr bool kDefer = Wn::QTILES >= kA7Groups;  // next tile at most one item ahead
+    long long t_prev = -1;  // tile whose epilogue is pending
+    float L_prev = 0.f;
+    if (grp < ntiles) start_tile(grp);
+    for (long long t = grp; t < ntiles; t += kA7Groups) {
+      const bool next = t + kA7Groups < ntiles;
+      const long long jj = t / Wn::QTILES;
+      const int X = (int)(jj & 1);
+      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim))
+        s_abort = 1;
+      const float* tb_row;
+      bool warp_active;
+      {
+        const TileRow c = tile_row(t);
+        tb_row = c.tb_row;
+        warp_active = c.warp_active;
+      }
+      const uint32_t v_base = s_base + Wn::OFF_V + X * Wn::KB;
       float L = 0.f;
 #pragma unroll
-      for (int b = 0; b < Wn::NBLK; ++b) {
+      for (int b = 0; b < Wn::NBLK; ++b, ++turn) {
+        const bool last = b == Wn::NBLK - 1;
         if (!s_abort && !mbar_wait(&s_full[grp], ph_s, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
         ph_s ^= 1;
+        if (lane == 0) VSWIN_TRACE_EVENT(trace_role, trace_n, 40);
         tc_fence_after();
+        // this tile's last scores are in, so its q columns are free: stage the
+        // next tile's (issued below, after the block's P v)
+        if (kDefer && last && next) stage_q(t + kA7Groups);
         if (warp_active && !s_abort) {
           if (b < Wn::NBLK - 1)
             L += w7_block<Wn, Wn::BL>(tS, b * Wn::BL, tb_row);
           else
             L += w7_block<Wn, Wn::LAST>(tS, b * Wn::BL, tb_row);
         }
+        // the previous tile's O was complete long ago; it must be read before
+        // this block's P v (issued after the barrier below) starts a new O
+        if (kDefer && b == 0 && t_prev >= 0) {
+          epilogue(t_prev, L_prev);
+          t_prev = -1;
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_full[grp]);
-      }
-      if (!s_abort && !mbar_wait(&o_full[grp], ph_o, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
-      ph_o ^= 1;
-      tc_fence_after();
-      if (warp_active && !s_abort) {
-        uint32_t o[32];
-        tmem_ld32(tS + kA7OCol, o);
-        tmem_wait_ld_keep(o);
-        if (active) {
-          __nv_bfloat16* dst = a.o + ((size_t)wl * Wn::N + i) * g.C + h * kD;
-          if (L >= a.exact_below && L <= 3.0e38f) {  // the common case
-            const float inv = 1.0f / L;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              reinterpret_cast<uint4*>(dst)[c] = make_uint4(
-                  pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
-                  pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
-                  pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
-                  pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
-          } else {  // the reference was too loose for this row (or overflowed): recompute it exactly
-            const int split = window_split_bits(g, (int)((a.win0 + wl) % g.nW));
-            uint32_t okt = 0xFFFFFFFFu, okh = 0xFFFFFFFFu, okw = 0x7Fu;
-            if (split & 1) {
-              okt = 0;
-              for (int k = 0; k < Wn::P; ++k) okt |= (uint32_t)((k >= cut_t) == (pt_i >= cut_t)) << k;
+        if (lane == 0) VSWIN_TRACE_EVENT(trace_role, trace_n, 42);
+        named_bar_sync(1 + grp, 128);
+        if (qd == (turn & 3)) {  // this warp issues the block's MMAs
+          tc_fence_after();
+          if (!s_abort && elect_one()) {
+            const uint64_t bv = smem_desc(v_base + (uint32_t)(b * Wn::BL) * 512, 512, 128);
+            if (last)
+              w7_issue_pv<Wn::LAST>(tG + kA7OCol, tG, bv, b == 0);
+            else
+              w7_issue_pv<Wn::BL>(tG + kA7OCol, tG, bv, b == 0);
+            if (last) {
+              umma_commit(&o_full[grp]);
+              umma_commit(&buf_free[X]);
+              if (kDefer && next) issue_s(t + kA7Groups, 0);  // its q was staged above
+            } else {
+              issue_s(t, b + 1);  // runs after P v, which reads these columns
             }
-            if (split & 2) {
-              okh = 0;
-              for (int k = 0; k < 7; ++k) okh |= (uint32_t)((k >= cut_h) == (ph_i >= cut_h)) << k;
-            }
-            if (split & 4) {
-              okw = 0;
-              for (int k = 0; k < 7; ++k) okw |= (uint32_t)((k >= cut_w) == (pw_i >= cut_w)) << k;
-            }
-            float oe[32];
-            w7_exact_row<Wn>(smem + Wn::OFF_Q + X * Wn::QB, smem + Wn::OFF_K + X * Wn::KB,
-                             smem + Wn::OFF_V + X * Wn::KB, tb_row, i, okt, okh, okw, oe);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              reinterpret_cast<uint4*>(dst)[c] =
-                  make_uint4(pack_bf16x2(oe[8 * c + 0], oe[8 * c + 1]), pack_bf16x2(oe[8 * c + 2], oe[8 * c + 3]),
-                             pack_bf16x2(oe[8 * c + 4], oe[8 * c + 5]), pack_bf16x2(oe[8 * c + 6], oe[8 * c + 7]));
           }
+          __syncwarp();
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&buf_free[X]);
+      if (kDefer) {
+        t_prev = t;
+        L_prev = L;
+      } else {
+        epilogue(t, L);
+        if (next) start_tile(t + kA7Groups);
+      }
     }
+    if (t_prev >= 0) epilogue(t_prev, L_prev);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kA7MmaWarp) tmem_dealloc(tmem, kA7TmemCols);
+  if (warp == 0) tmem_dealloc(tmem, kA7TmemCols);
 }
 
 template <class Wn>
@@ -1597,3 +1726,13 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
 }
 
 }  // namespace vswin
+
+#ifdef VSWIN_TRACE
+// Copies the trace (roles x capacity x (tag, clock)) to `host` and clears it.
+extern "C" int vswin_trace_read(long long* host) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(host, vswin::g_trace, sizeof(vswin::g_trace)) != cudaSuccess) return -1;
+  static long long zero[vswin::kTraceRoles][vswin::kTraceCap][2];
+  return cudaMemcpyToSymbol(vswin::g_trace, zero, sizeof(zero)) == cudaSuccess ? 0 : -1;
+}
+#endif
