@@ -870,9 +870,9 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st) {
 //   warps 4-15   three softmax groups of four warps (one per TMEM lane
 //                quarter); group g owns this CTA's query tiles g, g + 3, ...
 //                (128-row tiles, items in order).
-// Keys are taken in blocks of up to 12 lines of 8 columns (the 7 keys of one
+// Keys are taken in blocks of up to 14 lines of 8 columns (the 7 keys of one
 // (pt, ph) line and a padding column). Per block: S = q k^T into the group's
-// 96 TMEM columns (q from TMEM, where the group copies its tile's q rows and
+// 112 TMEM columns (q from TMEM, where the group copies its tile's q rows and
 // their extension rows, so that only keys are read from shared memory), the
 // group turns S into bf16 P in place (4 columns per line,
 // summing p as it goes), then O += P v on the tensor core. Each group issues
@@ -910,12 +910,14 @@ constexpr int kA7Groups = 3;
 constexpr int kA7Soft0 = kA7PrepWarps;                               // first softmax warp
 constexpr int kA7Threads = (kA7PrepWarps + 4 * kA7Groups) * 32;  // 512
 constexpr uint32_t kA7TmemCols = 512;
-// per group: S / P [0, 96), O [96, 128), q of the tile [128, 144), its
-// extension row (twice) [144, 152)
-constexpr uint32_t kA7GroupCols = 160;
-constexpr uint32_t kA7OCol = 96;
-constexpr uint32_t kA7QCol = 128;
-constexpr uint32_t kA7QXCol = 144;
+// TMEM columns: group g has S / P at [144 g, 144 g + 112) and O at
+// [144 g + 112, 144 g + 144); the q rows of its tile at [432 + 16 g, + 16) and
+// their extension rows (twice) at [480 + 8 g, + 8). Column offsets stay
+// aligned to the widths that access them.
+constexpr uint32_t kA7GroupCols = 144;
+constexpr uint32_t kA7OCol = 112;
+constexpr uint32_t kA7QBase = 432;
+constexpr uint32_t kA7QXBase = 480;
 
 template <int P_>
 struct W7 {
@@ -925,8 +927,8 @@ struct W7 {
   static constexpr int KLINES = P * 7;                       // key lines of 7 real keys
   static constexpr int KCOLS = (KLINES * 8 + 31) / 32 * 32;  // k / v slab rows (padded key columns)
   static constexpr int LINES = KCOLS / 8;
-  static constexpr int NBLK = (LINES + 11) / 12;
-  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 3) / 4 * 4;  // lines per block but the last
+  static constexpr int NBLK = (LINES + 13) / 14;
+  static constexpr int BL = ((LINES + NBLK - 1) / NBLK + 1) / 2 * 2;  // lines per block but the last
   static constexpr int LAST = LINES - (NBLK - 1) * BL;
   static constexpr int TABLE = (2 * P - 1) * 169;
   static constexpr int QTILES = (N + 127) / 128;
@@ -949,7 +951,7 @@ struct W7 {
   static constexpr int OFF_T = OFF_KX + 2 * KXB;
   static constexpr int OFF_BAR = OFF_T + 2 * TB;
   static constexpr int SMEM = OFF_BAR + 256;
-  static_assert(BL <= 12 && LAST > 0 && LAST % 4 == 0, "key blocks of 4-line groups must fit 96 TMEM columns");
+  static_assert(BL <= 14 && LAST > 0 && LAST % 2 == 0, "key blocks of line pairs must fit 112 TMEM columns");
   // a tile's operand rows beyond the q slab read the following buffers (their
   // results land in TMEM lanes that are never used)
   static_assert(OFF_Q + QB + QXROWS * kSlabRowBytes <= SMEM, "tile rows must stay inside shared memory");
@@ -1373,7 +1375,10 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     const int grp = (warp - kA7Soft0) >> 2;
     const int qd = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t tG = tmem + (uint32_t)grp * kA7GroupCols;  // the group's columns, lane 0
-    const uint32_t tS = tG + ((uint32_t)(qd * 32) << 16);     // ... at this warp's lanes
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;       // this warp's TMEM lanes
+    const uint32_t tS = tG + lane_off;
+    const uint32_t tQ = tmem + kA7QBase + 16u * (uint32_t)grp;    // the group's q columns, lane 0
+    const uint32_t tQX = tmem + kA7QXBase + 8u * (uint32_t)grp;
     const uint32_t s_base = smem_u32(smem);
     uint32_t ph_s = 0, ph_o = 0;
     int turn = 0;  // block counter: the block's issuer warp is the one with qd == turn & 3
@@ -1389,9 +1394,9 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       const uint64_t bx = smem_desc(s_base + Wn::OFF_KX + X * Wn::KXB + l0 * 128, 0, 128);
       const uint64_t bk = smem_desc(s_base + Wn::OFF_K + X * Wn::KB + l0 * 512, 128, 512);
       if (b == Wn::NBLK - 1)
-        w7_issue_s<Wn::LAST>(tG, tG + kA7QCol, tG + kA7QXCol, bx, bk);
+        w7_issue_s<Wn::LAST>(tG, tQ, tQX, bx, bk);
       else
-        w7_issue_s<Wn::BL>(tG, tG + kA7QCol, tG + kA7QXCol, bx, bk);
+        w7_issue_s<Wn::BL>(tG, tQ, tQX, bx, bk);
       umma_commit(&s_full[grp]);
     };
     // q rows and extension rows of tile t (this thread's TMEM lane) into the
@@ -1418,8 +1423,8 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       xv[1] = xv[5] = x.y;
       xv[2] = xv[6] = x.z;
       xv[3] = xv[7] = x.w;
-      tmem_st16(tS + kA7QCol, qv);
-      tmem_st8(tS + kA7QXCol, xv);
+      tmem_st16(tQ + lane_off, qv);
+      tmem_st8(tQX + lane_off, xv);
     };
     // stage tile t's q with the whole group, then one warp issues its first scores
     auto start_tile = [&](long long t) {
