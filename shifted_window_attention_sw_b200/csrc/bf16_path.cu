@@ -25,10 +25,11 @@ namespace vswin {
 
 // Optional event trace of the attention kernel, compiled in only with
 // -DVSWIN_TRACE: CTA 0 records (tag, clock64) pairs per role (preparation
-// thread, lane 0 of each softmax warp), read back by
+// thread, lane 0 of each softmax warp; for the GEMMs the producer, MMA and
+// first epilogue lanes, QKV then projection), read back by
 // vswin_trace_read.
 #ifdef VSWIN_TRACE
-constexpr int kTraceRoles = 17, kTraceCap = 1024;
+constexpr int kTraceRoles = 23, kTraceCap = 1024;
 __device__ long long g_trace[kTraceRoles][kTraceCap][2];
 __device__ __forceinline__ void trace_event(int role, int& n, int tag) {
   if (blockIdx.x == 0 && n < kTraceCap) {
@@ -111,6 +112,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Named barrier over `nthreads` threads (whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -295,11 +301,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
 // ============================================================================ persistent GEMM
 //
 // Warp-specialised persistent version of the two GEMMs for layers whose
-// per-CTA weight slice (K x BN bf16) fits in shared memory: warp 0 gathers
-// 128-row A tiles with cp.async (two stages), warp 1 issues tcgen05.mma into
-// two TMEM accumulators (BN columns each), warps 2..9 drain an accumulator
-// (two warps per TMEM lane quarter, half of the columns each) while the next
-// tile is multiplied. CTA c keeps N-tile c % NT and walks the M-tiles
+// per-CTA weight slice (K x BN bf16) fits in shared memory: warps 0-3 gather
+// 128-row A tiles with cp.async into a ring of STAGES buffers (each thread's
+// copies arrive on the stage's mbarrier when they land, so the gatherers only
+// wait for a free stage), warp 4 issues tcgen05.mma into two TMEM
+// accumulators (BN columns each), warps 5..12 drain an accumulator (two warps
+// per TMEM lane quarter, half of the columns each) while the next tile is
+// multiplied. CTA c keeps N-tile c % NT and walks the M-tiles
 // c / NT, c / NT + G / NT, ... (G = grid size, a multiple of NT).
 constexpr int kWsProdWarps = 4;
 constexpr int kWsEpiWarps = 8;
@@ -309,7 +317,19 @@ constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
 constexpr int kWsMaxBBytes = 96 * 1024;
 
 __host__ __device__ inline int ws_a_bytes(int K) { return kBM * K * 2; }
-__host__ __device__ inline int ws_smem_bytes(int K, int BN) { return K * BN * 2 + 2 * ws_a_bytes(K) + BN * 4 + 256; }
+// B slice, A stages, bias (BN floats), column-group table (BN / 8 x 16 B), barriers
+__host__ __device__ inline int ws_smem_bytes(int K, int BN, int stages) {
+  return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + 256;
+}
+
+// Destination facts of one group of 8 output columns of the QKV GEMM: element
+// offset of the group inside its window's q / k / v block, whether it is a q
+// column (row layout of the q slab, scaled by log2(e)/sqrt(d)) and its scale.
+struct ColGroup {
+  int off, is_q;
+  float scale;
+  int pad;
+};
 
 // Row sources of one chunk: token index (x row) of each window slot, -1 for
 // padding. Consumed by the QKV gather and the projection scatter.
@@ -321,20 +341,21 @@ __global__ void row_source_kernel(Geom g, long long win0, long long rows, int* _
   }
 }
 
-template <int MODE>
+template <int MODE, int STAGES>
 __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int K = a.K, BN = a.BN;
   uint8_t* sB = smem;                                     // K x BN, MN-major operand layout
-  uint8_t* sA = sB + K * BN * 2;                          // 2 stages of 128 x K, K-major
-  float* sBias = reinterpret_cast<float*>(sA + 2 * ws_a_bytes(K));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBias + BN);
-  uint64_t* b_full = bars;          // B resident
-  uint64_t* a_full = bars + 1;      // [2]
-  uint64_t* a_free = bars + 3;      // [2]
-  uint64_t* acc_full = bars + 5;    // [2]
-  uint64_t* acc_free = bars + 7;    // [2]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 9);
+  uint8_t* sA = sB + K * BN * 2;                          // STAGES x (128 x K), K-major
+  float* sBias = reinterpret_cast<float*>(sA + STAGES * ws_a_bytes(K));  // bias x column scale
+  ColGroup* sGrp = reinterpret_cast<ColGroup*>(sBias + BN);                // [BN / 8]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sGrp + BN / 8);
+  uint64_t* b_full = bars;                 // B resident
+  uint64_t* a_full = bars + 1;             // [STAGES]
+  uint64_t* a_free = a_full + STAGES;      // [STAGES]
+  uint64_t* acc_full = a_free + STAGES;    // [2]
+  uint64_t* acc_free = acc_full + 2;       // [2]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(acc_free + 2);
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -349,19 +370,47 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   const uint32_t sboA = (uint32_t)(K / 8) * 128u;   // A: 8-row group stride
   const uint32_t tcols = BN <= 64 ? 128 : BN <= 128 ? 256 : 512;
   constexpr int kProdThreads = kWsProdWarps * 32;
+  constexpr int kTraceG = MODE == kQKV ? 17 : 20;  // trace roles of this GEMM
+  int trace_n = 0;
+  (void)trace_n;
+  (void)kTraceG;
 
   if (tid == 0) {
     mbar_init(b_full, kProdThreads);
-    for (int k = 0; k < 2; ++k) {
-      mbar_init(&a_full[k], kProdThreads);
+    for (int k = 0; k < STAGES; ++k) {
+      mbar_init(&a_full[k], kProdThreads);  // one asynchronous arrival per gathering thread
       mbar_init(&a_free[k], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
       mbar_init(&acc_full[k], 1);
       mbar_init(&acc_free[k], kWsEpiWarps);
     }
     fence_mbar_init();
     s_abort = 0;
   }
-  for (int c = tid; c < BN; c += kWsThreads) sBias[c] = __bfloat162float(a.bias[n0 + c]);
+  // per 8-column group: destination facts (the QKV slabs: C is a multiple of
+  // 32, so a group lies in one (which, head) slab) and the scale folded into
+  // the bias
+  for (int c8 = tid; c8 < BN / 8; c8 += kWsThreads) {
+    ColGroup cg{0, 0, 1.0f, 0};
+    if (MODE == kQKV) {
+      const int col = n0 + 8 * c8;
+      const int sidx = col >> 5;
+      const int which = sidx / g.heads;
+      const int hh = sidx - which * g.heads;
+      const SlabLayout& L = a.slab;
+      cg.off = (int)((size_t)hh * L.head_elems() +
+                     (which == 0 ? 0 : ((size_t)L.qrows + (size_t)(which - 1) * L.kvrows) * 32)) +
+               ((col & 31) >> 3) * 64;
+      cg.is_q = which == 0;
+      cg.scale = which == 0 ? a.qscale : 1.0f;
+    }
+    sGrp[c8] = cg;
+  }
+  for (int c = tid; c < BN; c += kWsThreads) {
+    const float sc = (MODE == kQKV && (((n0 + c) >> 5) / g.heads) == 0) ? a.qscale : 1.0f;
+    sBias[c] = __bfloat162float(a.bias[n0 + c]) * sc;
+  }
   if (warp == kWsMmaWarp) {
     tmem_alloc(s_tmem, tcols);
     tmem_relinquish();
@@ -378,62 +427,69 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       const int kk = c / (BN / 8), nc = c % (BN / 8);
       cp_async_16(sB + (kk >> 3) * lboB + nc * 128 + (kk & 7) * 16, a.Wt + (size_t)kk * a.Ntot + n0 + nc * 8, 16u);
     }
-    cp_async_commit();
+    cp_async_mbar_arrive_noinc(b_full);
     // A gather: warp w fills rows [32w, 32w + 32) in groups of 8 rows; 4 lanes per
     // row, lane l moving chunks l%4, l%4 + 4, ... (64 contiguous bytes per row and
     // instruction).
     const int sub = lane >> 2, cq = lane & 3;
-    // Source offsets of this lane's 4 rows, fetched one tile ahead so that the
-    // table reads overlap the previous tile's copies.
-    auto row_src = [&](long long m, int grp) -> long long {
+    // Source offsets of this lane's 4 rows, fetched two tiles ahead so that the
+    // table reads (global loads) have landed by the time the copies need them.
+    // Row index of each of this lane's 4 rows in the source matrix (-1:
+    // padding): QKV looks it up in the row table, two tiles ahead, and keeps the
+    // raw value so that nothing waits for the load before it is needed.
+    auto row_tok = [&](long long m, int grp) -> int {
       const long long r = m * kBM + warp * 32 + grp * 8 + sub;
-      if (r >= a.rows) return -1;
-      if (MODE == kQKV) {
-        const int tok = a.rowsrc[r];
-        return tok < 0 ? -1 : (long long)tok * g.C;
-      }
-      return r * (long long)g.C;
+      if (m >= mtiles || r >= a.rows) return -1;
+      return MODE == kQKV ? a.rowsrc[r] : (int)r;
     };
-    long long src[4];
+    int tok0[4], tok1[4], tok2[4];
 #pragma unroll
-    for (int grp = 0; grp < 4; ++grp) src[grp] = m_first < mtiles ? row_src(m_first, grp) : -1;
+    for (int grp = 0; grp < 4; ++grp) {
+      tok0[grp] = row_tok(m_first, grp);
+      tok1[grp] = row_tok(m_first + m_step, grp);
+    }
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += m_step, ++t) {
-      const int s = (int)(t & 1);
-      if (t >= 2 && !s_abort && !mbar_wait(&a_free[s], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+      const int s = (int)(t % STAGES);
+      if (tid == 0) VSWIN_TRACE_EVENT(kTraceG + 0, trace_n, 50);
+      if (t >= STAGES && !s_abort &&
+          !mbar_wait(&a_free[s], (uint32_t)((t / STAGES) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
         s_abort = 1;
       uint8_t* dA = sA + s * ws_a_bytes(K);
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
         const int row = warp * 32 + grp * 8 + sub;
         uint8_t* drow = dA + (row >> 3) * sboA + (row & 7) * 16;
-        const long long sg = src[grp];
+        const int tk = tok0[grp];
+        const long long sg = tk < 0 ? 0 : (long long)tk * g.C;
         for (int kc = cq; kc < K / 8; kc += 4)
-          cp_async_16(drow + kc * 128, a.A + (sg < 0 ? 0 : sg + kc * 8), sg < 0 ? 0u : 16u);
+          cp_async_16(drow + kc * 128, a.A + sg + kc * 8, tk < 0 ? 0u : 16u);
       }
-      cp_async_commit();
-      const long long mn = m + m_step;
+      cp_async_mbar_arrive_noinc(&a_full[s]);  // arrives once this thread's copies have landed
+      if (tid == 0) VSWIN_TRACE_EVENT(kTraceG + 0, trace_n, 51);
 #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) src[grp] = mn < mtiles ? row_src(mn, grp) : -1;
-      cp_async_wait<1>();  // the previous group (B, or the previous tile) has landed
-      fence_proxy_async_smem();
-      if (t == 0) mbar_arrive(b_full);
-      else mbar_arrive(&a_full[(t - 1) & 1]);
+      for (int grp = 0; grp < 4; ++grp) tok2[grp] = row_tok(m + 2 * m_step, grp);
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        tok0[grp] = tok1[grp];
+        tok1[grp] = tok2[grp];
+      }
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (t == 0) mbar_arrive(b_full);
-    else mbar_arrive(&a_full[(t - 1) & 1]);
+    cp_async_wait_all();  // nothing in flight when the CTA ends
   } else if (warp == kWsMmaWarp) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
       if (!mbar_wait(b_full, 0, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      fence_proxy_async_smem();  // the gathered bytes, written by cp.async, are read by the tensor core
       const uint32_t idesc = idesc_bf16(kBM, BN, 0, 1);
       const uint32_t baddr = smem_u32(sB);
       long long t = 0;
       for (long long m = m_first; m < mtiles; m += m_step, ++t) {
-        const int s = (int)(t & 1), buf = (int)(t & 1);
-        if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        const int s = (int)(t % STAGES), buf = (int)(t & 1);
+        VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 60);
+        if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        fence_proxy_async_smem();
+        VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 61);
         if (t >= 2 && !s_abort &&
             !mbar_wait(&acc_free[buf], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
           s_abort = 1;
@@ -445,6 +501,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
                     smem_desc(baddr + ks * 2 * lboB, lboB, 128), idesc, ks > 0);
           umma_commit(&a_free[s]);
           umma_commit(&acc_full[buf]);
+          VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 62);
         }
       }
     }
@@ -456,75 +513,87 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     const int q = warp & 3, hf = (warp - kWsEpi0) >> 2;
     const int cw = BN / 2;  // columns of this warp (multiple of 8)
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const size_t win_elems = (size_t)g.heads * a.slab.head_elems();  // one window's q / k / v block
+    // projection: this row's output row, loaded one tile ahead (the loaded
+    // value is first used a tile later)
+    auto out_row = [&](long long m) -> int {
+      const long long r = m * kBM + q * 32 + lane;
+      return (MODE == kPROJ && m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
+    };
+    int dr_next = out_row(m_first);
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += m_step, ++t) {
       const int buf = (int)(t & 1);
       const long long r = m * kBM + q * 32 + lane;
       const bool row_ok = r < a.rows;
-      long long dst_row = -1;
-      int slot = 0;
-      long long slab_win = 0;
+      const int dr_cur = dr_next;
+      dr_next = out_row(m + m_step);
+      // this row's destination: QKV, the window's block and the row term of the
+      // q slab and of the k / v slabs; projection, the output row
+      __nv_bfloat16* rbase = nullptr;
+      int q_term = 0, kv_term = 0;
       if (row_ok) {
         if (MODE == kQKV) {
           const int ri = (int)r;  // rows < 2^31 (checked by the caller)
-          slab_win = ri / g.N;
-          slot = ri - (int)slab_win * g.N;
+          const int slab_win = ri / g.N;
+          const int slot = ri - slab_win * g.N;
+          const int kvr = a.slab.kv_row(slot);
+          q_term = (slot >> 3) * 256 + (slot & 7) * 8;
+          kv_term = (kvr >> 3) * 256 + (kvr & 7) * 8;
+          rbase = a.dst + (size_t)slab_win * win_elems;
         } else {
-          dst_row = a.rowsrc[r];
+          const long long dr = dr_cur;
+          if (dr >= 0) rbase = a.dst + dr * g.C + n0;
         }
       }
+      if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 70);
       if (!s_abort && !mbar_wait(&acc_full[buf], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 71);
       tc_fence_after();
       if (!s_abort && m * kBM + q * 32 < a.rows) {
-        for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += 32) {
-          const int n = (hf + 1) * cw - c0 < 32 ? (hf + 1) * cw - c0 : 32;  // 8, 16, 24 or 32
-          uint32_t u[32];
+        // all of this warp's columns (up to 96 at a time) loaded before one wait
+        for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += 96) {
+          const int n = (hf + 1) * cw - c0 < 96 ? (hf + 1) * cw - c0 : 96;  // a multiple of 8
+          uint32_t u[96];
           const uint32_t ta = tmem + lane_base + buf * BN + c0;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 12; ++j)
             if (j * 8 < n)
               asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                            : "=r"(u[8 * j + 0]), "=r"(u[8 * j + 1]), "=r"(u[8 * j + 2]), "=r"(u[8 * j + 3]),
                              "=r"(u[8 * j + 4]), "=r"(u[8 * j + 5]), "=r"(u[8 * j + 6]), "=r"(u[8 * j + 7])
                            : "r"(ta + 8 * j));
-          tmem_wait_ld();
+          tmem_wait_ld_keep(u);
 #pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) {
+          for (int g8 = 0; g8 < 12; ++g8) {
             if (g8 * 8 >= n) break;
             const int cc = c0 + g8 * 8;
-            const int col = n0 + cc;
             const float4 b0 = *reinterpret_cast<const float4*>(sBias + cc);
             const float4 b1 = *reinterpret_cast<const float4*>(sBias + cc + 4);
-            float v[8] = {__uint_as_float(u[g8 * 8 + 0]) + b0.x, __uint_as_float(u[g8 * 8 + 1]) + b0.y,
-                          __uint_as_float(u[g8 * 8 + 2]) + b0.z, __uint_as_float(u[g8 * 8 + 3]) + b0.w,
-                          __uint_as_float(u[g8 * 8 + 4]) + b1.x, __uint_as_float(u[g8 * 8 + 5]) + b1.y,
-                          __uint_as_float(u[g8 * 8 + 6]) + b1.z, __uint_as_float(u[g8 * 8 + 7]) + b1.w};
-            if (MODE == kQKV) {
-              if (row_ok) {
-                const int sidx = col >> 5;  // (which, head) slab: C is a multiple of 32
-                const int which = sidx / g.heads;
-                const int hh = sidx - which * g.heads;
-                const int jj = col & 31;
-                const float sc = which == 0 ? a.qscale : 1.0f;
-                const SlabLayout& L = a.slab;
-                __nv_bfloat16* slab = a.dst + ((size_t)slab_win * g.heads + hh) * L.head_elems() +
-                                      (which == 0 ? 0 : ((size_t)L.qrows + (size_t)(which - 1) * L.kvrows) * 32);
-                const int row = which == 0 ? slot : L.kv_row(slot);
-                __nv_bfloat16* dst = slab + (row >> 3) * 256 + (jj >> 3) * 64 + (row & 7) * 8;
-                *reinterpret_cast<uint4*>(dst) =
-                    make_uint4(pack_bf16x2(v[0] * sc, v[1] * sc), pack_bf16x2(v[2] * sc, v[3] * sc),
-                               pack_bf16x2(v[4] * sc, v[5] * sc), pack_bf16x2(v[6] * sc, v[7] * sc));
-              }
-            } else if (dst_row >= 0) {
-              *reinterpret_cast<uint4*>(a.dst + dst_row * g.C + col) =
-                  make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                             pack_bf16x2(v[6], v[7]));
+            const ColGroup cg = sGrp[cc >> 3];
+            const float2 sc = make_float2(cg.scale, cg.scale);
+            // v = acc * scale + bias * scale, two columns per instruction
+            const float2 v01 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 0]), __uint_as_float(u[g8 * 8 + 1])),
+                                          sc, make_float2(b0.x, b0.y));
+            const float2 v23 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 2]), __uint_as_float(u[g8 * 8 + 3])),
+                                          sc, make_float2(b0.z, b0.w));
+            const float2 v45 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 4]), __uint_as_float(u[g8 * 8 + 5])),
+                                          sc, make_float2(b1.x, b1.y));
+            const float2 v67 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 6]), __uint_as_float(u[g8 * 8 + 7])),
+                                          sc, make_float2(b1.z, b1.w));
+            const uint4 w = make_uint4(pack_bf16x2(v01.x, v01.y), pack_bf16x2(v23.x, v23.y),
+                                       pack_bf16x2(v45.x, v45.y), pack_bf16x2(v67.x, v67.y));
+            if (rbase) {
+              __nv_bfloat16* dst =
+                  MODE == kQKV ? rbase + cg.off + (cg.is_q ? q_term : kv_term) : rbase + cc;
+              *reinterpret_cast<uint4*>(dst) = w;
             }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
+      if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 72);
       if (lane == 0) mbar_arrive(&acc_free[buf]);
     }
   }
@@ -1105,11 +1174,6 @@ __device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, 
   for (int d = 0; d < 32; ++d) o[d] *= inv;
 }
 
-// Named barrier over `nthreads` threads (whole warps).
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // One elected lane of a converged warp.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
@@ -1623,12 +1687,16 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
     long long per_nt = sms / NT;
     if (per_nt < 1) per_nt = 1;
     if (per_nt > mtiles) per_nt = mtiles;
-    // at least 116 KB so that one CTA (up to 512 TMEM columns) owns each SM
-    const int smem_ws = ws_smem_bytes(a.K, a.BN) > 116 * 1024 ? ws_smem_bytes(a.K, a.BN) : 116 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(gemm_ws_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_ws);
+    // four A stages when they fit, else two; at least 116 KB so that one CTA
+    // (up to 512 TMEM columns) owns each SM
+    const bool four = ws_smem_bytes(a.K, a.BN, 4) <= 220 * 1024;
+    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2);
+    if (smem_ws < 116 * 1024) smem_ws = 116 * 1024;
+    auto kern = four ? gemm_ws_kernel<MODE, 4> : gemm_ws_kernel<MODE, 2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_ws);
     if (e != cudaSuccess) return e;
     prof_begin(MODE == kQKV ? kKindQkv : kKindProj, st);
-    gemm_ws_kernel<MODE><<<(unsigned)(per_nt * NT), kWsThreads, smem_ws, st>>>(a);
+    kern<<<(unsigned)(per_nt * NT), kWsThreads, smem_ws, st>>>(a);
     prof_end(MODE == kQKV ? kKindQkv : kKindProj, st);
     count_launch();
     return cudaGetLastError();
