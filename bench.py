@@ -133,20 +133,22 @@ def oracle_sample(wl, target_s, nthreads=0, layers=None):
     cores = oracle.max_threads(nthreads)
     layers = layers if layers is not None else wl.layers
     inputs = [workload_layer_inputs(wl, ly, scale="baseline").as_f64() for ly in layers]
+    # window maps (to count real tokens) are computed once, outside the timed region
+    geoms = [oracle.geometry(ly.T, ly.H, ly.W, ly.window, ly.shift) for ly in layers]
+    srcs = [oracle.index_maps(ly.B, ly.T, ly.H, ly.W, ly.window, ly.shift)[0] for ly in layers]
 
     def run(nwin_per_layer):
-        tokens = 0
-        t0 = time.perf_counter()
-        for ly, a in zip(layers, inputs):
-            g = oracle.geometry(ly.T, ly.H, ly.W, ly.window, ly.shift)
+        tokens, dt = 0, 0.0
+        for ly, a, g, src in zip(layers, inputs, geoms, srcs):
             total = ly.B * g["nW"]
             wins = np.linspace(0, total - 1, num=min(nwin_per_layer, total)).astype(np.int64)
+            t0 = time.perf_counter()
             oracle.forward_windows(a["x"], ly.window, ly.shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"],
                                    a["table"], ly.heads, wins, nthreads=nthreads)
-            src, _, _ = oracle.index_maps(ly.B, ly.T, ly.H, ly.W, ly.window, ly.shift)
+            dt += time.perf_counter() - t0
             N = g["N"]
             tokens += int(sum((src[w * N:(w + 1) * N] >= 0).sum() for w in wins))
-        return tokens, time.perf_counter() - t0
+        return tokens, dt
 
     tok, dt = run(cores)  # calibration: one window per thread and layer
     n = max(1, int(cores * target_s / max(dt, 1e-6)))
@@ -170,6 +172,7 @@ def run_reference(args):
     # calibrate the per-step sample so the whole run stays within a few minutes
     cal = oracle_sample(wl, budget)
     nwin = cal["windows_per_layer"]
+    _oracle_prep(wl, nwin)  # inputs and window maps, outside the timed steps
     times, toks = [], 0
     for k in range(args.warmup + args.steps):
         t0 = time.perf_counter()
@@ -200,22 +203,37 @@ _ORACLE_CACHE = {}
 
 
 def _oracle_fixed(wl, nwin):
+    """One reference-arm step: the oracle on `nwin` evenly spaced whole windows of each
+    layer; returns the real (non-padding) tokens of those windows. Inputs, window maps
+    and token counts are prepared once per workload and sample size, outside the
+    timed call."""
     import oracle
 
-    key = wl.name
-    if key not in _ORACLE_CACHE:
-        _ORACLE_CACHE[key] = [workload_layer_inputs(wl, ly, scale="baseline").as_f64() for ly in wl.layers]
     tokens = 0
-    for ly, a in zip(wl.layers, _ORACLE_CACHE[key]):
-        g = oracle.geometry(ly.T, ly.H, ly.W, ly.window, ly.shift)
-        total = ly.B * g["nW"]
-        wins = np.linspace(0, total - 1, num=min(nwin, total)).astype(np.int64)
+    for ly, a, wins, tok in _oracle_prep(wl, nwin):
         oracle.forward_windows(a["x"], ly.window, ly.shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"],
                                a["table"], ly.heads, wins)
-        src, _, _ = oracle.index_maps(ly.B, ly.T, ly.H, ly.W, ly.window, ly.shift)
-        N = g["N"]
-        tokens += int(sum((src[w * N:(w + 1) * N] >= 0).sum() for w in wins))
+        tokens += tok
     return tokens
+
+
+def _oracle_prep(wl, nwin):
+    import oracle
+
+    key = (wl.name, nwin)
+    if key not in _ORACLE_CACHE:
+        prep = []
+        for ly in wl.layers:
+            a = workload_layer_inputs(wl, ly, scale="baseline").as_f64()
+            g = oracle.geometry(ly.T, ly.H, ly.W, ly.window, ly.shift)
+            total = ly.B * g["nW"]
+            wins = np.linspace(0, total - 1, num=min(nwin, total)).astype(np.int64)
+            src, _, _ = oracle.index_maps(ly.B, ly.T, ly.H, ly.W, ly.window, ly.shift)
+            N = g["N"]
+            tok = int(sum((src[w * N:(w + 1) * N] >= 0).sum() for w in wins))
+            prep.append((ly, a, wins, tok))
+        _ORACLE_CACHE[key] = prep
+    return _ORACLE_CACHE[key]
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -394,7 +412,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--cpu-sample-s", type=float, default=20.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
