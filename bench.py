@@ -150,12 +150,16 @@ def oracle_sample(wl, target_s, nthreads=0, layers=None):
             tokens += int(sum((src[w * N:(w + 1) * N] >= 0).sum() for w in wins))
         return tokens, dt
 
-    tok, dt = run(cores)  # calibration: one window per thread and layer
-    n = max(1, int(cores * target_s / max(dt, 1e-6)))
-    if n > cores:
+    # calibration: start with one window per thread and layer, then scale the
+    # sample until the timed oracle work is at least half the target
+    n = cores
+    tok, dt = run(n)
+    total = max(ly.B * g["nW"] for ly, g in zip(layers, geoms))
+    for _ in range(4):
+        if dt >= 0.5 * target_s or n >= total:
+            break
+        n = min(total, max(n + 1, int(n * min(8.0, target_s / max(dt, 1e-6)))))
         tok, dt = run(n)
-    else:
-        n = cores
     return {"tokens": tok, "seconds": dt, "cores": cores, "windows_per_layer": n}
 
 

@@ -68,9 +68,9 @@ typedef enum {
 /*
  * bf16 layer forward: x, weights, biases, table and out are bf16; products
  * accumulate in fp32 on the tensor cores (tcgen05). Requires d = C/heads = 32,
- * C a multiple of 32, N = P*Mh*Mw <= 400, window (P, Mh, Mw) one of the
- * compiled shapes (8,7,7), (4,7,7), (2,7,7), (1,7,7), (4,4,4), (2,2,2),
- * (1,1,1); otherwise VSWIN_ERR_UNSUPPORTED. Pointers must be 16-byte aligned
+ * C a multiple of 32, window (P, Mh, Mw) one of the compiled shapes
+ * (16,7,7), (8,7,7), (4,7,7), (2,7,7), (1,7,7), (4,4,4), (2,2,2), (1,1,1)
+ * (N = P*Mh*Mw up to 784); otherwise VSWIN_ERR_UNSUPPORTED. Pointers must be 16-byte aligned
  * and x must not overlap out.
  * Scratch: stream-ordered allocation on `stream` from a memory pool the
  * library creates per device and keeps (freed scratch is reused by the next

@@ -72,7 +72,7 @@ struct SlabLayout {
 
 __host__ __device__ inline bool window_is_p77(const Geom& g) {
   const int P = g.win[0];
-  return g.win[1] == 7 && g.win[2] == 7 && (P == 1 || P == 2 || P == 4 || P == 8);
+  return g.win[1] == 7 && g.win[2] == 7 && (P == 1 || P == 2 || P == 4 || P == 8 || P == 16);
 }
 
 __host__ __device__ inline SlabLayout slab_layout(const Geom& g) {
@@ -1006,26 +1006,40 @@ struct W7 {
   // its work rotates over the four SM sub-partitions.
   static constexpr bool ROTATE = QTILES > 1 && TAIL <= 32;
   static constexpr int QXROWS = QTILES * 128;
-  // shared memory, two item buffers of each
+  // shared memory per item buffer
   static constexpr int QB = QSLAB * kSlabRowBytes;
   static constexpr int KB = KCOLS * kSlabRowBytes;
   static constexpr int QXB = QXROWS * 16;
   static constexpr int KXB = KCOLS * 16;
   static constexpr int TB = (TABLE * 4 + 127) / 128 * 128;
+  static constexpr int ITEM_BYTES = QB + 2 * KB + QXB + KXB + TB;
+  // two item buffers (the next item is prepared while this one is computed)
+  // when they fit, else one (temporal windows of 16: 210 KB per item)
+  static constexpr int NBUF = 2 * ITEM_BYTES + 256 <= 227 * 1024 ? 2 : 1;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * QB;
-  static constexpr int OFF_V = OFF_K + 2 * KB;
-  static constexpr int OFF_QX = OFF_V + 2 * KB;
-  static constexpr int OFF_KX = OFF_QX + 2 * QXB;
-  static constexpr int OFF_T = OFF_KX + 2 * KXB;
-  static constexpr int OFF_BAR = OFF_T + 2 * TB;
+  static constexpr int OFF_K = OFF_Q + NBUF * QB;
+  static constexpr int OFF_V = OFF_K + NBUF * KB;
+  static constexpr int OFF_QX = OFF_V + NBUF * KB;
+  static constexpr int OFF_KX = OFF_QX + NBUF * QXB;
+  static constexpr int OFF_T = OFF_KX + NBUF * KXB;
+  static constexpr int OFF_BAR = OFF_T + NBUF * TB;
   static constexpr int SMEM = OFF_BAR + 256;
   static_assert(BL <= 14 && LAST > 0 && LAST % 2 == 0, "key blocks of line pairs must fit 112 TMEM columns");
   // a tile's operand rows beyond the q slab read the following buffers (their
   // results land in TMEM lanes that are never used)
-  static_assert(OFF_Q + QB + QXROWS * kSlabRowBytes <= SMEM, "tile rows must stay inside shared memory");
+  static_assert(OFF_Q + (NBUF - 1) * QB + QXROWS * kSlabRowBytes <= SMEM, "tile rows must stay inside shared memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
+
+// Item buffer of this CTA's j-th item, and how many earlier items used it.
+template <class Wn>
+__device__ __forceinline__ int w7_buf(long long j) {
+  return Wn::NBUF == 2 ? (int)(j & 1) : 0;
+}
+template <class Wn>
+__device__ __forceinline__ long long w7_use(long long j) {
+  return Wn::NBUF == 2 ? (j >> 1) : j;
+}
 
 template <class Wn>
 __device__ __forceinline__ int w7_tile_row0(int qt, long long jj) {
@@ -1040,13 +1054,6 @@ __device__ __forceinline__ int w7_region(int split_bit, int c, int cut) { return
 // generic memory; their order relative to each other and to the fences is
 // kept because all of them are volatile), so that shared-memory loads of the
 // bias may be scheduled across them.
-__device__ __forceinline__ void tmem_st16_reg(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
-}
 template <int N>
 __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[N]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;");
@@ -1297,9 +1304,9 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     (void)trace_n;
     long long j = 0;
     for (long long item = blockIdx.x; item < nitems; item += gridDim.x, ++j) {
-      const int X = (int)(j & 1);
-      const uint32_t use = (uint32_t)(j >> 1);
-      if (j >= 2 && !mbar_wait(&buf_free[X], (use - 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      const int X = w7_buf<Wn>(j);
+      const uint32_t use = (uint32_t)w7_use<Wn>(j);  // earlier items in buffer X
+      if (j >= Wn::NBUF && !mbar_wait(&buf_free[X], (use - 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
       if (s_abort) break;
       if (pt_ == 0) VSWIN_TRACE_EVENT(0, trace_n, 1);
       const int h = (int)(item / a.nwin);
@@ -1449,11 +1456,12 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     int trace_n = 0;
     (void)trace_n;
     const int trace_role = 1 + warp - kA7Soft0;
+    (void)trace_role;
     // Scores of block b of tile t (elected lane). Item buffer X adds
     // X * (buffer bytes) / 16 to a descriptor; q row r is 16 B of extension
     // (r units) and 64 B of q (4 r units); key line l is 128 B / 512 B.
     auto issue_s = [&](long long t, int b) {
-      const uint32_t X = (uint32_t)((t / Wn::QTILES) & 1);
+      const uint32_t X = (uint32_t)w7_buf<Wn>(t / Wn::QTILES);
       const uint32_t l0 = (uint32_t)(b * Wn::BL);
       const uint64_t bx = smem_desc(s_base + Wn::OFF_KX + X * Wn::KXB + l0 * 128, 0, 128);
       const uint64_t bk = smem_desc(s_base + Wn::OFF_K + X * Wn::KB + l0 * 512, 128, 512);
@@ -1468,8 +1476,9 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     // both halves of its K step. Every thread of the group stages its lane.
     auto stage_q = [&](long long t) {
       const long long jj = t / Wn::QTILES;
-      const int X = (int)(jj & 1);
-      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      const int X = w7_buf<Wn>(jj);
+      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)w7_use<Wn>(jj) & 1, a.ctx.err, kErrWaitLoad, lim))
+        s_abort = 1;
       const int r = w7_tile_row0<Wn>((int)(t % Wn::QTILES), jj) + qd * 32 + lane;  // < QXROWS
       const uint8_t* sQ = smem + Wn::OFF_Q + X * Wn::QB;  // rows past the slab read the next buffer
       const uint8_t* sQX = smem + Wn::OFF_QX + X * Wn::QXB;
@@ -1513,7 +1522,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       TileRow c;
       const long long jj = t / Wn::QTILES;
       const int qt = (int)(t % Wn::QTILES);
-      c.X = (int)(jj & 1);
+      c.X = w7_buf<Wn>(jj);
       const long long item = (long long)blockIdx.x + jj * gridDim.x;
       c.h = (int)(item / a.nwin);
       c.wl = item % a.nwin;
@@ -1566,20 +1575,21 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
       }
     };
     // A group's next tile is three tiles on. With three or more tiles per item it
-    // lies at most one item ahead, whose preparation never waits for this tile:
-    // the epilogue can wait for the next tile's first block, and that tile's
-    // first scores can be issued from the last block of this one. With fewer
-    // tiles per item the next item's preparation may wait for this tile's
-    // epilogue, so the epilogue comes first and then the next tile starts.
-    constexpr bool kDefer = Wn::QTILES >= kA7Groups;  // next tile at most one item ahead
+    // lies at most one item ahead; with two item buffers that item's
+    // preparation never waits for this tile, so the epilogue can wait for the
+    // next tile's first block and that tile's first scores can be issued from
+    // the last block of this one. Otherwise the next item's preparation may
+    // wait for this tile's epilogue, so the epilogue comes first and then the
+    // next tile starts.
+    constexpr bool kDefer = Wn::NBUF == 2 && Wn::QTILES >= kA7Groups;
     long long t_prev = -1;  // tile whose epilogue is pending
     float L_prev = 0.f;
     if (grp < ntiles) start_tile(grp);
     for (long long t = grp; t < ntiles; t += kA7Groups) {
       const bool next = t + kA7Groups < ntiles;
       const long long jj = t / Wn::QTILES;
-      const int X = (int)(jj & 1);
-      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)(jj >> 1) & 1, a.ctx.err, kErrWaitLoad, lim))
+      const int X = w7_buf<Wn>(jj);
+      if (!s_abort && !mbar_wait(&prep_done[X], (uint32_t)w7_use<Wn>(jj) & 1, a.ctx.err, kErrWaitLoad, lim))
         s_abort = 1;
       const float* tb_row;
       bool warp_active;
@@ -1716,7 +1726,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
 
 bool bf16_window_supported(const Geom& g) {
   const int P = g.win[0], MH = g.win[1], MW = g.win[2];
-  return (P == 8 && MH == 7 && MW == 7) || (P == 4 && MH == 7 && MW == 7) || (P == 2 && MH == 7 && MW == 7) ||
+  return (P == 16 && MH == 7 && MW == 7) || (P == 8 && MH == 7 && MW == 7) || (P == 4 && MH == 7 && MW == 7) ||
+         (P == 2 && MH == 7 && MW == 7) ||
          (P == 1 && MH == 7 && MW == 7) || (P == 4 && MH == 4 && MW == 4) || (P == 2 && MH == 2 && MW == 2) ||
          (P == 1 && MH == 1 && MW == 1);
 }
@@ -1777,7 +1788,8 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   aa.slab = L;
   aa.exact_below = ctx.force_exact ? INFINITY : 7.8886e-31f;  // 2^-100
   const int P = g.win[0], MH = g.win[1], MW = g.win[2];
-  if (P == 8 && MH == 7 && MW == 7) e = launch_attention7<W7<8>>(aa, st);
+  if (P == 16 && MH == 7 && MW == 7) e = launch_attention7<W7<16>>(aa, st);
+  else if (P == 8 && MH == 7 && MW == 7) e = launch_attention7<W7<8>>(aa, st);
   else if (P == 4 && MH == 7 && MW == 7) e = launch_attention7<W7<4>>(aa, st);
   else if (P == 2 && MH == 7 && MW == 7) e = launch_attention7<W7<2>>(aa, st);
   else if (P == 1 && MH == 7 && MW == 7) e = launch_attention7<W7<1>>(aa, st);

@@ -75,7 +75,7 @@ def test_invalid_arguments_launch_nothing(L, name, kw):
     "kw",
     [dict(C=128, heads=2),                          # head width 64
      dict(window=(3, 7, 7), shift=(1, 3, 3)),      # no kernel compiled for this window
-     dict(window=(16, 7, 7), shift=(8, 3, 3))],    # N = 784 > 400
+     dict(window=(8, 8, 8), shift=(4, 4, 4))],     # N = 512, no kernel compiled for this window
 )
 def test_bf16_unsupported_shapes(L, kw):
     before = vswin.launch_count()

@@ -139,6 +139,7 @@ BF16_CASES = [
     ((2, 1, 14, 21, 64), 2, (1, 7, 7), (0, 3, 3)),      # 2D Swin special case
     ((1, 8, 14, 14, 64), 2, (4, 7, 7), (2, 3, 3)),      # temporal window 4
     ((2, 6, 14, 21, 64), 2, (2, 7, 7), (1, 3, 3)),      # temporal window 2 (one query tile per window)
+    ((1, 20, 14, 14, 64), 2, (16, 7, 7), (8, 3, 3)),    # temporal window 16 (N = 784, one item buffer)
     ((1, 8, 8, 12, 64), 2, (4, 4, 4), (2, 2, 2)),
     ((2, 3, 4, 5, 32), 1, (1, 1, 1), (0, 0, 0)),        # one-token windows
     ((1, 4, 6, 6, 32), 1, (2, 2, 2), (1, 1, 1)),
