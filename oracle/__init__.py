@@ -13,6 +13,12 @@ Two independent formulations live here:
   window_msa pseudocode; eq. 2.
 * ``group_rule.forward`` -- a NumPy float64 brute force over all token pairs of
   the padded grid with no roll and no partition (see that module).
+
+The attention half of a block (``block_forward``) is written on top of
+``forward`` in NumPy float64: layer norm of each token over its C channels,
+the layer, and the residual add ("Video Swin Transformer" summary page, Method
+step 3 and eq. 1; Video Swin code walk-through page, section 1.2: LayerNorm
+comes before F.pad, so padded tokens are zeros after the norm).
 """
 
 from __future__ import annotations
@@ -181,3 +187,57 @@ def index_maps(B, T, H, W, window, shift):
     if rc != 0:
         raise ValueError(f"oracle rejected the arguments (status {rc})")
     return win_src, region, bias_idx
+
+
+LN_EPS = 1e-5  # torch.nn.LayerNorm's default; the code walk-through page names nn.LayerNorm
+
+
+def layer_norm(x, gamma, beta, eps=LN_EPS):
+    """Layer norm of each token over its last axis, in float64.
+
+    (x - mean) / sqrt(var + eps) * gamma + beta with the biased variance
+    (mean of squared deviations), as torch.nn.LayerNorm computes it. "Video
+    Swin Transformer" summary page, Method step 3 and eq. 1 (LN).
+    """
+    x = _f64(x)
+    gamma, beta = _f64(gamma), _f64(beta)
+    mean = x.mean(axis=-1, keepdims=True)
+    dev = x - mean
+    var = (dev * dev).mean(axis=-1, keepdims=True)
+    return dev / np.sqrt(var + float(eps)) * gamma + beta
+
+
+def block_forward(x, gamma, beta, eps, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, flags=0,
+                  nthreads=0):
+    """Attention half of a Video Swin block in float64: x + layer(LN(x)).
+
+    "Video Swin Transformer" summary page, eq. 1 (z_hat = 3D(S)W-MSA(LN(z)) + z)
+    and the block pseudocode; the layer is ``forward`` with the same arguments.
+    """
+    x = _f64(x)
+    y = layer_norm(x, gamma, beta, eps)
+    return x + forward(y, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, flags=flags,
+                       nthreads=nthreads)
+
+
+def block_forward_windows(x, gamma, beta, eps, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads,
+                          windows, nthreads=0):
+    """``block_forward`` restricted to the listed windows (flat b * nW + w).
+
+    Returns (len(windows), N, C): for each window slot that holds a real
+    token, that token's block output; padding slots hold the layer's value
+    there without a residual (they are not outputs of the block). The norm
+    is per token, so normalising the whole tensor first is exact.
+    """
+    x = _f64(x)
+    y = layer_norm(x, gamma, beta, eps)
+    o = forward_windows(y, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, windows, nthreads=nthreads)
+    B, T, H, W, C = x.shape
+    src, _, _ = index_maps(B, T, H, W, window, shift)
+    N = o.shape[1]
+    flat = x.reshape(-1, C)
+    for k, w in enumerate(windows):
+        s = src[int(w) * N:(int(w) + 1) * N]
+        m = s >= 0
+        o[k][m] += flat[s[m]]
+    return o

@@ -12,6 +12,10 @@ Recipe (stands in for Kinetics clips; no dataset is used):
     table ~ N(0, 1); biases ~ N(0, 0.1), so that dropping the mask, the bias or
     a bias vector moves the output far outside the tolerances;
   * values drawn in float32, then rounded once to the run dtype.
+
+Block inputs (layer norm + layer + residual) add, from seeds k = 6, 7, 8: a
+per-token offset ~ N(0, 0.5) added to x (so that the norm's centring matters),
+gamma ~ 1 + N(0, 0.1) and beta ~ N(0, 0.1).
 """
 
 from __future__ import annotations
@@ -82,3 +86,34 @@ def workload_layer_inputs(workload, layer, scale="baseline") -> LayerInputs:
     base = 1000 * workload.index
     return make_layer_inputs(layer.shape, layer.heads, layer.window, workload.dtype, scale,
                              seed=base + layer.seed_offset, x_seed=base)
+
+
+@dataclass
+class BlockInputs:
+    layer: LayerInputs
+    gamma: torch.Tensor
+    beta: torch.Tensor
+
+    def as_f64(self):
+        d = self.layer.as_f64()
+        d["gamma"] = self.gamma.to(torch.float64).numpy()
+        d["beta"] = self.beta.to(torch.float64).numpy()
+        return d
+
+    def to(self, device):
+        return BlockInputs(self.layer.to(device), self.gamma.to(device), self.beta.to(device))
+
+
+def make_block_inputs(shape, heads, window, dtype="bf16", scale="baseline", seed=1000,
+                      x_seed=None) -> BlockInputs:
+    """Inputs for one call of the block's attention half (layer norm, layer, residual)."""
+    B, T, H, W, C = shape
+    dt = _DT[dtype]
+    xs = seed if x_seed is None else x_seed
+    li = make_layer_inputs(shape, heads, window, dtype, scale, seed=seed, x_seed=xs)
+    offset = _randn((B, T, H, W, 1), xs + 6, 0.5)
+    x = (li.x.float() + offset).to(dt).contiguous()
+    gamma = (1.0 + _randn((C,), seed + 7, 0.1)).to(dt).contiguous()
+    beta = _randn((C,), seed + 8, 0.1).to(dt).contiguous()
+    li = LayerInputs(x, li.Wqkv, li.bqkv, li.Wproj, li.bproj, li.table)
+    return BlockInputs(li, gamma, beta)

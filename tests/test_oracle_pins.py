@@ -288,3 +288,76 @@ def test_unmasked_fraction_matches_oracle_regions(oracle_mod):
         reg = region.reshape(g["nW"], g["N"])
         count = sum(int((r[:, None] == r[None, :]).sum()) for r in reg)
         assert layer_work(1, T, H, W, 8, 1, window, shift)["unmasked_pairs"] == count
+
+
+# ---- block (layer norm + layer + residual) -------------------------------------------------------
+def _block_inputs(shape, heads, window, seed=88):
+    from shifted_window_attention_sw_b200.inputs import make_block_inputs
+
+    return make_block_inputs(shape, heads, window, "f32", "sensitivity", seed=seed).as_f64()
+
+
+def _run_block(oracle_mod, a, window, shift, heads, eps=1e-5):
+    return oracle_mod.block_forward(a["x"], a["gamma"], a["beta"], eps, window, shift, a["Wqkv"], a["bqkv"],
+                                    a["Wproj"], a["bproj"], a["table"], heads)
+
+
+def test_b1_layer_norm_matches_torch(oracle_mod):
+    # the norm against the library routine (float64, biased variance, eps inside the root)
+    a = _block_inputs((2, 3, 4, 5, 24), 2, (2, 2, 2))
+    for eps in (1e-5, 1e-2):
+        ref = torch.nn.functional.layer_norm(torch.from_numpy(a["x"]), (24,), torch.from_numpy(a["gamma"]),
+                                             torch.from_numpy(a["beta"]), eps).numpy()
+        np.testing.assert_allclose(oracle_mod.layer_norm(a["x"], a["gamma"], a["beta"], eps), ref,
+                                   rtol=0, atol=1e-12)
+
+
+def test_b2_zero_projection_leaves_the_residual(oracle_mod):
+    # Wproj = 0 and bproj = 0: the attention branch is exactly zero and the block returns x
+    shape, heads, window, shift = (1, 5, 9, 10, 32), 2, (4, 4, 4), (2, 2, 2)
+    a = _block_inputs(shape, heads, window)
+    a["Wproj"] = np.zeros_like(a["Wproj"])
+    a["bproj"] = np.zeros_like(a["bproj"])
+    out = _run_block(oracle_mod, a, window, shift, heads)
+    assert np.array_equal(out, a["x"])
+
+
+def test_b3_constant_tokens_closed_form(oracle_mod):
+    # Tokens whose channels are all equal normalise to beta (zero variance), so with no
+    # padding every token feeds the same key and value: whatever the mask and bias do,
+    # each softmax row sums to 1 and the branch is (beta Wv + bv) Wproj + bproj.
+    shape, heads, window, shift = (1, 4, 6, 6, 16), 2, (2, 3, 3), (1, 1, 1)
+    a = _block_inputs(shape, heads, window)
+    rng = np.random.default_rng(5)
+    a["x"] = np.repeat(rng.normal(size=shape[:-1] + (1,)), shape[-1], axis=-1)
+    C = shape[-1]
+    v = a["beta"] @ a["Wqkv"][:, 2 * C:] + a["bqkv"][2 * C:]
+    branch = v @ a["Wproj"] + a["bproj"]
+    out = _run_block(oracle_mod, a, window, shift, heads)
+    np.testing.assert_allclose(out, a["x"] + branch, rtol=0, atol=1e-12)
+
+
+def test_b4_token_offset_invariance(oracle_mod):
+    # layer norm removes a per-token offset c, so block(x + c) = block(x) + c
+    shape, heads, window, shift = (1, 6, 9, 10, 32), 1, (4, 7, 7), (2, 3, 3)
+    a = _block_inputs(shape, heads, window)
+    c = np.random.default_rng(6).normal(scale=3.0, size=shape[:-1] + (1,))
+    out0 = _run_block(oracle_mod, a, window, shift, heads)
+    b = dict(a)
+    b["x"] = a["x"] + c
+    out1 = _run_block(oracle_mod, b, window, shift, heads)
+    np.testing.assert_allclose(out1 - out0, np.broadcast_to(c, out0.shape), rtol=0, atol=1e-9)
+
+
+def test_b5_padding_is_zero_after_the_norm(oracle_mod):
+    # The norm comes before the padding: padded slots are zero tokens for the layer, not
+    # the norm of zeros (beta). Built from the layer oracle on an explicitly padded input.
+    shape, heads, window, shift = (1, 3, 5, 6, 16), 2, (2, 3, 3), (1, 1, 1)
+    a = _block_inputs(shape, heads, window)
+    y = oracle_mod.layer_norm(a["x"], a["gamma"], a["beta"])
+    padded = np.zeros((1, 4, 6, 6, 16))
+    padded[:, :3, :5, :6] = y
+    full = oracle_mod.forward(padded, window, shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"], a["table"],
+                              heads)
+    out = _run_block(oracle_mod, a, window, shift, heads)
+    np.testing.assert_allclose(out, a["x"] + full[:, :3, :5, :6], rtol=0, atol=1e-12)
