@@ -407,6 +407,93 @@ def run_gpu(args):
     return 0
 
 
+def run_block(args):
+    """``--block``: the attention half of the blocks on the same workload, out = x +
+    layer(LN(x)) per layer, through the fused entry (vswin_block_msa_forward) and,
+    for comparison, unfused (torch layer_norm, vswin_wmsa_forward, torch add). One
+    GPU; prints its own JSON line."""
+    from shifted_window_attention_sw_b200 import build as build_mod
+    from shifted_window_attention_sw_b200 import vswin
+    from shifted_window_attention_sw_b200.inputs import make_block_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    build_mod.build()
+    vswin.lib()
+    wl = WORKLOADS[args.workload]
+    layers = wl.layers
+    base = 1000 * wl.index
+    bins = [make_block_inputs(ly.shape, ly.heads, ly.window, wl.dtype, "baseline", seed=base + ly.seed_offset,
+                              x_seed=base).to(device) for ly in layers]
+    outs = [torch.empty_like(b.layer.x) for b in bins]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    eps = 1e-5
+
+    def fused():
+        for ly, b, o in zip(layers, bins, outs):
+            li = b.layer
+            vswin.block_msa_forward(li.x, ly.window, ly.shift, b.gamma, b.beta, eps, li.Wqkv, li.bqkv, li.Wproj,
+                                    li.bproj, li.table, ly.heads, out=o, stream=stream)
+
+    def unfused():
+        for ly, b, o in zip(layers, bins, outs):
+            li = b.layer
+            y = torch.nn.functional.layer_norm(li.x, (ly.C,), b.gamma, b.beta, eps)
+            vswin.wmsa_forward(y, ly.window, ly.shift, li.Wqkv, li.bqkv, li.Wproj, li.bproj, li.table, ly.heads,
+                               out=o, stream=stream)
+            o.add_(li.x)
+
+    def timed(fn, profile):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize(device)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        launches0 = vswin.launch_count()
+        if profile:
+            vswin.profile_enable(True)
+        sampler = ClockSampler(device)
+        sampler.start()
+        for k in range(args.steps):
+            flush.zero_()
+            evs[k][0].record(stream)
+            fn()
+            evs[k][1].record(stream)
+        torch.cuda.synchronize(device)
+        clocks = sampler.stop()
+        prof = None
+        if profile:
+            vswin.profile_enable(False)
+            prof = vswin.profile_collect()
+        if vswin.poll_error(stream) != vswin.OK:
+            raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
+        ms = [a.elapsed_time(b) for a, b in evs]
+        return sum(ms) / len(ms), prof, vswin.launch_count() - launches0, clocks
+
+    f_ms, prof, launches, clocks = timed(fused, True)
+    u_ms, _, _, u_clocks = timed(unfused, False)
+    tokens = step_work(wl)["tokens"]
+    cfg = workload_config(wl)
+    cfg["ln_eps"] = eps
+    line = {
+        "metric": "block attention-half tokens/s (LN + (S)W-MSA + residual), " + wl.name,
+        "value": tokens / (f_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": f_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "api": "vswin_block_msa_forward",
+        "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+        "gpu_launches": int(launches),
+        "unfused": {"ms_per_step": u_ms, "value": tokens / (u_ms / 1e3),
+                    "what": "torch layer_norm + vswin_wmsa_forward + torch add_", "clocks": u_clocks},
+        "fused_speedup": u_ms / f_ms,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,11 +504,15 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=20.0)
+    ap.add_argument("--block", action="store_true",
+                    help="time the blocks' attention half (LN, layer, residual), fused and unfused, on one GPU")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.block:
+        return run_block(args)
     return run_gpu(args)
 
 

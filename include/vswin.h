@@ -84,6 +84,33 @@ int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int hea
                        const void* bias_table, void* out, void* stream);
 
 /*
+ * bf16 forward of a block's attention half: out = x + layer(LN(x)), the
+ * pre-norm and the residual fused into the layer ("Video Swin Transformer"
+ * summary page, Method step 3 and eq. 1; code walk-through page, section 1.2:
+ * LayerNorm comes before F.pad, so padded slots are zero tokens for the layer,
+ * and the shortcut is added after the window reverse).
+ *   LN(x) = (x - mean) / sqrt(var + ln_eps) * ln_gamma + ln_beta per token over
+ *   its C channels, var the biased variance (torch.nn.LayerNorm; its default
+ *   eps is 1e-5).
+ * ln_gamma, ln_beta: bf16 [C], device, 2-byte aligned; ln_eps finite, >= 0.
+ * Every other argument, layout and requirement is that of vswin_wmsa_forward,
+ * except that out may be x itself (in place); partial overlap is refused.
+ * Arithmetic: the norm is folded into the weights once per call
+ * (Wt = bf16(diag(gamma) Wqkv), its fp32 column sums, bqkv + beta Wqkv) and
+ * applied per row in the QKV epilogue as rstd * (x Wt - mean * colsum(Wt)) +
+ * (bqkv + beta Wqkv), with per-token mean and rstd in fp32; the residual is
+ * added to the fp32 projection before the one rounding to bf16. Tokens whose
+ * variance overflows fp32 (|x| above ~1e19) are out of range. Scratch: the
+ * layer's plus 8 bytes per window slot and C*3C*2 + 24*C bytes for the folded
+ * weights, from the same pool.
+ */
+int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, int heads,
+                            const int* window, const int* shift,
+                            const void* ln_gamma, const void* ln_beta, float ln_eps,
+                            const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                            const void* bias_table, void* out, void* stream);
+
+/*
  * fp32 layer forward (plain FP32 FMA arithmetic, no tensor cores): every
  * tensor is float. Any d; N <= 4096. Pointers 4-byte aligned; x must not
  * overlap out. Scratch: stream-ordered, from the library's pool (see above).

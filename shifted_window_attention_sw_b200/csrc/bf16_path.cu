@@ -97,6 +97,14 @@ struct GemmArgs {
   float qscale;
   SlabLayout slab;
   const int* rowsrc;          // [rows] source token of each chunk row (-1 = padding), or null
+  // Block fusion (all null for the plain layer). QKV: the pre-norm folded into
+  // the epilogue -- Wt is diag(gamma) Wqkv, ln_stats[r] = (-mean * rstd, rstd)
+  // of chunk row r's token ((0, 0) for padding), ln_colsum the column sums of
+  // Wt, ln_bias = bqkv + beta Wqkv. PROJ: resid (x) added to every output row.
+  const float2* ln_stats;
+  const float* ln_colsum;
+  const float* ln_bias;
+  const __nv_bfloat16* resid;
 };
 
 __host__ __device__ constexpr int gemm_smem_bytes() {
@@ -124,7 +132,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int MODE>
+template <int MODE, bool FUSE>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sA = smem;
@@ -250,9 +258,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
     long long dst_row = -1;     // kPROJ: token
     long long slab_win = 0;     // kQKV: chunk-relative window
     int slot = 0;
+    float2 st = make_float2(0.f, 0.f);  // kQKV + FUSE: (-mean * rstd, rstd) of the row's token
     if (MODE == kQKV) {
       slab_win = r / g.N;
       slot = (int)(r % g.N);
+      if (FUSE && row_ok) st = a.ln_stats[r];
     } else if (row_ok) {
       const long long gr = a.win0 * g.N + r;
       dst_row = slot_source(g, gr / g.N, (int)(gr % g.N));
@@ -263,8 +273,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
       tmem_wait_ld();
       const int col = n0 + c * 16;
       float v[16];
+      if (FUSE && MODE == kQKV && st.y != 0.f) {
+        // LN(x) Wqkv + bqkv = rstd * (x Wt - mean * colsum) + ln_bias
 #pragma unroll
-      for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(u[k]) + __bfloat162float(a.bias[col + k]);
+        for (int k = 0; k < 16; ++k)
+          v[k] = fmaf(st.y, __uint_as_float(u[k]), fmaf(st.x, a.ln_colsum[col + k], a.ln_bias[col + k]));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(u[k]) + __bfloat162float(a.bias[col + k]);
+      }
+      if (FUSE && MODE == kPROJ && dst_row >= 0) {
+        const __nv_bfloat16* xr = a.resid + dst_row * g.C + col;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] += __bfloat162float(xr[k]);
+      }
       uint4 w0, w1;
       if (MODE == kQKV && row_ok) {
         const int which = col / g.C;
@@ -317,9 +339,10 @@ constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
 constexpr int kWsMaxBBytes = 96 * 1024;
 
 __host__ __device__ inline int ws_a_bytes(int K) { return kBM * K * 2; }
-// B slice, A stages, bias (BN floats), column-group table (BN / 8 x 16 B), barriers
-__host__ __device__ inline int ws_smem_bytes(int K, int BN, int stages) {
-  return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + 256;
+// B slice, A stages, bias (BN floats), column-group table (BN / 8 x 16 B), with
+// the fused pre-norm the column sums and folded bias (2 x BN floats), barriers
+__host__ __device__ inline int ws_smem_bytes(int K, int BN, int stages, bool ln = false) {
+  return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + (ln ? BN * 8 : 0) + 256;
 }
 
 // Destination facts of one group of 8 output columns of the QKV GEMM: element
@@ -341,15 +364,120 @@ __global__ void row_source_kernel(Geom g, long long win0, long long rows, int* _
   }
 }
 
-template <int MODE, int STAGES>
+// Pre-norm folded into the QKV weights ("Video Swin Transformer" summary page,
+// eq. 1: the layer reads LN(x)). Since LN(x) = rstd * (x - mean) * gamma + beta,
+//   LN(x) Wqkv + bqkv = rstd * (x Wt - mean * colsum(Wt)) + (bqkv + beta Wqkv)
+// with Wt = diag(gamma) Wqkv. Wt is rounded to bf16 (gamma * w is exact in
+// fp32, so this is the only rounding) and colsum is taken from the rounded Wt
+// so that the mean term cancels what x Wt accumulates. Block (32 x 32): 32
+// output columns, the C rows split over 32 thread rows (independent loads),
+// partial sums reduced in shared memory.
+constexpr int kFoldCols = 32, kFoldRows = 32;
+__global__ void __launch_bounds__(kFoldCols * kFoldRows) ln_fold_kernel(
+    int C, int N3, const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta,
+    const __nv_bfloat16* __restrict__ Wqkv, const __nv_bfloat16* __restrict__ bqkv, __nv_bfloat16* __restrict__ wt,
+    float* __restrict__ colsum, float* __restrict__ bias_ln) {
+  __shared__ float s_cs[kFoldRows][kFoldCols + 1], s_bb[kFoldRows][kFoldCols + 1];
+  const int tx = threadIdx.x % kFoldCols, ty = threadIdx.x / kFoldCols;
+  const int j = blockIdx.x * kFoldCols + tx;
+  float cs = 0.f, bb = 0.f;
+  if (j < N3) {
+#pragma unroll 4
+    for (int c = ty; c < C; c += kFoldRows) {
+      const float w = __bfloat162float(Wqkv[(size_t)c * N3 + j]);
+      const __nv_bfloat16 wg = __float2bfloat16_rn(__bfloat162float(gamma[c]) * w);
+      wt[(size_t)c * N3 + j] = wg;
+      cs += __bfloat162float(wg);
+      bb = fmaf(__bfloat162float(beta[c]), w, bb);
+    }
+  }
+  s_cs[ty][tx] = cs;
+  s_bb[ty][tx] = bb;
+  __syncthreads();
+  if (ty == 0 && j < N3) {
+    for (int k = 1; k < kFoldRows; ++k) {
+      cs += s_cs[k][tx];
+      bb += s_bb[k][tx];
+    }
+    colsum[j] = cs;
+    bias_ln[j] = __bfloat162float(bqkv[j]) + bb;
+  }
+}
+
+// Row table plus the norm's statistics of each chunk row's token: rowsrc[r] as
+// row_source_kernel writes it and stats[r] = (-mean * rstd, rstd) with the
+// biased variance and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
+// definition), (0, 0) for a padding row. Four lanes per row (the first one
+// does the row's index math), each summing C/32 chunks of 8 channels; two
+// passes (mean, then squared deviations, the second re-reading the row from
+// L1). C is a multiple of 32.
+__global__ void row_stats_kernel(Geom g, long long win0, long long rows, const __nv_bfloat16* __restrict__ x,
+                                 float eps, int* __restrict__ rowsrc, float2* __restrict__ stats) {
+  const long long nthr = (long long)gridDim.x * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  const int cq = lane & 3;
+  const long long base0 = (long long)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  // whole warps iterate together (same trip count), so the shuffles see all lanes
+  for (long long base = base0; base < rows * 4; base += nthr) {
+    const long long i = base + lane;
+    const bool valid = i < rows * 4;
+    const long long r = i >> 2;
+    long long tok = -1;
+    if (valid && cq == 0) {
+      const long long gr = win0 * g.N + r;
+      tok = slot_source(g, gr / g.N, (int)(gr % g.N));
+    }
+    tok = __shfl_sync(0xffffffffu, tok, lane & ~3);  // the row's index math once, on its first lane
+    const __nv_bfloat16* row = x + (tok < 0 ? 0 : tok * g.C);
+    float sum = 0.f;
+    if (tok >= 0)
+      for (int kc = cq; kc < g.C / 8; kc += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 8);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          sum += f.x + f.y;
+        }
+      }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    const float mean = sum / (float)g.C;
+    float ss = 0.f;
+    if (tok >= 0)
+      for (int kc = cq; kc < g.C / 8; kc += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 8);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          const float d0 = f.x - mean, d1 = f.y - mean;
+          ss = fmaf(d0, d0, fmaf(d1, d1, ss));
+        }
+      }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    if (valid && cq == 0) {
+      rowsrc[r] = (int)tok;
+      const float rstd = 1.0f / sqrtf(ss / (float)g.C + eps);
+      stats[r] = tok < 0 ? make_float2(0.f, 0.f) : make_float2(-mean * rstd, rstd);
+    }
+  }
+}
+
+template <int MODE, int STAGES, bool FUSE>
 __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  constexpr bool kLn = FUSE && MODE == kQKV;      // pre-norm folded into the QKV epilogue
+  constexpr bool kResid = FUSE && MODE == kPROJ;  // residual added in the projection epilogue
   const int K = a.K, BN = a.BN;
   uint8_t* sB = smem;                                     // K x BN, MN-major operand layout
   uint8_t* sA = sB + K * BN * 2;                          // STAGES x (128 x K), K-major
   float* sBias = reinterpret_cast<float*>(sA + STAGES * ws_a_bytes(K));  // bias x column scale
   ColGroup* sGrp = reinterpret_cast<ColGroup*>(sBias + BN);                // [BN / 8]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sGrp + BN / 8);
+  float* sCs = reinterpret_cast<float*>(sGrp + BN / 8);  // kLn: column sums of Wt
+  float* sBb = sCs + BN;                                 // kLn: folded bias x column scale
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kLn ? sBb + BN : sCs);
   uint64_t* b_full = bars;                 // B resident
   uint64_t* a_full = bars + 1;             // [STAGES]
   uint64_t* a_free = a_full + STAGES;      // [STAGES]
@@ -410,6 +538,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   for (int c = tid; c < BN; c += kWsThreads) {
     const float sc = (MODE == kQKV && (((n0 + c) >> 5) / g.heads) == 0) ? a.qscale : 1.0f;
     sBias[c] = __bfloat162float(a.bias[n0 + c]) * sc;
+    if (kLn) {
+      sCs[c] = a.ln_colsum[n0 + c];
+      sBb[c] = a.ln_bias[n0 + c] * sc;
+    }
   }
   if (warp == kWsMmaWarp) {
     tmem_alloc(s_tmem, tcols);
@@ -531,7 +663,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       // this row's destination: QKV, the window's block and the row term of the
       // q slab and of the k / v slabs; projection, the output row
       __nv_bfloat16* rbase = nullptr;
+      const __nv_bfloat16* xres = nullptr;  // kResid: this row's residual, same columns as rbase
       int q_term = 0, kv_term = 0;
+      // kLn: (-mean * rstd, rstd) of this row's token, (0, 0) for a padding row
+      const float2 st = (kLn && row_ok) ? a.ln_stats[r] : make_float2(0.f, 0.f);
       if (row_ok) {
         if (MODE == kQKV) {
           const int ri = (int)r;  // rows < 2^31 (checked by the caller)
@@ -543,21 +678,37 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
           rbase = a.dst + (size_t)slab_win * win_elems;
         } else {
           const long long dr = dr_cur;
-          if (dr >= 0) rbase = a.dst + dr * g.C + n0;
+          if (dr >= 0) {
+            rbase = a.dst + dr * g.C + n0;
+            if (kResid) xres = a.resid + dr * g.C + n0;
+          }
         }
       }
+      // columns handled per TMEM wait (the residual's registers and the norm's
+      // extra terms need room)
+      constexpr int kCh = kResid ? 48 : kLn ? 72 : 96;
+      uint4 xr[kResid ? kCh / 8 : 1];
+      auto load_resid = [&](int c0) {
+        const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;
+#pragma unroll
+        for (int j = 0; j < kCh / 8; ++j)
+          xr[j] = (xres && j * 8 < n) ? *reinterpret_cast<const uint4*>(xres + c0 + 8 * j) : make_uint4(0, 0, 0, 0);
+      };
+      // the first column chunk's residual is in flight while the accumulator is awaited
+      if (kResid) load_resid(hf * cw);
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 70);
       if (!s_abort && !mbar_wait(&acc_full[buf], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 71);
       tc_fence_after();
       if (!s_abort && m * kBM + q * 32 < a.rows) {
-        // all of this warp's columns (up to 96 at a time) loaded before one wait
-        for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += 96) {
-          const int n = (hf + 1) * cw - c0 < 96 ? (hf + 1) * cw - c0 : 96;  // a multiple of 8
-          uint32_t u[96];
+        // all of this warp's columns (up to kCh at a time) loaded before one wait
+        for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += kCh) {
+          const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;  // a multiple of 8
+          uint32_t u[kCh];
+          if (kResid && c0 != hf * cw) load_resid(c0);
           const uint32_t ta = tmem + lane_base + buf * BN + c0;
 #pragma unroll
-          for (int j = 0; j < 12; ++j)
+          for (int j = 0; j < kCh / 8; ++j)
             if (j * 8 < n)
               asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                            : "=r"(u[8 * j + 0]), "=r"(u[8 * j + 1]), "=r"(u[8 * j + 2]), "=r"(u[8 * j + 3]),
@@ -565,22 +716,46 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
                            : "r"(ta + 8 * j));
           tmem_wait_ld_keep(u);
 #pragma unroll
-          for (int g8 = 0; g8 < 12; ++g8) {
+          for (int g8 = 0; g8 < kCh / 8; ++g8) {
             if (g8 * 8 >= n) break;
             const int cc = c0 + g8 * 8;
-            const float4 b0 = *reinterpret_cast<const float4*>(sBias + cc);
-            const float4 b1 = *reinterpret_cast<const float4*>(sBias + cc + 4);
             const ColGroup cg = sGrp[cc >> 3];
-            const float2 sc = make_float2(cg.scale, cg.scale);
-            // v = acc * scale + bias * scale, two columns per instruction
-            const float2 v01 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 0]), __uint_as_float(u[g8 * 8 + 1])),
-                                          sc, make_float2(b0.x, b0.y));
-            const float2 v23 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 2]), __uint_as_float(u[g8 * 8 + 3])),
-                                          sc, make_float2(b0.z, b0.w));
-            const float2 v45 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 4]), __uint_as_float(u[g8 * 8 + 5])),
-                                          sc, make_float2(b1.x, b1.y));
-            const float2 v67 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 6]), __uint_as_float(u[g8 * 8 + 7])),
-                                          sc, make_float2(b1.z, b1.w));
+            // plain: v = acc * scale + bias * scale. kLn (a token row): v = rs * acc
+            // + (ns * colsum + folded bias * scale) with rs = rstd * scale, ns =
+            // -mean * rstd * scale; a padding row (rstd = 0) keeps the plain bias.
+            const float* bsrc = (kLn && st.y != 0.f) ? sBb : sBias;
+            float4 b0 = *reinterpret_cast<const float4*>(bsrc + cc);
+            float4 b1 = *reinterpret_cast<const float4*>(bsrc + cc + 4);
+            float2 sc = make_float2(cg.scale, cg.scale);
+            if (kLn) {
+              const float rs = st.y * cg.scale, ns = st.x * cg.scale;
+              const float4 c0v = *reinterpret_cast<const float4*>(sCs + cc);
+              const float4 c1v = *reinterpret_cast<const float4*>(sCs + cc + 4);
+              const float2 ns2 = make_float2(ns, ns);
+              const float2 t01 = __ffma2_rn(make_float2(c0v.x, c0v.y), ns2, make_float2(b0.x, b0.y));
+              const float2 t23 = __ffma2_rn(make_float2(c0v.z, c0v.w), ns2, make_float2(b0.z, b0.w));
+              const float2 t45 = __ffma2_rn(make_float2(c1v.x, c1v.y), ns2, make_float2(b1.x, b1.y));
+              const float2 t67 = __ffma2_rn(make_float2(c1v.z, c1v.w), ns2, make_float2(b1.z, b1.w));
+              b0 = make_float4(t01.x, t01.y, t23.x, t23.y);
+              b1 = make_float4(t45.x, t45.y, t67.x, t67.y);
+              if (st.y != 0.f) sc = make_float2(rs, rs);
+            }
+            // two columns per instruction
+            float2 v01 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 0]), __uint_as_float(u[g8 * 8 + 1])),
+                                    sc, make_float2(b0.x, b0.y));
+            float2 v23 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 2]), __uint_as_float(u[g8 * 8 + 3])),
+                                    sc, make_float2(b0.z, b0.w));
+            float2 v45 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 4]), __uint_as_float(u[g8 * 8 + 5])),
+                                    sc, make_float2(b1.x, b1.y));
+            float2 v67 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 6]), __uint_as_float(u[g8 * 8 + 7])),
+                                    sc, make_float2(b1.z, b1.w));
+            if (kResid) {
+              const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xr[g8]);
+              v01 = __fadd2_rn(v01, __bfloat1622float2(xp[0]));
+              v23 = __fadd2_rn(v23, __bfloat1622float2(xp[1]));
+              v45 = __fadd2_rn(v45, __bfloat1622float2(xp[2]));
+              v67 = __fadd2_rn(v67, __bfloat1622float2(xp[3]));
+            }
             const uint4 w = make_uint4(pack_bf16x2(v01.x, v01.y), pack_bf16x2(v23.x, v23.y),
                                        pack_bf16x2(v45.x, v45.y), pack_bf16x2(v67.x, v67.y));
             if (rbase) {
@@ -1686,7 +1861,7 @@ int pick_bn(int n) {
   return 0;
 }
 
-template <int MODE>
+template <int MODE, bool FUSE>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
   if (a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0) {
     int dev = 0, sms = 148;
@@ -1699,10 +1874,11 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
     if (per_nt > mtiles) per_nt = mtiles;
     // four A stages when they fit, else two; at least 116 KB so that one CTA
     // (up to 512 TMEM columns) owns each SM
-    const bool four = ws_smem_bytes(a.K, a.BN, 4) <= 220 * 1024;
-    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2);
+    const bool ln = FUSE && MODE == kQKV;
+    const bool four = ws_smem_bytes(a.K, a.BN, 4, ln) <= 220 * 1024;
+    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2, ln);
     if (smem_ws < 116 * 1024) smem_ws = 116 * 1024;
-    auto kern = four ? gemm_ws_kernel<MODE, 4> : gemm_ws_kernel<MODE, 2>;
+    auto kern = four ? gemm_ws_kernel<MODE, 4, FUSE> : gemm_ws_kernel<MODE, 2, FUSE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_ws);
     if (e != cudaSuccess) return e;
     prof_begin(MODE == kQKV ? kKindQkv : kKindProj, st);
@@ -1712,11 +1888,11 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
     return cudaGetLastError();
   }
   cudaError_t e =
-      cudaFuncSetAttribute(gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes());
+      cudaFuncSetAttribute(gemm_kernel<MODE, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes());
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((a.rows + kBM - 1) / kBM), (unsigned)(a.Ntot / a.BN));
   prof_begin(MODE == kQKV ? kKindQkv : kKindProj, st);
-  gemm_kernel<MODE><<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(a);
+  gemm_kernel<MODE, FUSE><<<grid, kGemmThreads, gemm_smem_bytes(), st>>>(a);
   prof_end(MODE == kQKV ? kKindQkv : kKindProj, st);
   count_launch();
   return cudaGetLastError();
@@ -1739,20 +1915,48 @@ size_t bf16_scratch_bytes(const Geom& g, long long nwin) {
   return qkv + o + rows;
 }
 
+size_t bf16_block_scratch_bytes(const Geom& g, long long nwin) {
+  return bf16_scratch_bytes(g, nwin) + ((size_t)nwin * g.N * 8 + 255) / 256 * 256;
+}
+
+cudaError_t launch_ln_fold(const Geom& g, const void* gamma, const void* beta, const void* Wqkv, const void* bqkv,
+                           const BlockFuse& f, cudaStream_t st) {
+  const int n3 = 3 * g.C;
+  prof_begin(kKindOther, st);
+  ln_fold_kernel<<<(unsigned)((n3 + kFoldCols - 1) / kFoldCols), kFoldCols * kFoldRows, 0, st>>>(
+      g.C, n3, static_cast<const __nv_bfloat16*>(gamma), static_cast<const __nv_bfloat16*>(beta),
+      static_cast<const __nv_bfloat16*>(Wqkv), static_cast<const __nv_bfloat16*>(bqkv),
+      static_cast<__nv_bfloat16*>(f.wt), f.colsum, f.bias_ln);
+  prof_end(kKindOther, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
                               const void* bqkv, const void* Wproj, const void* bproj, const void* table,
-                              void* out, void* scratch, long long win0, long long nwin, cudaStream_t st) {
+                              void* out, void* scratch, long long win0, long long nwin, cudaStream_t st,
+                              const BlockFuse* fuse) {
   __nv_bfloat16* qkv = static_cast<__nv_bfloat16*>(scratch);
   const SlabLayout L = slab_layout(g);
   __nv_bfloat16* o = qkv + (size_t)nwin * g.heads * L.head_elems();
   int* rowsrc = reinterpret_cast<int*>(o + (size_t)nwin * g.N * g.C);
+  // fused block: per-row norm statistics after the row table
+  float2* stats = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(rowsrc) +
+                                            ((size_t)nwin * g.N * 4 + 255) / 256 * 256);
 
   {
     const long long rows = nwin * g.N;
-    long long blocks = (rows + 255) / 256;
-    if (blocks > 2048) blocks = 2048;
     prof_begin(kKindOther, st);
-    row_source_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, rowsrc);
+    if (fuse) {
+      long long blocks = (rows * 4 + 255) / 256;
+      if (blocks > 4096) blocks = 4096;
+      row_stats_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, static_cast<const __nv_bfloat16*>(x),
+                                                          fuse->eps, rowsrc, stats);
+    } else {
+      long long blocks = (rows + 255) / 256;
+      if (blocks > 2048) blocks = 2048;
+      row_source_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, rowsrc);
+    }
     prof_end(kKindOther, st);
     count_launch();
     cudaError_t e0 = cudaGetLastError();
@@ -1774,7 +1978,13 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   ga.qscale = kLog2e / sqrtf((float)kD);
   ga.slab = L;
   ga.rowsrc = rowsrc;
-  cudaError_t e = launch_gemm<kQKV>(ga, st);
+  if (fuse) {
+    ga.Wt = static_cast<const __nv_bfloat16*>(fuse->wt);
+    ga.ln_stats = stats;
+    ga.ln_colsum = fuse->colsum;
+    ga.ln_bias = fuse->bias_ln;
+  }
+  cudaError_t e = fuse ? launch_gemm<kQKV, true>(ga, st) : launch_gemm<kQKV, false>(ga, st);
   if (e != cudaSuccess) return e;
 
   AttnArgs aa{};
@@ -1807,7 +2017,11 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   gp.Ntot = g.C;
   gp.BN = pick_bn(g.C);
   gp.qscale = 1.0f;
-  return launch_gemm<kPROJ>(gp, st);
+  if (fuse) {
+    gp.resid = static_cast<const __nv_bfloat16*>(x);
+    return launch_gemm<kPROJ, true>(gp, st);
+  }
+  return launch_gemm<kPROJ, false>(gp, st);
 }
 
 }  // namespace vswin

@@ -42,8 +42,24 @@ cudaError_t launch_selftest_timeout(const KernelCtx& ctx, cudaStream_t st);
 bool bf16_window_supported(const Geom& g);
 // Scratch for `nwin` windows: QKV slabs then the attention output.
 size_t bf16_scratch_bytes(const Geom& g, long long nwin);
+// The block's pre-norm and residual fused into the layer: the norm folded into
+// the QKV weights (launch_ln_fold fills these buffers once per call) and
+// applied per row in the QKV epilogue; x added in the projection epilogue.
+struct BlockFuse {
+  void* wt;        // [C][3C] bf16: diag(gamma) Wqkv
+  float* colsum;   // [3C] column sums of wt
+  float* bias_ln;  // [3C] bqkv + beta Wqkv
+  float eps;
+};
+cudaError_t launch_ln_fold(const Geom& g, const void* gamma, const void* beta, const void* Wqkv, const void* bqkv,
+                           const BlockFuse& f, cudaStream_t st);
+// Chunk scratch of the fused block: the layer's plus the per-row norm statistics.
+size_t bf16_block_scratch_bytes(const Geom& g, long long nwin);
+// One chunk of windows; `fuse` null for the plain layer, else the fused block
+// (x is then also the residual, and out may be x itself).
 cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
                               const void* bqkv, const void* Wproj, const void* bproj, const void* table,
-                              void* out, void* scratch, long long win0, long long nwin, cudaStream_t st);
+                              void* out, void* scratch, long long win0, long long nwin, cudaStream_t st,
+                              const BlockFuse* fuse = nullptr);
 
 }  // namespace vswin

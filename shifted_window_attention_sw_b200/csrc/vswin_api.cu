@@ -1,6 +1,7 @@
 // C ABI of the library: argument validation, error reporting, scratch
 // management and dispatch to the fp32 and bf16 paths. See include/vswin.h.
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -160,7 +161,8 @@ int build_geom(int B, int T, int H, int W, int C, int heads, const int* window, 
 }
 
 int check_layer_ptrs(const void* x, const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
-                     const void* table, const void* out, const Geom& g, size_t elem, size_t align) {
+                     const void* table, const void* out, const Geom& g, size_t elem, size_t align,
+                     bool allow_in_place = false) {
   const void* ptrs[] = {x, Wqkv, bqkv, Wproj, bproj, table, out};
   const char* names[] = {"x", "Wqkv", "bqkv", "Wproj", "bproj", "bias_table", "out"};
   for (int k = 0; k < 7; ++k)
@@ -174,7 +176,8 @@ int check_layer_ptrs(const void* x, const void* Wqkv, const void* bqkv, const vo
   for (int k = 0; k < 3; ++k)
     if (!aligned(small[k], elem)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not %zu-byte aligned", smalln[k], elem);
   const size_t act = (size_t)g.tokens * g.C * elem;
-  if (overlap(x, act, out, act)) return fail(VSWIN_ERR_INVALID_ARG, "x and out overlap");
+  if (!(allow_in_place && x == out) && overlap(x, act, out, act))
+    return fail(VSWIN_ERR_INVALID_ARG, allow_in_place ? "x and out overlap without being equal" : "x and out overlap");
   return VSWIN_OK;
 }
 
@@ -219,6 +222,45 @@ int forward_bf16_device(const void* x, const Geom& g, const void* Wqkv, const vo
       cudaFreeAsync(scratch, st);
       return fail_cuda(e, "bf16 kernel launch");
     }
+  }
+  e = cudaFreeAsync(scratch, st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaFreeAsync");
+  return VSWIN_OK;
+}
+
+// The block's attention half: the norm folded once into scratch weights, then
+// the chunks with the fused statistics / epilogues.
+int forward_block_device(const void* x, const Geom& g, const void* gamma, const void* beta, float eps,
+                         const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj, const void* table,
+                         void* out, cudaStream_t st) {
+  if (g.d != 32) return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path needs head width 32 (C/heads = %d)", g.d);
+  if (!bf16_window_supported(g))
+    return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path has no kernel for window (%d,%d,%d)", g.win[0], g.win[1],
+                g.win[2]);
+  KernelCtx ctx;
+  int status = make_ctx(&ctx);
+  if (status != VSWIN_OK) return status;
+  const long long per_chunk = chunk_windows(g);
+  const size_t chunk_bytes = (bf16_block_scratch_bytes(g, per_chunk) + 255) / 256 * 256;
+  const size_t wt_bytes = ((size_t)g.C * 3 * g.C * 2 + 255) / 256 * 256;
+  const size_t vec_bytes = ((size_t)3 * g.C * 4 + 255) / 256 * 256;
+  void* scratch = nullptr;
+  status = scratch_alloc(&scratch, chunk_bytes + wt_bytes + 2 * vec_bytes, st);
+  if (status != VSWIN_OK) return status;
+  uint8_t* fold = static_cast<uint8_t*>(scratch) + chunk_bytes;
+  BlockFuse f;
+  f.wt = fold;
+  f.colsum = reinterpret_cast<float*>(fold + wt_bytes);
+  f.bias_ln = reinterpret_cast<float*>(fold + wt_bytes + vec_bytes);
+  f.eps = eps;
+  cudaError_t e = launch_ln_fold(g, gamma, beta, Wqkv, bqkv, f, st);
+  for (long long w0 = 0; e == cudaSuccess && w0 < g.windows; w0 += per_chunk) {
+    const long long n = (g.windows - w0) < per_chunk ? (g.windows - w0) : per_chunk;
+    e = launch_bf16_chunk(g, ctx, x, Wqkv, bqkv, Wproj, bproj, table, out, scratch, w0, n, st, &f);
+  }
+  if (e != cudaSuccess) {
+    cudaFreeAsync(scratch, st);
+    return fail_cuda(e, "bf16 block kernel launch");
   }
   e = cudaFreeAsync(scratch, st);
   if (e != cudaSuccess) return fail_cuda(e, "cudaFreeAsync");
@@ -355,6 +397,24 @@ int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int hea
   st = check_layer_ptrs(x, Wqkv, bqkv, Wproj, bproj, bias_table, out, g, 2, 16);
   if (st != VSWIN_OK) return st;
   return forward_bf16_device(x, g, Wqkv, bqkv, Wproj, bproj, bias_table, out, static_cast<cudaStream_t>(stream));
+}
+
+int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                            const int* shift, const void* ln_gamma, const void* ln_beta, float ln_eps,
+                            const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                            const void* bias_table, void* out, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  st = check_layer_ptrs(x, Wqkv, bqkv, Wproj, bproj, bias_table, out, g, 2, 16, true);
+  if (st != VSWIN_OK) return st;
+  if (!ln_gamma || !ln_beta) return fail(VSWIN_ERR_INVALID_ARG, "ln_gamma and ln_beta must be non-NULL");
+  if (!aligned(ln_gamma, 2) || !aligned(ln_beta, 2))
+    return fail(VSWIN_ERR_INVALID_ARG, "ln_gamma and ln_beta must be 2-byte aligned");
+  if (!(ln_eps >= 0.f) || !std::isfinite(ln_eps))
+    return fail(VSWIN_ERR_INVALID_ARG, "ln_eps must be finite and >= 0 (got %g)", (double)ln_eps);
+  return forward_block_device(x, g, ln_gamma, ln_beta, ln_eps, Wqkv, bqkv, Wproj, bproj, bias_table, out,
+                              static_cast<cudaStream_t>(stream));
 }
 
 int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,

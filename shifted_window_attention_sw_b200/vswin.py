@@ -34,6 +34,7 @@ EXPORTS = (
     "vswin_profile_collect",
     "vswin_wmsa_forward_noalloc",
     "vswin_set_exact_softmax",
+    "vswin_block_msa_forward",
 )
 
 KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other")
@@ -65,6 +66,8 @@ def lib():
             fn = getattr(L, name)
             fn.argtypes = layer
             fn.restype = _I
+        L.vswin_block_msa_forward.argtypes = layer[:9] + [_P, _P, ctypes.c_float] + layer[9:]
+        L.vswin_block_msa_forward.restype = _I
         L.vswin_wmsa_index_maps.argtypes = [_I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P]
         L.vswin_wmsa_index_maps.restype = _I
         L.vswin_clamp_window.argtypes = [_I, _I, _I, _IP, _IP, _IP, _IP]
@@ -139,6 +142,21 @@ def wmsa_forward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=N
     _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.bfloat16)
     return _layer_call(lib().vswin_wmsa_forward, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out,
                        stream)
+
+
+def block_msa_forward(x, window, shift, gamma, beta, eps, Wqkv, bqkv, Wproj, bproj, table, heads, out=None,
+                      stream=None):
+    """bf16 forward of a block's attention half, out = x + layer(LN(x)), with the
+    norm and the residual fused into the layer's kernels. ``out`` may be ``x``."""
+    if out is None:
+        out = torch.empty_like(x)
+    _prep(x, dict(x=x, gamma=gamma, beta=beta, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table,
+                  out=out), torch.bfloat16)
+    B, T, H, W, C = x.shape
+    _check(lib().vswin_block_msa_forward(
+        _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(gamma), _ptr(beta), float(eps),
+        _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out), _stream_handle(stream)))
+    return out
 
 
 def wmsa_forward_noalloc(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):

@@ -84,6 +84,48 @@ def test_bf16_unsupported_shapes(L, kw):
     assert vswin.launch_count() == before
 
 
+def _call_block(L, gamma=A16 * 7, beta=A16 * 8, eps=1e-5, **kw):
+    # the block entry takes the layer's arguments with (gamma, beta, eps) after the shift
+    captured = {}
+
+    def fn(*args):
+        captured["args"] = args
+        return 0
+
+    _call(fn, **kw)
+    a = list(captured["args"])
+    p = lambda v: ctypes.c_void_p(v) if v else None  # noqa: E731
+    a[9:9] = [p(gamma), p(beta), ctypes.c_float(eps)]
+    return L.vswin_block_msa_forward(*a)
+
+
+@pytest.mark.parametrize(
+    "kw",
+    [
+        dict(B=0), dict(C=96, heads=5), dict(shift=(8, 3, 3)), dict(window=None),
+        dict(x=0), dict(out=0), dict(Wqkv=0), dict(table=0), dict(gamma=0), dict(beta=0),
+        dict(gamma=A16 * 7 + 1),                  # misaligned
+        dict(eps=-1e-5), dict(eps=float("nan")), dict(eps=float("inf")),
+        dict(out=A16 + 64),                       # overlaps x without being x
+    ],
+)
+def test_block_invalid_arguments_launch_nothing(L, kw):
+    before = vswin.launch_count()
+    rc = _call_block(L, **kw)
+    assert rc == vswin.ERR_INVALID_ARG, (rc, vswin.last_error())
+    assert vswin.last_error()
+    assert vswin.launch_count() == before
+
+
+@pytest.mark.parametrize("kw", [dict(C=128, heads=2), dict(window=(3, 7, 7), shift=(1, 3, 3))])
+def test_block_unsupported_shapes(L, kw):
+    # in place (out == x) passes the pointer checks; the shape is then refused
+    before = vswin.launch_count()
+    rc = _call_block(L, out=A16, **kw)
+    assert rc == vswin.ERR_UNSUPPORTED, (rc, vswin.last_error())
+    assert vswin.launch_count() == before
+
+
 def test_index_maps_rejects_bad_window(L):
     w = (ctypes.c_int * 3)(8, 7, 7)
     s = (ctypes.c_int * 3)(8, 0, 0)
