@@ -407,60 +407,101 @@ __global__ void __launch_bounds__(kFoldCols * kFoldRows) ln_fold_kernel(
 // Row table plus the norm's statistics of each chunk row's token: rowsrc[r] as
 // row_source_kernel writes it and stats[r] = (-mean * rstd, rstd) with the
 // biased variance and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
-// definition), (0, 0) for a padding row. Four lanes per row (the first one
-// does the row's index math), each summing C/32 chunks of 8 channels; two
-// passes (mean, then squared deviations, the second re-reading the row from
-// L1). C is a multiple of 32.
-__global__ void row_stats_kernel(Geom g, long long win0, long long rows, const __nv_bfloat16* __restrict__ x,
-                                 float eps, int* __restrict__ rowsrc, float2* __restrict__ stats) {
-  const long long nthr = (long long)gridDim.x * blockDim.x;
-  const int lane = threadIdx.x & 31;
-  const int cq = lane & 3;
-  const long long base0 = (long long)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  // whole warps iterate together (same trip count), so the shuffles see all lanes
-  for (long long base = base0; base < rows * 4; base += nthr) {
-    const long long i = base + lane;
-    const bool valid = i < rows * 4;
-    const long long r = i >> 2;
-    long long tok = -1;
-    if (valid && cq == 0) {
-      const long long gr = win0 * g.N + r;
-      tok = slot_source(g, gr / g.N, (int)(gr % g.N));
+// definition), (0, 0) for a padding row. A warp takes 32 consecutive rows: each
+// lane does one row's index math (32-bit: window slots < 2^31, checked by the
+// caller), then four lanes per row (rows shuffled to them eight at a time) sum
+// C/32 chunks of 8 channels each. NCH = C/32 in 1..4 keeps all four row groups'
+// chunks in registers (mean, then squared deviations, from the same values);
+// NCH = 0 takes any C, reading each row twice (the second time from L1).
+template <int NCH>
+__global__ void __launch_bounds__(256) row_stats_kernel(Geom g, long long win0, long long rows,
+                                                        const __nv_bfloat16* __restrict__ x, float eps,
+                                                        int* __restrict__ rowsrc, float2* __restrict__ stats) {
+  const int lane = threadIdx.x & 31, cq = lane & 3, sub = lane >> 2;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  const long long warp0 = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nch = g.C / 32;
+  const float inv_c = 1.0f / (float)g.C;
+  auto chunk_sum = [](const uint4& v, float acc) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(h[k]);
+      acc += f.x + f.y;
     }
-    tok = __shfl_sync(0xffffffffu, tok, lane & ~3);  // the row's index math once, on its first lane
-    const __nv_bfloat16* row = x + (tok < 0 ? 0 : tok * g.C);
-    float sum = 0.f;
-    if (tok >= 0)
-      for (int kc = cq; kc < g.C / 8; kc += 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 8);
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    return acc;
+  };
+  auto chunk_sq = [](const uint4& v, float mean, float acc) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(h[k]);
-          sum += f.x + f.y;
-        }
-      }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    const float mean = sum / (float)g.C;
-    float ss = 0.f;
-    if (tok >= 0)
-      for (int kc = cq; kc < g.C / 8; kc += 4) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 8);
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(h[k]);
-          const float d0 = f.x - mean, d1 = f.y - mean;
-          ss = fmaf(d0, d0, fmaf(d1, d1, ss));
-        }
-      }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    if (valid && cq == 0) {
-      rowsrc[r] = (int)tok;
-      const float rstd = 1.0f / sqrtf(ss / (float)g.C + eps);
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(h[k]);
+      const float d0 = f.x - mean, d1 = f.y - mean;
+      acc = fmaf(d0, d0, fmaf(d1, d1, acc));
+    }
+    return acc;
+  };
+  auto finish = [&](long long r, int tok, float sum, float ss) {
+    // sum and ss are the row's totals (after the four-lane reduction)
+    if (cq == 0 && r < rows) {
+      const float mean = sum * inv_c;
+      const float rstd = 1.0f / sqrtf(ss * inv_c + eps);
       stats[r] = tok < 0 ? make_float2(0.f, 0.f) : make_float2(-mean * rstd, rstd);
+    }
+  };
+  // whole warps iterate together (same trip count), so the shuffles see all lanes
+  for (long long R = warp0 * 32; R < rows; R += nwarps * 32) {
+    int my_tok = -1;
+    if (R + lane < rows) {
+      const int gr = (int)(win0 * g.N + R + lane);
+      const int gw = gr / g.N;
+      my_tok = slot_source32(g, gw, gr - gw * g.N);
+      rowsrc[R + lane] = my_tok;
+    }
+    if (NCH > 0) {
+      uint4 v[4][NCH > 0 ? NCH : 1];
+      int tk[4];
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        tk[s] = __shfl_sync(0xffffffffu, my_tok, s * 8 + sub);
+        const __nv_bfloat16* row = x + (size_t)(tk[s] < 0 ? 0 : tk[s]) * g.C;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i)
+          v[s][i] = tk[s] >= 0 ? *reinterpret_cast<const uint4*>(row + (cq + 4 * i) * 8) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) sum = chunk_sum(v[s][i], sum);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        const float mean = sum * inv_c;
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) ss = chunk_sq(v[s][i], mean, ss);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        finish(R + s * 8 + sub, tk[s], sum, ss);
+      }
+    } else {
+      for (int s = 0; s < 4; ++s) {
+        const int tok = __shfl_sync(0xffffffffu, my_tok, s * 8 + sub);
+        const __nv_bfloat16* row = x + (size_t)(tok < 0 ? 0 : tok) * g.C;
+        float sum = 0.f;
+        if (tok >= 0)
+          for (int i = 0; i < nch; ++i) sum = chunk_sum(*reinterpret_cast<const uint4*>(row + (cq + 4 * i) * 8), sum);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        const float mean = sum * inv_c;
+        float ss = 0.f;
+        if (tok >= 0)
+          for (int i = 0; i < nch; ++i)
+            ss = chunk_sq(*reinterpret_cast<const uint4*>(row + (cq + 4 * i) * 8), mean, ss);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        finish(R + s * 8 + sub, tok, sum, ss);
+      }
     }
   }
 }
@@ -653,6 +694,22 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       return (MODE == kPROJ && m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
     };
     int dr_next = out_row(m_first);
+    // columns handled per TMEM wait (the residual's registers and the norm's
+    // extra terms need room)
+    constexpr int kCh = kResid ? 48 : kLn ? 72 : 96;
+    // kResid: the residual of this warp's first column chunk, loaded one tile
+    // ahead (the next tile's output row is known a tile early)
+    uint4 xr[kResid ? kCh / 8 : 1];
+    auto load_resid = [&](const __nv_bfloat16* xrow, int c0) {
+      const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;
+#pragma unroll
+      for (int j = 0; j < kCh / 8; ++j)
+        xr[j] = (xrow && j * 8 < n) ? *reinterpret_cast<const uint4*>(xrow + c0 + 8 * j) : make_uint4(0, 0, 0, 0);
+    };
+    auto resid_row = [&](int dr) -> const __nv_bfloat16* {
+      return dr >= 0 ? a.resid + (long long)dr * g.C + n0 : nullptr;
+    };
+    if (kResid) load_resid(resid_row(dr_next), hf * cw);
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += m_step, ++t) {
       const int buf = (int)(t & 1);
@@ -684,18 +741,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
           }
         }
       }
-      // columns handled per TMEM wait (the residual's registers and the norm's
-      // extra terms need room)
-      constexpr int kCh = kResid ? 48 : kLn ? 72 : 96;
-      uint4 xr[kResid ? kCh / 8 : 1];
-      auto load_resid = [&](int c0) {
-        const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;
-#pragma unroll
-        for (int j = 0; j < kCh / 8; ++j)
-          xr[j] = (xres && j * 8 < n) ? *reinterpret_cast<const uint4*>(xres + c0 + 8 * j) : make_uint4(0, 0, 0, 0);
-      };
-      // the first column chunk's residual is in flight while the accumulator is awaited
-      if (kResid) load_resid(hf * cw);
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 70);
       if (!s_abort && !mbar_wait(&acc_full[buf], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 71);
@@ -705,7 +750,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
         for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += kCh) {
           const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;  // a multiple of 8
           uint32_t u[kCh];
-          if (kResid && c0 != hf * cw) load_resid(c0);
+          if (kResid && c0 != hf * cw) load_resid(xres, c0);
           const uint32_t ta = tmem + lane_base + buf * BN + c0;
 #pragma unroll
           for (int j = 0; j < kCh / 8; ++j)
@@ -770,6 +815,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       __syncwarp();
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 72);
       if (lane == 0) mbar_arrive(&acc_free[buf]);
+      if (kResid) load_resid(resid_row(dr_next), hf * cw);  // next tile's first chunk
     }
   }
   tc_fence_before();
@@ -1863,7 +1909,11 @@ int pick_bn(int n) {
 
 template <int MODE, bool FUSE>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
-  if (a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0) {
+  // persistent version when its weight slice and two A stages fit in shared
+  // memory (227 KB per CTA); otherwise the tiled version (e.g. C = 544: BN = 32
+  // for the projection, two 139 KB A stages)
+  if (a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0 &&
+      ws_smem_bytes(a.K, a.BN, 2, FUSE && MODE == kQKV) <= 227 * 1024) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1948,10 +1998,17 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
     const long long rows = nwin * g.N;
     prof_begin(kKindOther, st);
     if (fuse) {
-      long long blocks = (rows * 4 + 255) / 256;
+      // one warp per 32 rows, eight warps per block
+      long long blocks = (rows + 255) / 256;
       if (blocks > 4096) blocks = 4096;
-      row_stats_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, static_cast<const __nv_bfloat16*>(x),
-                                                          fuse->eps, rowsrc, stats);
+      const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+      switch (g.C / 32) {
+        case 1: row_stats_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
+        case 2: row_stats_kernel<2><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
+        case 3: row_stats_kernel<3><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
+        case 4: row_stats_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
+        default: row_stats_kernel<0><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats);
+      }
     } else {
       long long blocks = (rows + 255) / 256;
       if (blocks > 2048) blocks = 2048;

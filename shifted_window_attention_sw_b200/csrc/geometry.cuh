@@ -66,6 +66,24 @@ __host__ __device__ inline long long slot_source(const Geom& g, long long win, i
   return (((long long)b * g.T + o[0]) * g.H + o[1]) * g.W + o[2];
 }
 
+// slot_source in 32-bit arithmetic, for layers whose window slots (and hence
+// tokens) number below 2^31: window `gw` = b * nW + w, slot n.
+__host__ __device__ inline int slot_source32(const Geom& g, int gw, int n) {
+  const int b = gw / g.nW;
+  const int w = gw - b * g.nW;
+  int wp[3], p[3];
+  window_position(g, w, wp);
+  slot_position(g, n, p);
+  int o[3];
+  for (int a = 0; a < 3; ++a) {
+    int r = wp[a] * g.win[a] + p[a] + g.sh[a];
+    if (r >= g.Lp[a]) r -= g.Lp[a];
+    if (r >= g.L[a]) return -1;
+    o[a] = r;
+  }
+  return ((b * g.T + o[0]) * g.H + o[1]) * g.W + o[2];
+}
+
 __host__ __device__ inline int axis_region(int r, int Lp, int w, int s) {
   if (s == 0 || r < Lp - w) return 0;
   return r < Lp - s ? 1 : 2;

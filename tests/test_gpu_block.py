@@ -66,6 +66,7 @@ BLOCK_CASES = [
     ((1, 8, 14, 14, 96), 3, (8, 7, 7), (0, 0, 0)),
     ((1, 12, 12, 12, 128), 4, (8, 7, 7), (4, 3, 3)),    # pads T, H, W
     ((1, 8, 14, 14, 384), 12, (8, 7, 7), (4, 3, 3)),    # Swin-T stage-3 width: tiled GEMMs
+    ((1, 8, 7, 14, 544), 17, (8, 7, 7), (4, 0, 3)),     # 17 heads: statistics for any C/32
     ((2, 1, 14, 21, 64), 2, (1, 7, 7), (0, 3, 3)),      # 2D Swin special case
     ((1, 5, 9, 10, 64), 2, (4, 4, 4), (2, 1, 3)),       # padding on every axis, generic attention kernel
 ]

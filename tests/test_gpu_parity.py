@@ -136,6 +136,7 @@ BF16_CASES = [
     ((1, 16, 14, 21, 64), 2, (8, 7, 7), (4, 3, 0)),
     ((1, 8, 14, 14, 384), 12, (8, 7, 7), (4, 3, 3)),    # Swin-T stage-3 width
     ((1, 8, 7, 7, 1024), 32, (8, 7, 7), (4, 0, 0)),     # Swin-B stage-4 width (K = 1024)
+    ((1, 8, 7, 14, 544), 17, (8, 7, 7), (4, 0, 3)),     # 17 heads: projection BN = 32, tiled GEMMs
     ((2, 1, 14, 21, 64), 2, (1, 7, 7), (0, 3, 3)),      # 2D Swin special case
     ((1, 8, 14, 14, 64), 2, (4, 7, 7), (2, 3, 3)),      # temporal window 4
     ((2, 6, 14, 21, 64), 2, (2, 7, 7), (1, 3, 3)),      # temporal window 2 (one query tile per window)
