@@ -14,6 +14,10 @@ Two independent formulations live here:
 * ``group_rule.forward`` -- a NumPy float64 brute force over all token pairs of
   the padded grid with no roll and no partition (see that module).
 
+Gradients of the layer (``oracle.backward``, NumPy float64) follow the same
+steps per window and the chain rule back through them; they are pinned by
+central finite differences of ``forward``.
+
 The attention half of a block (``block_forward``) is written on top of
 ``forward`` in NumPy float64: layer norm of each token over its C channels,
 the layer, and the residual add ("Video Swin Transformer" summary page, Method
