@@ -494,6 +494,82 @@ def run_block(args):
     return 0
 
 
+def run_backward(args):
+    """``--backward``: the fp32 backward (vswin_wmsa_backward_f32: forward recompute plus
+    every gradient) of each layer of the workload, on fp32 inputs of the same shapes. One
+    GPU; prints its own JSON line. The path is plain FP32 arithmetic, so the roofline is
+    the FP32 ALU peak: 148 SMs x 128 FP32 lanes x 2 FLOP x 1.965 GHz = 74.4 TFLOP/s."""
+    from shifted_window_attention_sw_b200 import build as build_mod
+    from shifted_window_attention_sw_b200 import vswin
+    from shifted_window_attention_sw_b200.inputs import make_layer_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    build_mod.build()
+    vswin.lib()
+    wl = WORKLOADS[args.workload]
+    layers = wl.layers
+    base = 1000 * wl.index
+    ins = [make_layer_inputs(ly.shape, ly.heads, ly.window, "f32", "baseline", seed=base + ly.seed_offset,
+                             x_seed=base).to(device) for ly in layers]
+    dys = [torch.randn(*ly.shape, generator=torch.Generator().manual_seed(base + 77 + k)).to(device)
+           for k, ly in enumerate(layers)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for ly, i, dy in zip(layers, ins, dys):
+            vswin.wmsa_backward_f32(i.x, ly.window, ly.shift, i.Wqkv, i.bqkv, i.Wproj, i.bproj, i.table, ly.heads,
+                                    dy, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = vswin.launch_count()
+    sampler = ClockSampler(device)
+    sampler.start()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if vswin.poll_error(stream) != vswin.OK:
+        raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    # FLOPs of the kernels as built, per layer (rows = window slots):
+    # forward recompute 2 rows C 3C + 4 windows N^2 C + 2 rows C^2; dO 2 rows C^2;
+    # row pass 6 N^2 C per window; column pass 8 N^2 C; dx 2 rows 3C C; dWqkv 2 rows C 3C;
+    # dWproj 2 rows C^2
+    flops = 0
+    for ly in layers:
+        g = layer_work(ly.B, ly.T, ly.H, ly.W, ly.C, ly.heads, ly.window, ly.shift, 4)
+        win, N = g["windows"], g["N"]
+        rows = win * N
+        C = ly.C
+        flops += 2 * rows * C * 3 * C * 3 + 2 * rows * C * C * 3 + (4 + 6 + 8) * win * N * N * C
+    tokens = step_work(wl)["tokens"]
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    line = {
+        "metric": "fp32 layer backward tokens/s (forward recompute + all gradients), " + wl.name,
+        "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(wl),
+        "api": "vswin_wmsa_backward_f32",
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                     "flops_per_step": flops},
+        "gpu_launches": int(vswin.launch_count() - launches0),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -506,6 +582,8 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-s", type=float, default=20.0)
     ap.add_argument("--block", action="store_true",
                     help="time the blocks' attention half (LN, layer, residual), fused and unfused, on one GPU")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the fp32 backward of each layer of the workload on one GPU")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -513,6 +591,8 @@ def main(argv=None):
         return run_reference(args)
     if args.block:
         return run_block(args)
+    if args.backward:
+        return run_backward(args)
     return run_gpu(args)
 
 

@@ -121,6 +121,30 @@ int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int
                            const void* bias_table, void* out, void* stream);
 
 /*
+ * fp32 backward of the layer (plain FP32 FMA arithmetic, no tensor cores):
+ * for the output gradient dy (same layout as out), writes dx (layout of x),
+ * dWqkv [C][3C], dbqkv [3C], dWproj [C][C], dbproj [C] and dtable (layout of
+ * bias_table) -- the chain rule back through the layer's steps above
+ * ("Video Swin Transformer" summary page, Method steps 4-6 and eq. 2; the
+ * softmax gradient dS = P * (dP - rowsum(dP * P)), zero on masked pairs;
+ * padded slots are keys with zero input, so they reach dbqkv but not dx; the
+ * table gradient of head h sums dS over every pair that reads that row).
+ * Every tensor is float, 4-byte aligned, on the device; the six gradient
+ * buffers are overwritten (not accumulated) and may overlap neither one
+ * another nor any input. The forward is recomputed inside the call. Any head
+ * width; N <= 4096 and (2N + 2d) * 4 bytes and 12C bytes within 48 KB,
+ * otherwise VSWIN_ERR_UNSUPPORTED. Results are not bitwise deterministic
+ * (the table and weight gradients are summed with atomics). Scratch: from
+ * the library's pool, about (13C + 3 heads) * 4 bytes per window slot plus
+ * the forward's output.
+ */
+int vswin_wmsa_backward_f32(const void* x, int B, int T, int H, int W, int C, int heads,
+                            const int* window, const int* shift,
+                            const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                            const void* bias_table, const void* dy, void* dx, void* dWqkv, void* dbqkv,
+                            void* dWproj, void* dbproj, void* dtable, void* stream);
+
+/*
  * bf16 layer forward with the activations in HOST memory: copies x_host to
  * the device, runs vswin_wmsa_forward, copies the result to out_host and
  * synchronises `stream`. Weights, biases and table are device pointers (they

@@ -34,6 +34,14 @@ cudaError_t launch_f32_forward(const Geom& g, const float* x, const float* Wqkv,
                                float* scratch_qkv, float* scratch_o, cudaStream_t st);
 size_t f32_scratch_floats(const Geom& g, size_t* qkv_floats, size_t* o_floats);
 
+// fp32 backward (backward_f32.cu): gradients of x, Wqkv, bqkv, Wproj, bproj and
+// the table for output gradient dy; scratch of f32_backward_scratch_bytes.
+size_t f32_backward_scratch_bytes(const Geom& g);
+cudaError_t launch_f32_backward(const Geom& g, const float* x, const float* Wqkv, const float* bqkv,
+                                const float* Wproj, const float* bproj, const float* table, const float* dy,
+                                float* dx, float* dWqkv, float* dbqkv, float* dWproj, float* dbproj, float* dtable,
+                                void* scratch, cudaStream_t st);
+
 cudaError_t launch_index_maps(const Geom& g, int* win_src, int* region, int* bias_idx, cudaStream_t st);
 
 cudaError_t launch_selftest_timeout(const KernelCtx& ctx, cudaStream_t st);

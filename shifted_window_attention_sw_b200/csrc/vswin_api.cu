@@ -443,6 +443,55 @@ int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int
   return VSWIN_OK;
 }
 
+int vswin_wmsa_backward_f32(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                            const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
+                            const void* bproj, const void* bias_table, const void* dy, void* dx, void* dWqkv,
+                            void* dbqkv, void* dWproj, void* dbproj, void* dtable, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  const void* ptrs[] = {x, Wqkv, bqkv, Wproj, bproj, bias_table, dy, dx, dWqkv, dbqkv, dWproj, dbproj, dtable};
+  const char* names[] = {"x", "Wqkv", "bqkv", "Wproj", "bproj", "bias_table", "dy",
+                         "dx", "dWqkv", "dbqkv", "dWproj", "dbproj", "dtable"};
+  for (int k = 0; k < 13; ++k) {
+    if (!ptrs[k]) return fail(VSWIN_ERR_INVALID_ARG, "%s is NULL", names[k]);
+    if (!aligned(ptrs[k], 4)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not 4-byte aligned", names[k]);
+  }
+  const size_t act = (size_t)g.tokens * g.C * 4;
+  const size_t wq = (size_t)g.C * 3 * g.C * 4, wp = (size_t)g.C * g.C * 4;
+  const size_t tb = (size_t)g.table_rows * g.heads * 4;
+  // every output against every input it could alias
+  const void* outs[] = {dx, dWqkv, dbqkv, dWproj, dbproj, dtable};
+  const size_t out_n[] = {act, wq, (size_t)3 * g.C * 4, wp, (size_t)g.C * 4, tb};
+  const void* ins[] = {x, dy, Wqkv, bqkv, Wproj, bproj, bias_table};
+  const size_t in_n[] = {act, act, wq, (size_t)3 * g.C * 4, wp, (size_t)g.C * 4, tb};
+  for (int a = 0; a < 6; ++a) {
+    for (int b = 0; b < 7; ++b)
+      if (overlap(outs[a], out_n[a], ins[b], in_n[b]))
+        return fail(VSWIN_ERR_INVALID_ARG, "gradient buffer %s overlaps an input", names[7 + a]);
+    for (int b = a + 1; b < 6; ++b)
+      if (overlap(outs[a], out_n[a], outs[b], out_n[b]))
+        return fail(VSWIN_ERR_INVALID_ARG, "gradient buffers %s and %s overlap", names[7 + a], names[7 + b]);
+  }
+  if (g.N > 4096) return fail(VSWIN_ERR_UNSUPPORTED, "fp32 backward supports N <= 4096 (N = %d)", g.N);
+  if ((2 * (size_t)g.N + 2 * g.d) * 4 > 48 * 1024 || (size_t)3 * g.C * 4 > 48 * 1024)
+    return fail(VSWIN_ERR_UNSUPPORTED, "fp32 backward: window or width too large for its shared-memory rows");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  st = scratch_alloc(&scratch, f32_backward_scratch_bytes(g), s);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = launch_f32_backward(
+      g, static_cast<const float*>(x), static_cast<const float*>(Wqkv), static_cast<const float*>(bqkv),
+      static_cast<const float*>(Wproj), static_cast<const float*>(bproj), static_cast<const float*>(bias_table),
+      static_cast<const float*>(dy), static_cast<float*>(dx), static_cast<float*>(dWqkv),
+      static_cast<float*>(dbqkv), static_cast<float*>(dWproj), static_cast<float*>(dbproj),
+      static_cast<float*>(dtable), scratch, s);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) return fail_cuda(e, "fp32 backward launch");
+  if (e2 != cudaSuccess) return fail_cuda(e2, "cudaFreeAsync");
+  return VSWIN_OK;
+}
+
 int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads, const int* window,
                             const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                             const void* bproj, const void* bias_table, void* out_host, void* stream) {

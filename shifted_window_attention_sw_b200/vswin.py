@@ -35,6 +35,7 @@ EXPORTS = (
     "vswin_wmsa_forward_noalloc",
     "vswin_set_exact_softmax",
     "vswin_block_msa_forward",
+    "vswin_wmsa_backward_f32",
 )
 
 KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other")
@@ -68,6 +69,8 @@ def lib():
             fn.restype = _I
         L.vswin_block_msa_forward.argtypes = layer[:9] + [_P, _P, ctypes.c_float] + layer[9:]
         L.vswin_block_msa_forward.restype = _I
+        L.vswin_wmsa_backward_f32.argtypes = layer[:15] + [_P] * 6 + [_P]  # ..., dy, six gradients, stream
+        L.vswin_wmsa_backward_f32.restype = _I
         L.vswin_wmsa_index_maps.argtypes = [_I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P]
         L.vswin_wmsa_index_maps.restype = _I
         L.vswin_clamp_window.argtypes = [_I, _I, _I, _IP, _IP, _IP, _IP]
@@ -157,6 +160,20 @@ def block_msa_forward(x, window, shift, gamma, beta, eps, Wqkv, bqkv, Wproj, bpr
         _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(gamma), _ptr(beta), float(eps),
         _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out), _stream_handle(stream)))
     return out
+
+
+def wmsa_backward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, dy, stream=None):
+    """fp32 gradients (dx, dWqkv, dbqkv, dWproj, dbproj, dtable) of the layer for output
+    gradient ``dy``. All tensors float32 on one CUDA device."""
+    outs = [torch.empty_like(t) for t in (x, Wqkv, bqkv, Wproj, bproj, table)]
+    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, dy=dy), torch.float32)
+    if dy.shape != x.shape:
+        raise ValueError("dy must have the shape of x")
+    B, T, H, W, C = x.shape
+    _check(lib().vswin_wmsa_backward_f32(
+        _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj),
+        _ptr(bproj), _ptr(table), _ptr(dy), *[_ptr(o) for o in outs], _stream_handle(stream)))
+    return tuple(outs)
 
 
 def wmsa_forward_noalloc(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):

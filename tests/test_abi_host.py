@@ -145,3 +145,31 @@ def test_index_maps_rejects_bad_window(L):
 def test_clamp_window(L, dims, window, shift, ew, es):
     w, s = vswin.clamp_window(*dims, window, shift)
     assert w == ew and s == es
+
+
+def _call_backward(L, dx=A16 * 9, dy=A16 * 10, **kw):
+    # the backward entry takes the layer's arguments (without out) then dy and six gradients
+    captured = {}
+
+    def fn(*args):
+        captured["args"] = args
+        return 0
+
+    _call(fn, **kw)
+    a = list(captured["args"])
+    p = lambda v: ctypes.c_void_p(v) if v else None  # noqa: E731
+    grads = [p(dx), p(A16 * 11), p(A16 * 12), p(A16 * 13), p(A16 * 14), p(A16 * 15)]
+    return L.vswin_wmsa_backward_f32(*(a[:14] + [p(dy)] + grads + [a[15]]))
+
+
+@pytest.mark.parametrize(
+    "kw",
+    [dict(B=0), dict(window=None), dict(x=0), dict(dy=0), dict(dx=0), dict(Wqkv=0),
+     dict(dx=A16 * 9 + 2),       # misaligned
+     dict(dx=A16 + 64)],         # overlaps x
+)
+def test_backward_invalid_arguments_launch_nothing(L, kw):
+    before = vswin.launch_count()
+    rc = _call_backward(L, **kw)
+    assert rc == vswin.ERR_INVALID_ARG, (rc, vswin.last_error())
+    assert vswin.launch_count() == before
