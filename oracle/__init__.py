@@ -245,3 +245,33 @@ def block_forward_windows(x, gamma, beta, eps, window, shift, Wqkv, bqkv, Wproj,
         m = s >= 0
         o[k][m] += flat[s[m]]
     return o
+
+
+def gelu(x):
+    """x * Phi(x), Phi the standard normal CDF (the erf form of torch.nn.GELU)."""
+    from scipy.special import erf
+
+    x = _f64(x)
+    return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+def mlp_half(z, gamma, beta, eps, W1, b1, W2, b2):
+    """Second half of a block in float64: z + GELU(LN(z) W1 + b1) W2 + b2.
+
+    "Video Swin Transformer" summary page, Method step 3 and eq. 1 (layer norm,
+    a two-layer MLP with GELU, residual add). W1 [C][hidden], W2 [hidden][C];
+    the pages do not give the hidden width (Swin's models use 4C).
+    """
+    z = _f64(z)
+    W1, b1, W2, b2 = map(_f64, (W1, b1, W2, b2))
+    y = layer_norm(z, gamma, beta, eps)
+    return z + gelu(y @ W1 + b1) @ W2 + b2
+
+
+def block_full_forward(x, attn, mlp, window, shift, heads, eps=LN_EPS):
+    """One whole Video Swin block in float64 (eq. 1): the attention half
+    (``block_forward``) then ``mlp_half``. ``attn`` = dict(gamma, beta, Wqkv, bqkv,
+    Wproj, bproj, table); ``mlp`` = dict(gamma, beta, W1, b1, W2, b2)."""
+    z = block_forward(x, attn["gamma"], attn["beta"], eps, window, shift, attn["Wqkv"], attn["bqkv"],
+                      attn["Wproj"], attn["bproj"], attn["table"], heads)
+    return mlp_half(z, mlp["gamma"], mlp["beta"], eps, mlp["W1"], mlp["b1"], mlp["W2"], mlp["b2"])

@@ -361,3 +361,70 @@ def test_b5_padding_is_zero_after_the_norm(oracle_mod):
                               heads)
     out = _run_block(oracle_mod, a, window, shift, heads)
     np.testing.assert_allclose(out, a["x"] + full[:, :3, :5, :6], rtol=0, atol=1e-12)
+
+
+# ---- MLP half of the block and the whole block --------------------------------------------------
+def _mlp_params(C, hidden, seed):
+    rng = np.random.default_rng(seed)
+    return dict(gamma=1 + 0.1 * rng.normal(size=C), beta=0.1 * rng.normal(size=C),
+                W1=rng.normal(size=(C, hidden)) / np.sqrt(C), b1=0.1 * rng.normal(size=hidden),
+                W2=rng.normal(size=(hidden, C)) / np.sqrt(hidden), b2=0.1 * rng.normal(size=C))
+
+
+def test_m1_gelu(oracle_mod):
+    # against torch's exact GELU in float64, and the identity GELU(x) - GELU(-x) = x
+    x = np.linspace(-6, 6, 241)
+    ref = torch.nn.functional.gelu(torch.from_numpy(x)).numpy()
+    np.testing.assert_allclose(oracle_mod.gelu(x), ref, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(oracle_mod.gelu(x) - oracle_mod.gelu(-x), x, rtol=0, atol=1e-14)
+    assert oracle_mod.gelu(np.array([0.0]))[0] == 0.0
+
+
+def test_m2_zero_second_layer_is_identity(oracle_mod):
+    z = np.random.default_rng(1).normal(size=(2, 3, 4, 5, 16))
+    p = _mlp_params(16, 64, 2)
+    p["W2"] = np.zeros_like(p["W2"])
+    p["b2"] = np.zeros_like(p["b2"])
+    out = oracle_mod.mlp_half(z, p["gamma"], p["beta"], 1e-5, p["W1"], p["b1"], p["W2"], p["b2"])
+    assert np.array_equal(out, z)
+
+
+def test_m3_constant_tokens_closed_form(oracle_mod):
+    # a token with equal channels normalises to beta: the branch is GELU(beta W1 + b1) W2 + b2
+    rng = np.random.default_rng(3)
+    z = np.repeat(rng.normal(size=(1, 2, 3, 4, 1)), 16, axis=-1)
+    p = _mlp_params(16, 64, 4)
+    branch = oracle_mod.gelu(p["beta"] @ p["W1"] + p["b1"]) @ p["W2"] + p["b2"]
+    out = oracle_mod.mlp_half(z, p["gamma"], p["beta"], 1e-5, p["W1"], p["b1"], p["W2"], p["b2"])
+    np.testing.assert_allclose(out, z + branch, rtol=0, atol=1e-12)
+
+
+def test_m4_mlp_matches_torch_modules(oracle_mod):
+    # the MLP half against torch's LayerNorm / Linear / GELU / Linear in float64
+    z = np.random.default_rng(5).normal(size=(1, 2, 3, 4, 16)) * 2 + 0.5
+    p = _mlp_params(16, 64, 6)
+    t = torch.from_numpy
+    y = torch.nn.functional.layer_norm(t(z), (16,), t(p["gamma"]), t(p["beta"]), 1e-5)
+    h = torch.nn.functional.gelu(y @ t(p["W1"]) + t(p["b1"]))
+    ref = (t(z) + h @ t(p["W2"]) + t(p["b2"])).numpy()
+    out = oracle_mod.mlp_half(z, p["gamma"], p["beta"], 1e-5, p["W1"], p["b1"], p["W2"], p["b2"])
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_m5_whole_block_is_the_two_halves(oracle_mod):
+    # eq. 1: z_hat = x + attention(LN(x)), z = z_hat + MLP(LN(z_hat)); checked through the
+    # zero-projection special cases: with both branches' last weights and biases zero the
+    # block is the identity, with only the MLP's zero it is the attention half
+    shape, heads, window, shift = (1, 4, 6, 6, 16), 2, (2, 3, 3), (1, 1, 1)
+    a = _block_inputs(shape, heads, window)
+    attn = {k: a[k] for k in ("gamma", "beta", "Wqkv", "bqkv", "Wproj", "bproj", "table")}
+    mlp = _mlp_params(16, 64, 7)
+    mlp0 = dict(mlp, W2=np.zeros_like(mlp["W2"]), b2=np.zeros_like(mlp["b2"]))
+    half = _run_block(oracle_mod, a, window, shift, heads)
+    np.testing.assert_allclose(oracle_mod.block_full_forward(a["x"], attn, mlp0, window, shift, heads), half,
+                               rtol=0, atol=0)
+    attn0 = dict(attn, Wproj=np.zeros_like(attn["Wproj"]), bproj=np.zeros_like(attn["bproj"]))
+    assert np.array_equal(oracle_mod.block_full_forward(a["x"], attn0, mlp0, window, shift, heads), a["x"])
+    full = oracle_mod.block_full_forward(a["x"], attn, mlp, window, shift, heads)
+    np.testing.assert_allclose(full, oracle_mod.mlp_half(half, mlp["gamma"], mlp["beta"], 1e-5, mlp["W1"],
+                                                         mlp["b1"], mlp["W2"], mlp["b2"]), rtol=0, atol=0)
