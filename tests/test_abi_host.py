@@ -173,3 +173,26 @@ def test_backward_invalid_arguments_launch_nothing(L, kw):
     rc = _call_backward(L, **kw)
     assert rc == vswin.ERR_INVALID_ARG, (rc, vswin.last_error())
     assert vswin.launch_count() == before
+
+
+def test_binding_rejects_wrong_dtype_and_layout(L):
+    # the Python binding checks dtypes, contiguity and shapes before calling the library
+    import torch
+
+    x = torch.zeros(1, 8, 14, 14, 96, dtype=torch.bfloat16)
+    W = torch.zeros(96, 288, dtype=torch.bfloat16)
+    b = torch.zeros(288, dtype=torch.bfloat16)
+    Wp = torch.zeros(96, 96, dtype=torch.bfloat16)
+    bp = torch.zeros(96, dtype=torch.bfloat16)
+    t = torch.zeros(2535, 3, dtype=torch.bfloat16)
+    before = vswin.launch_count()
+    with pytest.raises(TypeError):
+        vswin.wmsa_forward(x.float(), (8, 7, 7), (4, 3, 3), W, b, Wp, bp, t, 3)
+    with pytest.raises(ValueError):
+        vswin.wmsa_forward(x, (8, 7, 7), (4, 3, 3), W.t(), b, Wp, bp, t, 3)
+    with pytest.raises(TypeError):
+        vswin.block_msa_forward(x, (8, 7, 7), (4, 3, 3), bp.float(), bp, 1e-5, W, b, Wp, bp, t, 3)
+    f = [a.float() for a in (x, W, b, Wp, bp, t)]
+    with pytest.raises(ValueError):
+        vswin.wmsa_backward_f32(*f[:1], (8, 7, 7), (4, 3, 3), *f[1:], 3, f[0][:, :4])
+    assert vswin.launch_count() == before
