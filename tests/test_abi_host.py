@@ -196,3 +196,20 @@ def test_binding_rejects_wrong_dtype_and_layout(L):
     with pytest.raises(ValueError):
         vswin.wmsa_backward_f32(*f[:1], (8, 7, 7), (4, 3, 3), *f[1:], 3, f[0][:, :4])
     assert vswin.launch_count() == before
+
+
+@pytest.mark.parametrize("name", ["vswin_wmsa_forward", "vswin_wmsa_forward_f32", "vswin_wmsa_forward_noalloc"])
+def test_layers_beyond_the_index_range_are_refused(L, name):
+    # B * windows * N must stay below 2^31 (slot indices are 32-bit in the kernels)
+    before = vswin.launch_count()
+    rc = _call(getattr(L, name), B=1 << 20, T=16, H=56, W=56)
+    assert rc == vswin.ERR_UNSUPPORTED, (rc, vswin.last_error())
+    assert "2^31" in vswin.last_error()
+    assert vswin.launch_count() == before
+
+
+def test_block_and_backward_beyond_the_index_range_are_refused(L):
+    before = vswin.launch_count()
+    assert _call_block(L, B=1 << 20, T=16, H=56, W=56, out=A16) == vswin.ERR_UNSUPPORTED
+    assert _call_backward(L, B=1 << 20, T=16, H=56, W=56) == vswin.ERR_UNSUPPORTED
+    assert vswin.launch_count() == before
