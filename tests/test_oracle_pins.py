@@ -428,3 +428,38 @@ def test_m5_whole_block_is_the_two_halves(oracle_mod):
     full = oracle_mod.block_full_forward(a["x"], attn, mlp, window, shift, heads)
     np.testing.assert_allclose(full, oracle_mod.mlp_half(half, mlp["gamma"], mlp["beta"], 1e-5, mlp["W1"],
                                                          mlp["b1"], mlp["W2"], mlp["b2"]), rtol=0, atol=0)
+
+
+# ---- per-window entry points (used for sampled parity at full size) ----------------------------
+def test_w1_forward_windows_match_the_layer(oracle_mod):
+    # forward_windows returns, per listed window and real slot, the layer's output at the
+    # slot's token (the pinned forward), and some value at padding slots
+    shape, heads, window, shift = (2, 5, 9, 10, 16), 2, (4, 4, 4), (2, 1, 3)
+    a = _inputs(shape, heads, window)
+    full = _run(oracle_mod, a, window, shift, heads).reshape(-1, shape[-1])
+    g = oracle_mod.geometry(*shape[1:4], window, shift)
+    wins = [0, 3, g["nW"] - 1, g["nW"] + 5, 2 * g["nW"] - 1]
+    y = oracle_mod.forward_windows(a["x"], window, shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"], a["table"],
+                                   heads, wins)
+    src, _, _ = oracle_mod.index_maps(shape[0], *shape[1:4], window, shift)
+    N = g["N"]
+    for k, w in enumerate(wins):
+        s = src[w * N:(w + 1) * N]
+        m = s >= 0
+        np.testing.assert_allclose(y[k][m], full[s[m]], rtol=0, atol=1e-12)
+
+
+def test_w2_block_forward_windows_match_the_block(oracle_mod):
+    shape, heads, window, shift = (1, 5, 9, 10, 16), 2, (4, 4, 4), (2, 1, 3)
+    a = _block_inputs(shape, heads, window)
+    full = _run_block(oracle_mod, a, window, shift, heads).reshape(-1, shape[-1])
+    g = oracle_mod.geometry(*shape[1:4], window, shift)
+    wins = [0, 4, g["nW"] - 1]
+    y = oracle_mod.block_forward_windows(a["x"], a["gamma"], a["beta"], 1e-5, window, shift, a["Wqkv"], a["bqkv"],
+                                         a["Wproj"], a["bproj"], a["table"], heads, wins)
+    src, _, _ = oracle_mod.index_maps(1, *shape[1:4], window, shift)
+    N = g["N"]
+    for k, w in enumerate(wins):
+        s = src[w * N:(w + 1) * N]
+        m = s >= 0
+        np.testing.assert_allclose(y[k][m], full[s[m]], rtol=0, atol=1e-12)
