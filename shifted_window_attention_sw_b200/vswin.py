@@ -113,9 +113,11 @@ def _i3(v):
     return (ctypes.c_int * 3)(*v)
 
 
-def _stream_handle(stream):
+def _stream_handle(stream, device=None):
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -123,26 +125,67 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def _layer_call(fn, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out, stream):
+def _layer_call(fn, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out, stream, device=None):
+    # the library launches on the current device, so make the tensors' device current
     B, T, H, W, C = x.shape
-    _check(fn(_ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv),
-              _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out), _stream_handle(stream)))
+    dev = device or x.device
+    with torch.cuda.device(dev):
+        _check(fn(_ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv),
+                  _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out), _stream_handle(stream, dev)))
     return out
 
 
-def _prep(x, tensors, dtype):
+def _prep(x, tensors, dtype, device=None):
+    """dtype and contiguity of every tensor; with ``device``, that every tensor is a
+    CUDA tensor on that device. The library reads raw pointers, so a host tensor or
+    one on another GPU must be refused here."""
     for name, t in tensors.items():
         if t.dtype != dtype:
             raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    if device is not None:
+        for name, t in tensors.items():
+            if not t.is_cuda or t.device != device:
+                raise ValueError(f"{name} must be a CUDA tensor on {device}, got {t.device}")
+
+
+def _table_rows(window):
+    w = tuple(int(a) for a in window)
+    if len(w) != 3:
+        raise ValueError("window and shift need 3 entries")
+    return (2 * w[0] - 1) * (2 * w[1] - 1) * (2 * w[2] - 1)
+
+
+def _check_shapes(x, window, heads, Wqkv=None, bqkv=None, Wproj=None, bproj=None, table=None, **same_as_x):
+    """Shapes the header fixes for a layer on x (B, T, H, W, C): Wqkv [C][3C], bqkv [3C],
+    Wproj [C][C], bproj [C], bias_table [(2P-1)(2Mh-1)(2Mw-1)][heads]; every tensor in
+    ``same_as_x`` has x's shape. The library trusts these sizes, so a short buffer would
+    be read or written past its end."""
+    if x.dim() != 5:
+        raise ValueError(f"x must be (B, T, H, W, C), got shape {tuple(x.shape)}")
+    C = x.shape[-1]
+    want = {"Wqkv": (Wqkv, (C, 3 * C)), "bqkv": (bqkv, (3 * C,)), "Wproj": (Wproj, (C, C)),
+            "bproj": (bproj, (C,)), "bias_table": (table, (_table_rows(window), int(heads)))}
+    for name, (t, shape) in want.items():
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    for name, t in same_as_x.items():
+        if t is not None and t.shape != x.shape:
+            raise ValueError(f"{name} must have the shape of x {tuple(x.shape)}, got {tuple(t.shape)}")
+
+
+def _layer_args(x, window, heads, dtype, Wqkv, bqkv, Wproj, bproj, table, out, **more):
+    tensors = dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out, **more)
+    _prep(x, tensors, dtype, x.device)
+    _check_shapes(x, window, heads, Wqkv, bqkv, Wproj, bproj, table, out=out)
 
 
 def wmsa_forward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):
     """bf16 layer forward on the GPU (tcgen05 path). All tensors bf16 on one CUDA device."""
     if out is None:
         out = torch.empty_like(x)
-    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.bfloat16)
+    _layer_args(x, window, heads, torch.bfloat16, Wqkv, bqkv, Wproj, bproj, table, out)
     return _layer_call(lib().vswin_wmsa_forward, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out,
                        stream)
 
@@ -153,26 +196,31 @@ def block_msa_forward(x, window, shift, gamma, beta, eps, Wqkv, bqkv, Wproj, bpr
     norm and the residual fused into the layer's kernels. ``out`` may be ``x``."""
     if out is None:
         out = torch.empty_like(x)
-    _prep(x, dict(x=x, gamma=gamma, beta=beta, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table,
-                  out=out), torch.bfloat16)
+    _layer_args(x, window, heads, torch.bfloat16, Wqkv, bqkv, Wproj, bproj, table, out, gamma=gamma, beta=beta)
     B, T, H, W, C = x.shape
-    _check(lib().vswin_block_msa_forward(
-        _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(gamma), _ptr(beta), float(eps),
-        _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out), _stream_handle(stream)))
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        if tuple(t.shape) != (C,):
+            raise ValueError(f"{name} must have shape ({C},), got {tuple(t.shape)}")
+    with torch.cuda.device(x.device):
+        _check(lib().vswin_block_msa_forward(
+            _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(gamma), _ptr(beta), float(eps),
+            _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out),
+            _stream_handle(stream, x.device)))
     return out
 
 
 def wmsa_backward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, dy, stream=None):
     """fp32 gradients (dx, dWqkv, dbqkv, dWproj, dbproj, dtable) of the layer for output
     gradient ``dy``. All tensors float32 on one CUDA device."""
+    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, dy=dy), torch.float32,
+          x.device)
+    _check_shapes(x, window, heads, Wqkv, bqkv, Wproj, bproj, table, dy=dy)
     outs = [torch.empty_like(t) for t in (x, Wqkv, bqkv, Wproj, bproj, table)]
-    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, dy=dy), torch.float32)
-    if dy.shape != x.shape:
-        raise ValueError("dy must have the shape of x")
     B, T, H, W, C = x.shape
-    _check(lib().vswin_wmsa_backward_f32(
-        _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj),
-        _ptr(bproj), _ptr(table), _ptr(dy), *[_ptr(o) for o in outs], _stream_handle(stream)))
+    with torch.cuda.device(x.device):
+        _check(lib().vswin_wmsa_backward_f32(
+            _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj),
+            _ptr(bproj), _ptr(table), _ptr(dy), *[_ptr(o) for o in outs], _stream_handle(stream, x.device)))
     return tuple(outs)
 
 
@@ -182,7 +230,7 @@ def wmsa_forward_noalloc(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, head
     passed in by callers that cannot allocate; if it is None a tensor is created."""
     if out is None:
         out = torch.empty_like(x)
-    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.bfloat16)
+    _layer_args(x, window, heads, torch.bfloat16, Wqkv, bqkv, Wproj, bproj, table, out)
     return _layer_call(lib().vswin_wmsa_forward_noalloc, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads,
                        out, stream)
 
@@ -191,7 +239,7 @@ def wmsa_forward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, o
     """fp32 layer forward on the GPU (FP32 FMA path). All tensors float32 on one CUDA device."""
     if out is None:
         out = torch.empty_like(x)
-    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, out=out), torch.float32)
+    _layer_args(x, window, heads, torch.float32, Wqkv, bqkv, Wproj, bproj, table, out)
     return _layer_call(lib().vswin_wmsa_forward_f32, x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads,
                        out, stream)
 
@@ -199,8 +247,14 @@ def wmsa_forward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, o
 def wmsa_forward_host(x_host, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out_host, stream=None):
     """bf16 forward with x and out in host memory (copies inside the call; synchronises)."""
     _prep(x_host, dict(x_host=x_host, out_host=out_host), torch.bfloat16)
+    for name, t in (("x_host", x_host), ("out_host", out_host)):
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+    dev = Wqkv.device
+    _prep(x_host, dict(Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table), torch.bfloat16, dev)
+    _check_shapes(x_host, window, heads, Wqkv, bqkv, Wproj, bproj, table, out_host=out_host)
     return _layer_call(lib().vswin_wmsa_forward_host, x_host, window, shift, Wqkv, bqkv, Wproj, bproj, table,
-                       heads, out_host, stream)
+                       heads, out_host, stream, dev)
 
 
 def index_maps(B, T, H, W, window, shift, device="cuda", stream=None):
@@ -213,8 +267,12 @@ def index_maps(B, T, H, W, window, shift, device="cuda", stream=None):
     win_src = torch.empty(B * nW * N, dtype=torch.int32, device=device)
     region = torch.empty(nW * N, dtype=torch.int32, device=device)
     bias_idx = torch.empty(N * N, dtype=torch.int32, device=device)
-    _check(lib().vswin_wmsa_index_maps(B, T, H, W, _i3(window), _i3(shift), _ptr(win_src), _ptr(region),
-                                       _ptr(bias_idx), _stream_handle(stream)))
+    dev = win_src.device
+    if not win_src.is_cuda:
+        raise ValueError(f"index maps are written on a CUDA device, got {dev}")
+    with torch.cuda.device(dev):
+        _check(lib().vswin_wmsa_index_maps(B, T, H, W, _i3(window), _i3(shift), _ptr(win_src), _ptr(region),
+                                           _ptr(bias_idx), _stream_handle(stream, dev)))
     return win_src, region, bias_idx
 
 

@@ -213,3 +213,81 @@ def test_block_and_backward_beyond_the_index_range_are_refused(L):
     assert _call_block(L, B=1 << 20, T=16, H=56, W=56, out=A16) == vswin.ERR_UNSUPPORTED
     assert _call_backward(L, B=1 << 20, T=16, H=56, W=56) == vswin.ERR_UNSUPPORTED
     assert vswin.launch_count() == before
+
+
+def _layer_tensors(dtype="bf16", C=96, heads=3, window=(8, 7, 7)):
+    import torch
+
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    rows = (2 * window[0] - 1) * (2 * window[1] - 1) * (2 * window[2] - 1)
+    return dict(x=torch.zeros(1, 8, 14, 14, C, dtype=dt), Wqkv=torch.zeros(C, 3 * C, dtype=dt),
+                bqkv=torch.zeros(3 * C, dtype=dt), Wproj=torch.zeros(C, C, dtype=dt), bproj=torch.zeros(C, dtype=dt),
+                table=torch.zeros(rows, heads, dtype=dt))
+
+
+@pytest.mark.parametrize("entry", ["wmsa_forward", "wmsa_forward_noalloc", "wmsa_forward_f32"])
+def test_binding_rejects_host_tensors(L, entry):
+    # The library reads raw device pointers: a CPU tensor must be refused by the binding,
+    # before any call into the library.
+    t = _layer_tensors("f32" if entry.endswith("f32") else "bf16")
+    before = vswin.launch_count()
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        getattr(vswin, entry)(t["x"], (8, 7, 7), (4, 3, 3), t["Wqkv"], t["bqkv"], t["Wproj"], t["bproj"],
+                              t["table"], 3)
+    assert vswin.launch_count() == before
+
+
+def _fake_cuda(t):
+    """A stand-in that passes the dtype / contiguity / device checks on a machine with no
+    GPU (is_cuda and device report cuda:0) while keeping the real shape, so that the shape
+    checks that follow can be exercised on the CPU."""
+    import torch
+
+    class Fake:
+        def __init__(self, real):
+            self.real = real
+            self.shape = real.shape
+            self.dtype = real.dtype
+            self.is_cuda = True
+            self.device = torch.device("cuda", 0)
+
+        def is_contiguous(self):
+            return True
+
+        def dim(self):
+            return self.real.dim()
+
+    return Fake(t)
+
+
+@pytest.mark.parametrize(
+    "name,bad_shape",
+    [("Wqkv", (96, 96)), ("Wqkv", (288, 96)), ("bqkv", (96,)), ("Wproj", (96, 48)), ("bproj", (288,)),
+     ("table", (2535, 2)), ("table", (169, 3)), ("out", (1, 8, 14, 14, 48))],
+)
+def test_binding_rejects_wrong_shapes(L, name, bad_shape):
+    # A short weight, table or output buffer would be read or written past its end by the
+    # kernels: every shape the header fixes is checked before the library is called.
+    import torch
+
+    t = _layer_tensors()
+    t["out"] = torch.zeros_like(t["x"])
+    t[name] = torch.zeros(bad_shape, dtype=torch.bfloat16)
+    f = {k: _fake_cuda(v) for k, v in t.items()}
+    before = vswin.launch_count()
+    with pytest.raises(ValueError, match="shape"):
+        vswin.wmsa_forward(f["x"], (8, 7, 7), (4, 3, 3), f["Wqkv"], f["bqkv"], f["Wproj"], f["bproj"], f["table"],
+                           3, out=f["out"])
+    assert vswin.launch_count() == before
+
+
+def test_binding_rejects_mixed_devices(L):
+    import torch
+
+    t = _layer_tensors()
+    f = {k: _fake_cuda(v) for k, v in t.items()}
+    f["table"].device = torch.device("cuda", 1)
+    out = _fake_cuda(torch.zeros_like(t["x"]))
+    with pytest.raises(ValueError, match="cuda:0"):
+        vswin.wmsa_forward(f["x"], (8, 7, 7), (4, 3, 3), f["Wqkv"], f["bqkv"], f["Wproj"], f["bproj"], f["table"],
+                           3, out=out)
