@@ -607,8 +607,9 @@ int vswin_wmsa_forward_noalloc(const void* x, int B, int T, int H, int W, int C,
   const size_t per_window = bf16_scratch_bytes(g, 1);
   if (per_window > kNoAllocScratchBytes)
     return fail(VSWIN_ERR_UNSUPPORTED,
-                "one window of this layer needs %zu bytes of scratch; the no-allocation entry point has %zu",
-                per_window, kNoAllocScratchBytes);
+                "one window of this layer needs %zu bytes of scratch; the no-allocation entry point has %zu bytes "
+                "(%zu MiB)",
+                per_window, kNoAllocScratchBytes, kNoAllocScratchBytes >> 20);
   KernelCtx ctx;
   st = make_ctx(&ctx);
   if (st != VSWIN_OK) return st;
