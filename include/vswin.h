@@ -112,8 +112,11 @@ int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, in
 
 /*
  * fp32 layer forward (plain FP32 FMA arithmetic, no tensor cores): every
- * tensor is float. Any d; N <= 4096. Pointers 4-byte aligned; x must not
- * overlap out. Scratch: stream-ordered, from the library's pool (see above).
+ * tensor is float. The same layer as vswin_wmsa_forward, steps 1-7 above
+ * ("Video Swin Transformer" summary page, Method steps 4-6 and eq. 2), with
+ * every product and sum in fp32 and the softmax as max, exp, sum, divide.
+ * Any d; N <= 4096. Pointers 4-byte aligned; x must not overlap out.
+ * Scratch: stream-ordered, from the library's pool (see above).
  */
 int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads,
                            const int* window, const int* shift,
@@ -188,7 +191,11 @@ int vswin_wmsa_forward_noalloc(const void* x, int B, int T, int H, int W, int C,
 
 /*
  * Index maps of the layer, written to caller-allocated device int32 buffers
- * (any of them may be NULL to skip it):
+ * (any of them may be NULL to skip it). They spell out steps 1-3 and 5 above:
+ * the padding and cyclic shift of the token grid and the window partition
+ * ("Video Swin Transformer" summary page, Method steps 4-5 and the window_msa
+ * pseudocode), the regions of the shifted-window mask (Method step 5) and the
+ * relative-position index of the bias table (Method step 8):
  *   win_src [B*nW*N]  flat source token b*T*H*W + (t*H + h)*W + w of each
  *                     window slot, or -1 for a padding slot;
  *   region  [nW*N]    9*rt + 3*rh + rw of each slot (0 when unshifted);

@@ -1,18 +1,27 @@
 // bf16 path of the layer on sm_100a tensor cores (tcgen05 / TMEM).
 //
-// Per chunk of windows, three launches:
-//   1. gemm_kernel<kQKV>:  gather window slots from x (roll + pad + partition
-//      folded into the row index, padding zero-filled by the copy), tcgen05 GEMM
-//      with Wqkv, epilogue adds bqkv, scales q by log2(e)/sqrt(d) and writes
-//      per-(window, head) q / k / v slabs in the tensor-core operand layout;
-//   2. attention_kernel:   per (window, head): S = q k^T on tcgen05 into TMEM,
-//      relative-position bias + shifted-window mask + softmax in registers
-//      (exp2 domain), P as bf16 back into TMEM, O = P v on tcgen05 with P
-//      read from TMEM; keys in up to three blocks, each with its own running
-//      max, merged in the epilogue;
-//   3. gemm_kernel<kPROJ>: tcgen05 GEMM of the attention output with Wproj,
-//      epilogue adds bproj and scatters rows back through the inverse window
-//      map (un-partition, roll by +shift, drop padding).
+// Per chunk of windows, four launches:
+//   1. row_source_kernel: the source token of every window slot of the chunk
+//      (roll + pad + partition as index arithmetic; -1 for padding). For the
+//      block entry row_stats_kernel does this and also writes each row's
+//      layer-norm statistics, after ln_fold_kernel has folded gamma and beta
+//      into the QKV weights once per call.
+//   2. gemm_ws_kernel<kQKV>: persistent warp-specialised tcgen05 GEMM (gather
+//      warps cp.async the rows named by the row table, zero-filling padding;
+//      one MMA warp; epilogue warps). The epilogue adds bqkv, scales q by
+//      log2(e)/sqrt(d) and writes per-(window, head) q / k / v slabs in the
+//      tensor-core operand layout. gemm_kernel<kQKV> is the tiled fallback
+//      used when the persistent kernel's resident weight slice does not fit.
+//   3. attention7_kernel: persistent warp-specialised attention for (P,7,7)
+//      windows: S = q k^T on tcgen05 into TMEM with the shifted-window mask
+//      and a per-row reference folded into one extra MMA step, relative-
+//      position bias and exp2 in registers, P as bf16 over S in TMEM,
+//      O = P v on tcgen05 with P read from TMEM. attention_kernel handles the
+//      other window shapes, one (window, head) per CTA.
+//   4. gemm_ws_kernel<kPROJ> (or gemm_kernel<kPROJ>): the attention output
+//      times Wproj, epilogue adds bproj (and, for the block entry, the
+//      residual) and scatters rows back through the row table (reverse
+//      partition, roll by +shift, drop padding).
 //
 // Shared-memory operand layout everywhere: the no-swizzle canonical layout of
 // 8-row x 16-byte core matrices (128 contiguous bytes).

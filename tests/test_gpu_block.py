@@ -135,3 +135,15 @@ def test_block_full_size_sampled():
         xs.append(xf[s[m]])
     _check(np.concatenate(got), np.concatenate(exp), np.concatenate(xs), True)
     assert np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("scale", ["baseline", "sensitivity"])
+def test_block_headline_whole_tensor(scale):
+    # the headline SW-MSA layer shape as a block, every output element against the oracle
+    wl = WORKLOADS["swin_t_s1_b8"]
+    layer = wl.layers[1]
+    inp = make_block_inputs(layer.shape, layer.heads, layer.window, "bf16", scale, seed=5400)
+    a = inp.as_f64()
+    out = _gpu(inp, layer.window, layer.shift, layer.heads)
+    ref = _ref(a, layer.window, layer.shift, layer.heads)
+    _check(out, ref, a["x"], scale == "sensitivity")

@@ -275,6 +275,42 @@ def test_bf16_full_size_baseline_gates_headline():
             _check_bf16(flat[s[m]], y[k][m], False)
 
 
+# ------------------------------------------------------------------ whole tensors: full size and multi-item
+# The persistent kernels give each CTA several (window, head) items and several GEMM
+# tiles only when a layer has more of them than the GPU has SMs. These cases compare
+# every output element with the oracle on layers where every CTA runs several items
+# (reused item buffers, barrier phases flipping across uses, a tile's epilogue deferred
+# into the next item, alternating TMEM accumulators in the GEMMs), including the
+# headline layers themselves.
+@pytest.mark.parametrize("scale", ["baseline", "sensitivity"])
+@pytest.mark.parametrize("k", [0, 1], ids=["wmsa", "swmsa"])
+def test_bf16_headline_whole_tensor(k, scale):
+    wl = WORKLOADS["swin_t_s1_b8"]
+    layer = wl.layers[k]
+    inp = workload_layer_inputs(wl, layer, scale=scale)
+    out = _gpu(inp, layer.window, layer.shift, layer.heads, "bf16")
+    ref = _oracle(inp.as_f64(), layer.window, layer.shift, layer.heads)
+    _check_bf16(out, ref, scale == "sensitivity")
+
+
+MULTI_ITEM_CASES = [
+    # (shape, heads, window, shift): items = windows x heads, per CTA on 148 SMs
+    ((8, 16, 28, 28, 96), 3, (8, 7, 7), (4, 3, 3)),    # 768 items (5.2 per CTA), 784 GEMM tiles
+    ((8, 16, 28, 28, 96), 3, (8, 7, 7), (0, 0, 0)),
+    ((8, 32, 28, 14, 128), 4, (16, 7, 7), (8, 3, 3)),  # N = 784, one item buffer: 512 items (3.5 per CTA)
+    ((4, 16, 28, 28, 64), 2, (4, 7, 7), (2, 3, 3)),    # 512 items of N = 196
+    ((8, 16, 32, 32, 64), 2, (4, 4, 4), (2, 2, 2)),    # generic kernel, 4096 items
+]
+
+
+@pytest.mark.parametrize("shape,heads,window,shift", MULTI_ITEM_CASES)
+def test_bf16_multi_item_whole_tensor(shape, heads, window, shift):
+    inp = make_layer_inputs(shape, heads, window, "bf16", "sensitivity", seed=7000 + sum(shape))
+    ref = _oracle(inp.as_f64(), window, shift, heads)
+    out = _gpu(inp, window, shift, heads, "bf16")
+    _check_bf16(out, ref, True)
+
+
 # ------------------------------------------------------------------ bounded waits
 def test_timeout_path_reports_and_recovers():
     vswin.set_wait_limit_ns(20_000_000)  # 20 ms
