@@ -275,3 +275,46 @@ def block_full_forward(x, attn, mlp, window, shift, heads, eps=LN_EPS):
     z = block_forward(x, attn["gamma"], attn["beta"], eps, window, shift, attn["Wqkv"], attn["bqkv"],
                       attn["Wproj"], attn["bproj"], attn["table"], heads)
     return mlp_half(z, mlp["gamma"], mlp["beta"], eps, mlp["W1"], mlp["b1"], mlp["W2"], mlp["b2"])
+
+
+def patch_merge_gather(x):
+    """The 2x2 spatial neighbour concatenation of patch merging, in float64.
+
+    "Video Swin Transformer" summary page, Method step 2 (each 2x2 group of
+    spatial neighbours, 4C values; no temporal merging) and the code walk-through
+    page, section 1.2 (PatchMerging: interval sampling of H and W, channels x4).
+    The pages do not fix the order of the four neighbours inside the 4C vector
+    nor what happens at an odd H or W. Readings taken: neighbour (dh, dw) of
+    merged token (i, j) is x[2i + dh, 2j + dw] and sits at channels
+    [(2 dw + dh) C, (2 dw + dh + 1) C) -- the order (0,0), (1,0), (0,1), (1,1) --
+    and an odd H or W is zero-padded by one row or column at the high end (the
+    padding convention of the window partition). Returns (B, T, ceil(H/2),
+    ceil(W/2), 4C).
+    """
+    x = _f64(x)
+    B, T, H, W, C = x.shape
+    Hp, Wp = H + H % 2, W + W % 2
+    xp = np.zeros((B, T, Hp, Wp, C))
+    xp[:, :, :H, :W] = x
+    parts = []
+    for dw in (0, 1):
+        for dh in (0, 1):
+            parts.append(xp[:, :, dh::2, dw::2, :])
+    return np.concatenate(parts, axis=-1)
+
+
+def patch_merge(x, gamma, beta, eps, Wr, br=None):
+    """Patch merging between stages in float64: LN over the 4C concatenation of each
+    2x2 spatial neighbourhood, then one linear layer 4C -> 2C.
+
+    "Video Swin Transformer" summary page, Method step 2 (concatenate each 2x2
+    group of spatial neighbours and project 4C to 2C with a linear layer); the
+    code walk-through page, section 1.2 (PatchMerging: nn.LayerNorm then
+    nn.Linear(4 * dim, 2 * dim)). Wr is [4C][2C]; ``br`` is an optional bias
+    (the pages do not say whether the projection has one; None = none).
+    """
+    z = layer_norm(patch_merge_gather(x), gamma, beta, eps)
+    y = z @ _f64(Wr)
+    if br is not None:
+        y = y + _f64(br)
+    return y

@@ -463,3 +463,61 @@ def test_w2_block_forward_windows_match_the_block(oracle_mod):
         s = src[w * N:(w + 1) * N]
         m = s >= 0
         np.testing.assert_allclose(y[k][m], full[s[m]], rtol=0, atol=1e-12)
+
+
+# ---- patch merging ------------------------------------------------------------------------------
+def test_pm1_gather_is_space_to_depth_up_to_a_channel_permutation(oracle_mod):
+    # torch's pixel_unshuffle is the textbook 2x2 space-to-depth: output channel c*4 + dh*2 + dw
+    # of (C, H, W) input holds x[c, 2i + dh, 2j + dw]. The oracle's gather must hold the same
+    # values with channel (2 dw + dh) C + c.
+    B, T, H, W, C = 2, 3, 6, 8, 5
+    x = np.random.default_rng(3).standard_normal((B, T, H, W, C))
+    g = oracle_mod.patch_merge_gather(x)
+    xt = torch.from_numpy(x).permute(0, 1, 4, 2, 3).reshape(B * T, C, H, W)
+    pu = torch.nn.functional.pixel_unshuffle(xt, 2).numpy()  # (BT, 4C, H/2, W/2)
+    pu = pu.reshape(B, T, C, 2, 2, H // 2, W // 2)           # c, dh, dw
+    ref = np.transpose(pu, (0, 1, 5, 6, 4, 3, 2)).reshape(B, T, H // 2, W // 2, 4 * C)  # dw, dh, c
+    np.testing.assert_array_equal(g, ref)
+
+
+def test_pm2_patch_merge_is_layer_norm_then_linear(oracle_mod):
+    # LN over the 4C vector (torch's layer_norm) then x @ Wr (torch's linear), float64
+    B, T, H, W, C = 1, 2, 4, 6, 8
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((B, T, H, W, C))
+    gamma, beta = 1 + 0.1 * rng.standard_normal(4 * C), 0.1 * rng.standard_normal(4 * C)
+    Wr, br = rng.standard_normal((4 * C, 2 * C)), rng.standard_normal(2 * C)
+    y = oracle_mod.patch_merge(x, gamma, beta, 1e-5, Wr, br)
+    xt = torch.from_numpy(x).permute(0, 1, 4, 2, 3).reshape(B * T, C, H, W)
+    cat = torch.nn.functional.pixel_unshuffle(xt, 2).reshape(B, T, C, 2, 2, H // 2, W // 2)
+    cat = cat.permute(0, 1, 5, 6, 4, 3, 2).reshape(B, T, H // 2, W // 2, 4 * C)
+    z = torch.nn.functional.layer_norm(cat, (4 * C,), torch.from_numpy(gamma), torch.from_numpy(beta), 1e-5)
+    ref = torch.nn.functional.linear(z, torch.from_numpy(Wr).T, torch.from_numpy(br)).numpy()
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12)
+    assert y.shape == (B, T, H // 2, W // 2, 2 * C)
+
+
+def test_pm3_odd_extent_is_zero_padding(oracle_mod):
+    # an odd H or W merges as if the input carried a zero row / column at the high end
+    B, T, H, W, C = 1, 2, 5, 7, 4
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((B, T, H, W, C))
+    xp = np.zeros((B, T, H + 1, W + 1, C))
+    xp[:, :, :H, :W] = x
+    np.testing.assert_array_equal(oracle_mod.patch_merge_gather(x), oracle_mod.patch_merge_gather(xp))
+    assert oracle_mod.patch_merge_gather(x).shape == (B, T, 3, 4, 4 * C)
+
+
+def test_pm4_no_temporal_merging_and_swin_t_shapes(oracle_mod):
+    # The pages: Swin-T stage 1 (B, 56, 56, 96) merges to (B, 28, 28, 192) with no temporal
+    # merging; a clip's frames stay separate (merging each frame alone gives the same result).
+    B, T, H, W, C = 1, 3, 56, 56, 96
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((B, T, H, W, C)).astype(np.float32)
+    gamma, beta = np.ones(4 * C), np.zeros(4 * C)
+    Wr = rng.standard_normal((4 * C, 2 * C)) / np.sqrt(4 * C)
+    y = oracle_mod.patch_merge(x, gamma, beta, 1e-5, Wr)
+    assert y.shape == (B, T, 28, 28, 192)
+    for t in range(T):
+        yt = oracle_mod.patch_merge(x[:, t:t + 1], gamma, beta, 1e-5, Wr)
+        np.testing.assert_allclose(y[:, t:t + 1], yt, rtol=0, atol=1e-12)
