@@ -111,6 +111,50 @@ int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, in
                             const void* bias_table, void* out, void* stream);
 
 /*
+ * bf16 forward of a block's MLP half ("Video Swin Transformer" summary page,
+ * Method step 3 and eq. 1: layer norm, a two-layer MLP with GELU, residual
+ * add; the code walk-through page, section 1.2, names nn.LayerNorm):
+ *   out = x + GELU(LN(x) W1 + b1) W2 + b2       for every token of x
+ * x, out       (B, T, H, W, C) bf16, channels last; out may be x (in place),
+ *              partial overlap is refused
+ * ln_gamma, ln_beta, ln_eps   as for vswin_block_msa_forward
+ * W1 [C][hidden], b1 [hidden], W2 [hidden][C], b2 [C]   bf16, row-major
+ * GELU is the erf form x * Phi(x) (torch.nn.GELU's default); the kernel
+ * evaluates it through a fitted tanh form on the hardware tanh, within 1e-3
+ * |x| of the erf form. Products accumulate in fp32 on the tensor cores; the
+ * normalised tokens and the hidden activations are rounded to bf16 as MMA
+ * operands and never leave the SM; the output is rounded once.
+ * Requires C a multiple of 32 up to 128 and hidden a multiple of 64 that
+ * splits into at most 8 hidden chunks of 128 (or 64) columns whose weights fit
+ * in shared memory -- hidden 4C for C = 32 .. 128 does -- else
+ * VSWIN_ERR_UNSUPPORTED; x, out, W1, W2 16-byte aligned, the vectors 2-byte
+ * aligned; B*T*H*W < 2^31. No scratch memory.
+ */
+int vswin_mlp_forward(const void* x, int B, int T, int H, int W, int C, int hidden,
+                      const void* ln_gamma, const void* ln_beta, float ln_eps,
+                      const void* W1, const void* b1, const void* W2, const void* b2,
+                      void* out, void* stream);
+
+/*
+ * bf16 forward of one whole Video Swin block ("Video Swin Transformer"
+ * summary page, Method step 3 and eq. 1):
+ *   z   = x + layer(LN1(x))               vswin_block_msa_forward
+ *   out = z + GELU(LN2(z) W1 + b1) W2 + b2 vswin_mlp_forward, in place on out
+ * The arguments are those of the two entry points (one ln_eps for both
+ * norms); every one of them is checked before anything is launched, and the
+ * requirements of both apply. out may be x. Scratch: that of
+ * vswin_block_msa_forward.
+ */
+int vswin_block_forward(const void* x, int B, int T, int H, int W, int C, int heads,
+                        const int* window, const int* shift,
+                        const void* ln1_gamma, const void* ln1_beta,
+                        const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                        const void* bias_table,
+                        const void* ln2_gamma, const void* ln2_beta, int hidden,
+                        const void* W1, const void* b1, const void* W2, const void* b2,
+                        float ln_eps, void* out, void* stream);
+
+/*
  * fp32 layer forward (plain FP32 FMA arithmetic, no tensor cores): every
  * tensor is float. The same layer as vswin_wmsa_forward, steps 1-7 above
  * ("Video Swin Transformer" summary page, Method steps 4-6 and eq. 2), with
@@ -259,7 +303,8 @@ enum {
   VSWIN_KERNEL_ATTENTION = 1,  /* window attention (bf16) */
   VSWIN_KERNEL_PROJ_GEMM = 2,  /* output projection + scatter (bf16) */
   VSWIN_KERNEL_OTHER = 3,      /* fp32 path, index maps, self-test */
-  VSWIN_KERNEL_KINDS = 4
+  VSWIN_KERNEL_MLP = 4,        /* fused MLP half of a block (bf16) */
+  VSWIN_KERNEL_KINDS = 5
 };
 int vswin_profile_enable(int on);
 int vswin_profile_collect(double* ms, unsigned long long* launches, int nkinds);

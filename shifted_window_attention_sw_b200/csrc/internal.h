@@ -26,7 +26,7 @@ void count_launch(int n = 1);
 // Optional per-kernel CUDA-event timing (vswin_profile_enable).
 void prof_begin(int kind, cudaStream_t st);
 void prof_end(int kind, cudaStream_t st);
-enum { kKindQkv = 0, kKindAttn = 1, kKindProj = 2, kKindOther = 3, kKinds = 4 };
+enum { kKindQkv = 0, kKindAttn = 1, kKindProj = 2, kKindOther = 3, kKindMlp = 4, kKinds = 5 };
 
 // fp32 path (simt_path.cu)
 cudaError_t launch_f32_forward(const Geom& g, const float* x, const float* Wqkv, const float* bqkv,
@@ -69,5 +69,12 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
                               const void* bqkv, const void* Wproj, const void* bproj, const void* table,
                               void* out, void* scratch, long long win0, long long nwin, cudaStream_t st,
                               const BlockFuse* fuse = nullptr);
+
+// MLP half of a block (mlp_path.cu): out = x + GELU(LN(x) W1 + b1) W2 + b2 for
+// M tokens of C channels, one fused persistent kernel. out may be x.
+bool mlp_supported(int C, int hidden);
+cudaError_t launch_mlp(const KernelCtx& ctx, long long M, int C, int hidden, const void* x, const void* gamma,
+                       const void* beta, float eps, const void* W1, const void* b1, const void* W2, const void* b2,
+                       void* out, cudaStream_t st);
 
 }  // namespace vswin

@@ -1,0 +1,566 @@
+// The MLP half of a Video Swin block on sm_100a tensor cores, fused into one
+// persistent kernel ("Video Swin Transformer" summary page, Method step 3 and
+// eq. 1: layer norm, a two-layer MLP with GELU, residual add):
+//
+//   out = x + GELU(LN(x) W1 + b1) W2 + b2        per token (row of x)
+//
+// One CTA per SM walks 128-token tiles. Per tile the tokens are read from HBM
+// once (TMA) and the result is written once (TMA store); the hidden
+// activations (128 x hidden) never leave the SM:
+//   * warp 0 loads x tiles (double-buffered) and the weight chunks (W1
+//     columns and W2 rows of one hidden chunk of HC = 128) with TMA; when
+//     every chunk fits in shared memory at once they are loaded once per CTA;
+//   * warps 2-5 normalise the tile in shared memory (fp32 statistics, bf16
+//     result in the MMA operand layout);
+//   * warp 1 issues, per hidden chunk, fc1 = LN(x) W1[:, chunk] into one of
+//     two TMEM accumulators, and fc2 += h_chunk W2[chunk, :] with h read
+//     from TMEM (the A operand of a TS MMA) into one of two output
+//     accumulators;
+//   * warps 2-9 turn each fc1 accumulator into h = GELU(acc + b1) (bf16,
+//     written over the accumulator's own columns), and at the end of a tile
+//     add b2 and the residual to the output accumulator, stage the bf16
+//     result over the tile's x in shared memory and store it with TMA.
+//
+// GELU: the erf form x * Phi(x) (torch.nn.GELU's default) evaluated as
+// 0.5 x (1 + tanh(x (g1 + g3 x^2 + g5 x^4))) with x^2 clamped at 64, whose
+// coefficients are a least-squares fit of Phi(x) = (1 + erf(x / sqrt(2))) / 2
+// over [-8, 8] (max abs error of the formula 3.3e-5); tanh is the hardware
+// tanh.approx.f32 (max relative error about 2^-11), so the GELU value carries
+// an absolute error below 1e-3 * |x|, under the bf16 rounding of h.
+//
+// Operand layouts in shared memory: the no-swizzle canonical layout (8-row x
+// 16-byte core matrices). A tile of x (128 rows x C) is stored as C/8 column
+// groups of 128 rows x 16 bytes (LBO = 2048 B along K, SBO = 128 B along M),
+// which is what one 3D TMA box (8 channels, 128 rows, C/8 groups) writes.
+// Weight chunks are MN-major: element (k, n) at (k/8)*LBO + (n/8)*128 +
+// (k%8)*16 + (n%8)*2, one 4D TMA box each.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace vswin {
+namespace {
+
+constexpr int kMlpMaxHC = 128;       // hidden columns per chunk: 128, or 64 when two 128-column stages do not fit
+constexpr int kMlpThreads = 10 * 32;  // producer, MMA, 8 epilogue warps
+constexpr int kMlpEpi0 = 2;           // first epilogue warp
+constexpr int kMlpMaxC = 128;
+
+// GELU via tanh: coefficients of x (g1 + g3 x^2 + g5 x^4), least-squares fit
+// of Phi on [-8, 8] (see the file comment).
+constexpr float kG1 = 0.797458471f, kG3 = 0.0370503451f, kG5 = -0.000358732362f;
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GELU of two values (packed fp32 arithmetic where the ISA has it).
+__device__ __forceinline__ float2 gelu2(float2 v) {
+  const float2 x2 = __fmul2_rn(v, v);
+  const float2 s = make_float2(fminf(x2.x, 64.f), fminf(x2.y, 64.f));
+  float2 p = __ffma2_rn(s, make_float2(kG5, kG5), make_float2(kG3, kG3));
+  p = __ffma2_rn(s, p, make_float2(kG1, kG1));
+  const float2 arg = __fmul2_rn(v, p);
+  const float2 t = make_float2(tanh_approx(arg.x), tanh_approx(arg.y));
+  const float2 hx = __fmul2_rn(v, make_float2(0.5f, 0.5f));
+  return __ffma2_rn(hx, t, hx);
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------ TMA
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+struct MlpArgs {
+  long long M;  // tokens (rows)
+  int C, hidden, hc, nch, stages;
+  bool resident;  // every weight chunk has its own stage (loaded once per CTA)
+  float eps;
+  const __nv_bfloat16* gamma;
+  const __nv_bfloat16* beta;
+  const __nv_bfloat16* b1;
+  const __nv_bfloat16* b2;
+  KernelCtx ctx;
+};
+
+// Shared-memory plan (bytes from the dynamically allocated base).
+struct MlpSmem {
+  int x0, x1, xn, w, wstage, w2off, gam, bet, b1, b2, bars, total;
+};
+__host__ __device__ inline MlpSmem mlp_smem(int C, int hidden, int hc, int stages) {
+  MlpSmem s;
+  const int xb = 128 * C * 2;
+  s.x0 = 0;
+  s.x1 = xb;
+  s.xn = 2 * xb;
+  s.w = 3 * xb;
+  s.w2off = C * hc * 2;  // W2 chunk after the W1 chunk inside a stage
+  s.wstage = 2 * C * hc * 2;
+  s.gam = s.w + stages * s.wstage;
+  s.bet = s.gam + C * 4;
+  s.b1 = s.bet + C * 4;
+  s.b2 = s.b1 + hidden * 4;
+  s.bars = (s.b2 + C * 4 + 15) / 16 * 16;
+  s.total = s.bars + 32 * 8 + 16;
+  return s;
+}
+
+__global__ void __launch_bounds__(kMlpThreads, 1)
+    mlp_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_out,
+               const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2, MlpArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int C = a.C, NCH = a.nch, S = a.stages, HC = a.hc;
+  const MlpSmem L = mlp_smem(C, a.hidden, HC, S);
+  uint8_t* sX[2] = {smem + L.x0, smem + L.x1};
+  uint8_t* sXn = smem + L.xn;
+  float* sGam = reinterpret_cast<float*>(smem + L.gam);
+  float* sBet = reinterpret_cast<float*>(smem + L.bet);
+  float* sB1 = reinterpret_cast<float*>(smem + L.b1);
+  float* sB2 = reinterpret_cast<float*>(smem + L.b2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* x_full = bars;         // [2] x tile landed
+  uint64_t* x_free = bars + 2;     // [2] x buffer's output store has read it
+  uint64_t* xn_full = bars + 4;    // normalised tile written (4 warps)
+  uint64_t* xn_free = bars + 5;    // the tile's fc1 MMAs have read it
+  uint64_t* acc1_full = bars + 6;  // [2]
+  uint64_t* h_full = bars + 8;     // [2] h written over the fc1 accumulator (8 warps)
+  uint64_t* acc2_full = bars + 10; // [2]
+  uint64_t* acc2_free = bars + 12; // [2] (8 warps)
+  uint64_t* w_full = bars + 14;    // [S <= 8]
+  uint64_t* w_free = bars + 22;    // [S <= 8]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 30);
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long mtiles = (a.M + 127) / 128;
+  const long long ntiles = mtiles > blockIdx.x ? (mtiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const uint64_t lim = a.ctx.wait_limit;
+  const uint32_t xbytes = 128u * (uint32_t)C * 2u;
+  const uint32_t wbytes = (uint32_t)(2 * C * HC * 2);
+
+  if (tid == 0) {
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&x_full[k], 1);
+      mbar_init(&x_free[k], 1);
+      mbar_init(&acc1_full[k], 1);
+      mbar_init(&h_full[k], 8);
+      mbar_init(&acc2_full[k], 1);
+      mbar_init(&acc2_free[k], 8);
+    }
+    mbar_init(xn_full, 4);
+    mbar_init(xn_free, 1);
+    for (int k = 0; k < S; ++k) {
+      mbar_init(&w_full[k], 1);
+      mbar_init(&w_free[k], 1);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  for (int c = tid; c < C; c += kMlpThreads) {
+    sGam[c] = __bfloat162float(a.gamma[c]);
+    sBet[c] = __bfloat162float(a.beta[c]);
+    sB2[c] = __bfloat162float(a.b2[c]);
+  }
+  for (int c = tid; c < a.hidden; c += kMlpThreads) sB1[c] = __bfloat162float(a.b1[c]);
+  if (warp == 1) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  // TMEM columns: fc1 accumulators [0, 128) and [128, 256); output
+  // accumulators [256, 256 + C) and [256 + C, 256 + 2C).
+  const uint32_t tAcc1 = tmem, tAcc2 = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      long long g = 0;  // global chunk counter
+      for (long long t = 0; t < ntiles && !s_abort; ++t) {
+        const long long m = blockIdx.x + t * gridDim.x;
+        const int xb = (int)(t & 1);
+        if (t >= 2 && !mbar_wait(&x_free[xb], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim)) {
+          s_abort = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&x_full[xb], xbytes);
+        tma_load_3d(sX[xb], &tm_x, 0, (int)(m * 128), 0, &x_full[xb]);
+        for (int c = 0; c < NCH; ++c, ++g) {
+          if (a.resident && t > 0) continue;
+          const int s = (int)(g % S);
+          if (g >= S && !mbar_wait(&w_free[s], (uint32_t)((g / S) - 1) & 1, a.ctx.err, kErrWaitMma, lim)) {
+            s_abort = 1;
+            break;
+          }
+          uint8_t* dst = smem + L.w + s * L.wstage;
+          mbar_arrive_expect_tx(&w_full[s], wbytes);
+          tma_load_4d(dst, &tm_w1, 0, 0, c * (HC / 8), 0, &w_full[s]);
+          tma_load_4d(dst + L.w2off, &tm_w2, 0, 0, 0, c * (HC / 8), &w_full[s]);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t id1 = idesc_bf16(128, HC, 0, 1);  // A K-major (x), B MN-major (W1)
+      const uint32_t id2 = idesc_bf16(128, C, 0, 1);       // A from TMEM (h), B MN-major (W2)
+      const uint32_t lbo1 = (uint32_t)(HC / 8) * 128u;  // W1 chunk: K-group stride
+      const uint32_t lbo2 = (uint32_t)(C / 8) * 128u;       // W2 chunk: K-group stride
+      const uint32_t xn_addr = smem_u32(sXn);
+      const long long total = ntiles * NCH;
+      auto stage_of = [&](long long g) -> int { return a.resident ? (int)(g % NCH) : (int)(g % S); };
+      auto w_phase = [&](long long g) -> uint32_t { return a.resident ? 0u : (uint32_t)(g / S) & 1; };
+      // fc1 of global chunk g: waits for its tile's normalised x (first chunk
+      // of a tile) and its weight stage
+      auto fc1 = [&](long long g) {
+        const long long t = g / NCH;
+        const int c = (int)(g % NCH);
+        if (c == 0 && !s_abort && !mbar_wait(xn_full, (uint32_t)t & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        const int s = stage_of(g);
+        if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        tc_fence_after();
+        if (s_abort) return;
+        const uint32_t wa = smem_u32(smem + L.w + s * L.wstage);
+        const uint32_t d = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_ss(d, smem_desc(xn_addr + ks * 2 * 2048, 2048, 128), smem_desc(wa + ks * 2 * lbo1, lbo1, 128), id1,
+                  ks > 0);
+        umma_commit(&acc1_full[g & 1]);
+        if (c == NCH - 1) umma_commit(xn_free);
+      };
+      if (total > 0) fc1(0);
+      if (total > 1) fc1(1);
+      for (long long g = 0; g < total && !s_abort; ++g) {
+        const long long t = g / NCH;
+        const int c = (int)(g % NCH);
+        const int ob = (int)(t & 1);
+        // h of chunk g is in TMEM (and its fc1 accumulator was read)
+        if (!mbar_wait(&h_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+        // the output accumulator of this tile was drained two tiles ago
+        if (c == 0 && t >= 2 && !s_abort &&
+            !mbar_wait(&acc2_free[ob], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+          s_abort = 1;
+        tc_fence_after();
+        if (s_abort) break;
+        const int s = stage_of(g);
+        const uint32_t wa2 = smem_u32(smem + L.w + s * L.wstage + L.w2off);
+        const uint32_t hb = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
+        const uint32_t d2 = tAcc2 + (uint32_t)ob * (uint32_t)C;
+        // h element k of the chunk sits at column hf * HC/2 + (k - hf * HC/2) / 2,
+        // hf = k / (HC/2) (each epilogue half packs its own columns in place)
+        for (int j = 0; j < HC / 16; ++j) {
+          const int hf = (16 * j) / (HC / 2);
+          const uint32_t hcol = (uint32_t)(hf * (HC / 2) + (16 * j - hf * (HC / 2)) / 2);
+          umma_ts(d2, hb + hcol, smem_desc(wa2 + j * 2 * lbo2, lbo2, 128), id2, (c > 0 || j > 0) ? 1u : 0u);
+        }
+        if (!a.resident) umma_commit(&w_free[s]);
+        if (c == NCH - 1) umma_commit(&acc2_full[ob]);
+        if (g + 2 < total) fc1(g + 2);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue warps
+    const int q = warp & 3;               // TMEM lane quarter
+    const int hf = (warp - kMlpEpi0) >> 2; // 0: warps 2-5, 1: warps 6-9
+    const int r = q * 32 + lane;          // this thread's row of the tile
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const bool norm_warp = hf == 0;
+    // Normalise tile t (norm warps): row r of sX[t & 1] -> sXn.
+    auto normalise = [&](long long t) {
+      const int xb = (int)(t & 1);
+      if (!s_abort && !mbar_wait(&x_full[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      if (t >= 1 && !s_abort && !mbar_wait(xn_free, (uint32_t)(t - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+        s_abort = 1;
+      if (!s_abort) {
+        const uint8_t* src = sX[xb] + r * 16;
+        uint4 v[kMlpMaxC / 8];
+        float sum = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMlpMaxC / 8; ++k) {
+          if (k < C / 8) {
+            v[k] = *reinterpret_cast<const uint4*>(src + k * 2048);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              sum += f.x + f.y;
+            }
+          }
+        }
+        const float mean = sum / (float)C;
+        float ss = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMlpMaxC / 8; ++k) {
+          if (k < C / 8) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              const float d0 = f.x - mean, d1 = f.y - mean;
+              ss = fmaf(d0, d0, fmaf(d1, d1, ss));
+            }
+          }
+        }
+        const float rstd = 1.0f / sqrtf(ss / (float)C + a.eps);
+        uint8_t* dst = sXn + r * 16;
+#pragma unroll
+        for (int k = 0; k < kMlpMaxC / 8; ++k) {
+          if (k < C / 8) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              const int ch = k * 8 + 2 * e;
+              w[e] = pack2(fmaf((f.x - mean) * rstd, sGam[ch], sBet[ch]),
+                           fmaf((f.y - mean) * rstd, sGam[ch + 1], sBet[ch + 1]));
+            }
+            *reinterpret_cast<uint4*>(dst + k * 2048) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();  // generic writes -> tensor-core operand reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(xn_full);
+    };
+    // GELU of chunk g: this warp's HC/2 fc1 columns (half hf of the chunk) ->
+    // HC/4 columns of bf16 pairs over the first half of the same columns.
+    auto gelu_chunk = [&](long long g) {
+      const int c = (int)(g % NCH);
+      if (!s_abort && !mbar_wait(&acc1_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
+        s_abort = 1;
+      tc_fence_after();
+      if (!s_abort) {
+        const uint32_t ta = tAcc1 + lane_base + (uint32_t)(g & 1) * (uint32_t)HC + (uint32_t)(hf * (HC / 2));
+        const float* b1 = sB1 + c * HC + hf * (HC / 2);
+        uint32_t u[32], w[16];
+        for (int part = 0; part < HC / 64; ++part) {
+          tmem_ld32(ta + 32 * part, u);
+          tmem_wait_ld_keep(u);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 bb = *reinterpret_cast<const float2*>(b1 + 32 * part + 2 * e);
+            const float2 v = __fadd2_rn(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), bb);
+            const float2 gv = gelu2(v);
+            w[e] = pack2(gv.x, gv.y);
+          }
+          tmem_st16(ta + 16 * part, w);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(&h_full[g & 1]);
+    };
+    // Output of tile t: acc2 + b2 + x -> bf16 over x in shared memory, then one
+    // thread stores the tile with TMA and releases the x buffer.
+    auto finish_tile = [&](long long t) {
+      const int xb = (int)(t & 1), ob = (int)(t & 1);
+      if (!s_abort && !mbar_wait(&acc2_full[ob], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      tc_fence_after();
+      if (!s_abort) {
+        const int half = C / 2;  // a multiple of 16
+        const uint32_t ta = tAcc2 + lane_base + (uint32_t)ob * (uint32_t)C + (uint32_t)(hf * half);
+        uint8_t* row = sX[xb] + r * 16;
+        for (int c0 = 0; c0 < half; c0 += 16) {
+          uint32_t u[16];
+          tmem_ld16(ta + c0, u);
+          tmem_wait_ld_keep(u);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int ch = hf * half + c0 + 8 * k;  // first channel of this 8-channel group
+            uint4* p = reinterpret_cast<uint4*>(row + (ch >> 3) * 2048);
+            const uint4 xv = *p;
+            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 xf = __bfloat1622float2(x2[e]);
+              const float2 bb = *reinterpret_cast<const float2*>(sB2 + ch + 2 * e);
+              float2 v = __fadd2_rn(make_float2(__uint_as_float(u[8 * k + 2 * e]), __uint_as_float(u[8 * k + 2 * e + 1])),
+                                    bb);
+              v = __fadd2_rn(v, xf);
+              w[e] = pack2(v.x, v.y);
+            }
+            *p = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(&acc2_free[ob]);
+      fence_proxy_async_smem();  // staged rows -> TMA store
+      named_sync(1, 8 * 32);
+      if (warp == kMlpEpi0 && lane == 0) {
+        if (!s_abort) {
+          const long long m = blockIdx.x + t * gridDim.x;
+          tma_store_3d(&tm_out, sX[xb], 0, (int)(m * 128), 0);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        mbar_arrive_cta(&x_free[xb]);
+      }
+    };
+
+    long long g = 0;
+    if (norm_warp && ntiles > 0) normalise(0);
+    for (long long t = 0; t < ntiles; ++t) {
+      for (int c = 0; c < NCH; ++c, ++g) gelu_chunk(g);
+      if (norm_warp && t + 1 < ntiles) normalise(t + 1);
+      finish_tile(t);
+    }
+    if (warp == kMlpEpi0 && lane == 0) bulk_wait0();  // the last stores have completed
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// bf16 tensor map of `rank` dims (dims[0] innermost), strides in bytes for
+// dims 1.., box sizes per dim; no swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+              const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Hidden chunk width and weight stages that fit next to the x buffers: one
+// stage per chunk (resident) when they all fit, else 2 (streamed), with
+// 128-column chunks when possible, else 64; {0, 0} when nothing fits.
+struct MlpPlan {
+  int hc, stages;
+};
+MlpPlan mlp_plan(int C, int hidden) {
+  for (int hc = kMlpMaxHC; hc >= 64; hc /= 2) {
+    if (hidden % hc) continue;
+    const int nch = hidden / hc;
+    if (nch > 8) continue;
+    const int base = mlp_smem(C, hidden, hc, 0).total;
+    const int room = (227 * 1024 - 1024 - base) / (2 * C * hc * 2);  // 1 KB left for static shared memory
+    if (room >= nch) return {hc, nch};
+    if (room >= 2) return {hc, 2};
+  }
+  return {0, 0};
+}
+
+}  // namespace
+
+bool mlp_supported(int C, int hidden) {
+  return C >= 32 && C <= kMlpMaxC && C % 32 == 0 && hidden >= 64 && mlp_plan(C, hidden).stages > 0;
+}
+
+cudaError_t launch_mlp(const KernelCtx& ctx, long long M, int C, int hidden, const void* x, const void* gamma,
+                       const void* beta, float eps, const void* W1, const void* b1, const void* W2, const void* b2,
+                       void* out, cudaStream_t st) {
+  if (!mlp_supported(C, hidden) || M <= 0 || M > (1LL << 31) - 1) return cudaErrorInvalidValue;
+  const MlpPlan plan = mlp_plan(C, hidden);
+  const int S = plan.stages, HC = plan.hc;
+  CUtensorMap mx, mo, m1, m2;
+  // x / out as (8 channels, M rows, C/8 groups): one box is a 128-row tile in
+  // the K-major operand layout
+  const cuuint64_t xd[3] = {8, (cuuint64_t)M, (cuuint64_t)(C / 8)};
+  const cuuint64_t xs[2] = {(cuuint64_t)C * 2, 16};
+  const cuuint32_t xbox[3] = {8, 128, (cuuint32_t)(C / 8)};
+  // W1 [C][hidden] as (8 n, 8 k, hidden/8 n-groups, C/8 k-groups); box = one
+  // hidden chunk, all of K
+  const cuuint64_t w1d[4] = {8, 8, (cuuint64_t)(hidden / 8), (cuuint64_t)(C / 8)};
+  const cuuint64_t w1s[3] = {(cuuint64_t)hidden * 2, 16, (cuuint64_t)hidden * 16};
+  const cuuint32_t w1box[4] = {8, 8, (cuuint32_t)(HC / 8), (cuuint32_t)(C / 8)};
+  // W2 [hidden][C] as (8 n, 8 k, C/8 n-groups, hidden/8 k-groups); box = the
+  // rows of one hidden chunk, all of N
+  const cuuint64_t w2d[4] = {8, 8, (cuuint64_t)(C / 8), (cuuint64_t)(hidden / 8)};
+  const cuuint64_t w2s[3] = {(cuuint64_t)C * 2, 16, (cuuint64_t)C * 16};
+  const cuuint32_t w2box[4] = {8, 8, (cuuint32_t)(C / 8), (cuuint32_t)(HC / 8)};
+  if (!make_map(&mx, x, 3, xd, xs, xbox) || !make_map(&mo, out, 3, xd, xs, xbox) ||
+      !make_map(&m1, W1, 4, w1d, w1s, w1box) || !make_map(&m2, W2, 4, w2d, w2s, w2box))
+    return cudaErrorInvalidValue;
+  MlpArgs a;
+  a.M = M;
+  a.C = C;
+  a.hidden = hidden;
+  a.hc = HC;
+  a.nch = hidden / HC;
+  a.stages = S;
+  a.resident = S == a.nch;
+  a.eps = eps;
+  a.gamma = static_cast<const __nv_bfloat16*>(gamma);
+  a.beta = static_cast<const __nv_bfloat16*>(beta);
+  a.b1 = static_cast<const __nv_bfloat16*>(b1);
+  a.b2 = static_cast<const __nv_bfloat16*>(b2);
+  a.ctx = ctx;
+  const int smem = mlp_smem(C, hidden, HC, S).total;
+  cudaError_t e = cudaFuncSetAttribute(mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = (M + 127) / 128;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  prof_begin(kKindMlp, st);
+  mlp_kernel<<<grid, kMlpThreads, smem, st>>>(mx, mo, m1, m2, a);
+  prof_end(kKindMlp, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace vswin

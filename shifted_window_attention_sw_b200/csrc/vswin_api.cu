@@ -200,6 +200,41 @@ long long chunk_windows(const Geom& g) {
   return (g.windows + nchunks - 1) / nchunks;
 }
 
+// Arguments of the MLP half (see vswin_mlp_forward); M = tokens on success.
+int check_mlp_args(const void* x, int B, int T, int H, int W, int C, int hidden, const void* ln_gamma,
+                   const void* ln_beta, float ln_eps, const void* W1, const void* b1, const void* W2, const void* b2,
+                   const void* out, long long* M_out) {
+  if (B <= 0 || T <= 0 || H <= 0 || W <= 0 || C <= 0 || hidden <= 0)
+    return fail(VSWIN_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d H=%d W=%d C=%d hidden=%d)", B, T, H, W,
+                C, hidden);
+  const void* ptrs[] = {x, ln_gamma, ln_beta, W1, b1, W2, b2, out};
+  const char* names[] = {"x", "ln_gamma", "ln_beta", "W1", "b1", "W2", "b2", "out"};
+  for (int k = 0; k < 8; ++k)
+    if (!ptrs[k]) return fail(VSWIN_ERR_INVALID_ARG, "%s is NULL", names[k]);
+  const void* big[] = {x, W1, W2, out};
+  const char* bign[] = {"x", "W1", "W2", "out"};
+  for (int k = 0; k < 4; ++k)
+    if (!aligned(big[k], 16)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not 16-byte aligned", bign[k]);
+  const void* vec[] = {ln_gamma, ln_beta, b1, b2};
+  const char* vecn[] = {"ln_gamma", "ln_beta", "b1", "b2"};
+  for (int k = 0; k < 4; ++k)
+    if (!aligned(vec[k], 2)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not 2-byte aligned", vecn[k]);
+  if (!(ln_eps >= 0.f) || !std::isfinite(ln_eps))
+    return fail(VSWIN_ERR_INVALID_ARG, "ln_eps must be finite and >= 0 (got %g)", (double)ln_eps);
+  const long long M = (long long)B * T * H * W;
+  if (M > (1LL << 31) - 1) return fail(VSWIN_ERR_UNSUPPORTED, "B * T * H * W exceeds 2^31");
+  const size_t act = (size_t)M * C * 2;
+  if (x != out && overlap(x, act, out, act))
+    return fail(VSWIN_ERR_INVALID_ARG, "x and out overlap without being equal");
+  if (!mlp_supported(C, hidden))
+    return fail(VSWIN_ERR_UNSUPPORTED,
+                "the fused MLP needs C a multiple of 32 up to 128 and hidden a multiple of 64 that splits "
+                "into at most 8 chunks whose weights fit in shared memory (C=%d hidden=%d)",
+                C, hidden);
+  *M_out = M;
+  return VSWIN_OK;
+}
+
 int forward_bf16_device(const void* x, const Geom& g, const void* Wqkv, const void* bqkv, const void* Wproj,
                         const void* bproj, const void* table, void* out, cudaStream_t st) {
   if (g.d != 32) return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path needs head width 32 (C/heads = %d)", g.d);
@@ -280,7 +315,7 @@ std::atomic<int> g_prof_on{0};
 std::mutex g_prof_mu;
 std::vector<ProfRecord> g_prof_records;
 std::vector<cudaEvent_t> g_prof_pool;
-cudaEvent_t g_prof_open[kKinds] = {nullptr, nullptr, nullptr, nullptr};
+cudaEvent_t g_prof_open[kKinds] = {};
 
 cudaEvent_t prof_event() {
   if (!g_prof_pool.empty()) {
@@ -415,6 +450,53 @@ int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, in
     return fail(VSWIN_ERR_INVALID_ARG, "ln_eps must be finite and >= 0 (got %g)", (double)ln_eps);
   return forward_block_device(x, g, ln_gamma, ln_beta, ln_eps, Wqkv, bqkv, Wproj, bproj, bias_table, out,
                               static_cast<cudaStream_t>(stream));
+}
+
+int vswin_mlp_forward(const void* x, int B, int T, int H, int W, int C, int hidden, const void* ln_gamma,
+                      const void* ln_beta, float ln_eps, const void* W1, const void* b1, const void* W2,
+                      const void* b2, void* out, void* stream) {
+  long long M = 0;
+  int st = check_mlp_args(x, B, T, H, W, C, hidden, ln_gamma, ln_beta, ln_eps, W1, b1, W2, b2, out, &M);
+  if (st != VSWIN_OK) return st;
+  KernelCtx ctx;
+  st = make_ctx(&ctx);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = launch_mlp(ctx, M, C, hidden, x, ln_gamma, ln_beta, ln_eps, W1, b1, W2, b2, out,
+                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "MLP kernel launch");
+  return VSWIN_OK;
+}
+
+int vswin_block_forward(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                        const int* shift, const void* ln1_gamma, const void* ln1_beta, const void* Wqkv,
+                        const void* bqkv, const void* Wproj, const void* bproj, const void* bias_table,
+                        const void* ln2_gamma, const void* ln2_beta, int hidden, const void* W1, const void* b1,
+                        const void* W2, const void* b2, float ln_eps, void* out, void* stream) {
+  // every argument of both halves is checked before anything is launched
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  st = check_layer_ptrs(x, Wqkv, bqkv, Wproj, bproj, bias_table, out, g, 2, 16, true);
+  if (st != VSWIN_OK) return st;
+  if (!ln1_gamma || !ln1_beta) return fail(VSWIN_ERR_INVALID_ARG, "ln1_gamma and ln1_beta must be non-NULL");
+  if (!aligned(ln1_gamma, 2) || !aligned(ln1_beta, 2))
+    return fail(VSWIN_ERR_INVALID_ARG, "ln1_gamma and ln1_beta must be 2-byte aligned");
+  long long M = 0;
+  st = check_mlp_args(out, B, T, H, W, C, hidden, ln2_gamma, ln2_beta, ln_eps, W1, b1, W2, b2, out, &M);
+  if (st != VSWIN_OK) return st;
+  if (g.d != 32) return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path needs head width 32 (C/heads = %d)", g.d);
+  if (!bf16_window_supported(g))
+    return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path has no kernel for window (%d,%d,%d)", g.win[0], g.win[1],
+                g.win[2]);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = forward_block_device(x, g, ln1_gamma, ln1_beta, ln_eps, Wqkv, bqkv, Wproj, bproj, bias_table, out, s);
+  if (st != VSWIN_OK) return st;
+  KernelCtx ctx;
+  st = make_ctx(&ctx);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = launch_mlp(ctx, M, C, hidden, out, ln2_gamma, ln2_beta, ln_eps, W1, b1, W2, b2, out, s);
+  if (e != cudaSuccess) return fail_cuda(e, "MLP kernel launch");
+  return VSWIN_OK;
 }
 
 int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,

@@ -16,6 +16,11 @@ Recipe (stands in for Kinetics clips; no dataset is used):
 Block inputs (layer norm + layer + residual) add, from seeds k = 6, 7, 8: a
 per-token offset ~ N(0, 0.5) added to x (so that the norm's centring matters),
 gamma ~ 1 + N(0, 0.1) and beta ~ N(0, 0.1).
+
+MLP-half inputs (layer norm + two linear layers with GELU + residual), seeds
+k = 10..16: x ~ N(0, 1) plus a per-token offset ~ N(0, 0.5); gamma ~ 1 + N(0, 0.1),
+beta ~ N(0, 0.1); "baseline" W1, W2 ~ N(0, 0.02) and biases 0; "sensitivity"
+W1 ~ N(0, 1/C), W2 ~ N(0, 1/hidden), biases ~ N(0, 0.1).
 """
 
 from __future__ import annotations
@@ -117,3 +122,42 @@ def make_block_inputs(shape, heads, window, dtype="bf16", scale="baseline", seed
     beta = _randn((C,), seed + 8, 0.1).to(dt).contiguous()
     li = LayerInputs(x, li.Wqkv, li.bqkv, li.Wproj, li.bproj, li.table)
     return BlockInputs(li, gamma, beta)
+
+
+@dataclass
+class MlpInputs:
+    x: torch.Tensor
+    gamma: torch.Tensor
+    beta: torch.Tensor
+    W1: torch.Tensor
+    b1: torch.Tensor
+    W2: torch.Tensor
+    b2: torch.Tensor
+
+    _KEYS = ("x", "gamma", "beta", "W1", "b1", "W2", "b2")
+
+    def as_f64(self):
+        return {k: getattr(self, k).to(torch.float64).numpy() for k in self._KEYS}
+
+    def to(self, device):
+        return MlpInputs(*(getattr(self, k).to(device) for k in self._KEYS))
+
+
+def make_mlp_inputs(shape, hidden, dtype="bf16", scale="baseline", seed=1000) -> MlpInputs:
+    """Inputs for one call of a block's MLP half. ``shape`` = (B, T, H, W, C)."""
+    B, T, H, W, C = shape
+    dt = _DT[dtype]
+    if scale == "baseline":
+        w1_std, w2_std, b_std = 0.02, 0.02, 0.0
+    elif scale == "sensitivity":
+        w1_std, w2_std, b_std = 1.0 / np.sqrt(C), 1.0 / np.sqrt(hidden), 0.1
+    else:
+        raise ValueError(scale)
+    x = _randn((B, T, H, W, C), seed + 10, 1.0) + _randn((B, T, H, W, 1), seed + 11, 0.5)
+    gamma = 1.0 + _randn((C,), seed + 12, 0.1)
+    beta = _randn((C,), seed + 13, 0.1)
+    W1 = _randn((C, hidden), seed + 14, w1_std)
+    W2 = _randn((hidden, C), seed + 15, w2_std)
+    b1 = _randn((hidden,), seed + 16, b_std) if b_std else torch.zeros(hidden)
+    b2 = _randn((C,), seed + 17, b_std) if b_std else torch.zeros(C)
+    return MlpInputs(*(t.to(dt).contiguous() for t in (x, gamma, beta, W1, b1, W2, b2)))

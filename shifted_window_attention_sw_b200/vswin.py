@@ -36,9 +36,11 @@ EXPORTS = (
     "vswin_set_exact_softmax",
     "vswin_block_msa_forward",
     "vswin_wmsa_backward_f32",
+    "vswin_mlp_forward",
+    "vswin_block_forward",
 )
 
-KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other")
+KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other", "mlp")
 
 
 class VswinError(RuntimeError):
@@ -71,6 +73,12 @@ def lib():
         L.vswin_block_msa_forward.restype = _I
         L.vswin_wmsa_backward_f32.argtypes = layer[:15] + [_P] * 6 + [_P]  # ..., dy, six gradients, stream
         L.vswin_wmsa_backward_f32.restype = _I
+        L.vswin_mlp_forward.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
+                                        _P]
+        L.vswin_mlp_forward.restype = _I
+        L.vswin_block_forward.argtypes = (layer[:9] + [_P, _P] + [_P] * 5 + [_P, _P, _I] + [_P] * 4 +
+                                          [ctypes.c_float, _P, _P])
+        L.vswin_block_forward.restype = _I
         L.vswin_wmsa_index_maps.argtypes = [_I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P]
         L.vswin_wmsa_index_maps.restype = _I
         L.vswin_clamp_window.argtypes = [_I, _I, _I, _IP, _IP, _IP, _IP]
@@ -206,6 +214,56 @@ def block_msa_forward(x, window, shift, gamma, beta, eps, Wqkv, bqkv, Wproj, bpr
             _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(gamma), _ptr(beta), float(eps),
             _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj), _ptr(bproj), _ptr(table), _ptr(out),
             _stream_handle(stream, x.device)))
+    return out
+
+
+def mlp_forward(x, gamma, beta, eps, W1, b1, W2, b2, out=None, stream=None):
+    """bf16 forward of a block's MLP half, out = x + GELU(LN(x) W1 + b1) W2 + b2, as one
+    fused kernel. W1 [C][hidden], W2 [hidden][C]. ``out`` may be ``x``."""
+    if out is None:
+        out = torch.empty_like(x)
+    _prep(x, dict(x=x, gamma=gamma, beta=beta, W1=W1, b1=b1, W2=W2, b2=b2, out=out), torch.bfloat16, x.device)
+    if x.dim() != 5:
+        raise ValueError(f"x must be (B, T, H, W, C), got shape {tuple(x.shape)}")
+    B, T, H, W, C = x.shape
+    if W1.dim() != 2 or W1.shape[0] != C:
+        raise ValueError(f"W1 must have shape ({C}, hidden), got {tuple(W1.shape)}")
+    hidden = W1.shape[1]
+    want = {"gamma": (gamma, (C,)), "beta": (beta, (C,)), "b1": (b1, (hidden,)), "W2": (W2, (hidden, C)),
+            "b2": (b2, (C,)), "out": (out, tuple(x.shape))}
+    for name, (t, shape) in want.items():
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    with torch.cuda.device(x.device):
+        _check(lib().vswin_mlp_forward(_ptr(x), B, T, H, W, C, int(hidden), _ptr(gamma), _ptr(beta), float(eps),
+                                       _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(out),
+                                       _stream_handle(stream, x.device)))
+    return out
+
+
+def block_forward(x, window, shift, attn, mlp, heads, eps=1e-5, out=None, stream=None):
+    """bf16 forward of a whole block: z = x + layer(LN1(x)), out = z + MLP(LN2(z)).
+    ``attn`` = dict(gamma, beta, Wqkv, bqkv, Wproj, bproj, table); ``mlp`` = dict(gamma, beta,
+    W1, b1, W2, b2). ``out`` may be ``x``."""
+    if out is None:
+        out = torch.empty_like(x)
+    _layer_args(x, window, heads, torch.bfloat16, attn["Wqkv"], attn["bqkv"], attn["Wproj"], attn["bproj"],
+                attn["table"], out, gamma1=attn["gamma"], beta1=attn["beta"], gamma2=mlp["gamma"], beta2=mlp["beta"],
+                W1=mlp["W1"], b1=mlp["b1"], W2=mlp["W2"], b2=mlp["b2"])
+    B, T, H, W, C = x.shape
+    hidden = mlp["W1"].shape[1] if mlp["W1"].dim() == 2 else -1
+    want = {"gamma1": (attn["gamma"], (C,)), "beta1": (attn["beta"], (C,)), "gamma2": (mlp["gamma"], (C,)),
+            "beta2": (mlp["beta"], (C,)), "W1": (mlp["W1"], (C, hidden)), "b1": (mlp["b1"], (hidden,)),
+            "W2": (mlp["W2"], (hidden, C)), "b2": (mlp["b2"], (C,))}
+    for name, (t, shape) in want.items():
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    with torch.cuda.device(x.device):
+        _check(lib().vswin_block_forward(
+            _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(attn["gamma"]), _ptr(attn["beta"]),
+            _ptr(attn["Wqkv"]), _ptr(attn["bqkv"]), _ptr(attn["Wproj"]), _ptr(attn["bproj"]), _ptr(attn["table"]),
+            _ptr(mlp["gamma"]), _ptr(mlp["beta"]), int(hidden), _ptr(mlp["W1"]), _ptr(mlp["b1"]), _ptr(mlp["W2"]),
+            _ptr(mlp["b2"]), float(eps), _ptr(out), _stream_handle(stream, x.device)))
     return out
 
 

@@ -291,3 +291,48 @@ def test_binding_rejects_mixed_devices(L):
     with pytest.raises(ValueError, match="cuda:0"):
         vswin.wmsa_forward(f["x"], (8, 7, 7), (4, 3, 3), f["Wqkv"], f["bqkv"], f["Wproj"], f["bproj"], f["table"],
                            3, out=out)
+
+
+def _call_mlp(L, x=A16, B=1, T=8, H=14, W=14, C=96, hidden=384, gamma=A16 * 7, beta=A16 * 8, eps=1e-5,
+              W1=A16 * 2, b1=A16 * 3, W2=A16 * 4, b2=A16 * 5, out=A16 * 64):
+    p = lambda v: ctypes.c_void_p(v) if v else None  # noqa: E731
+    return L.vswin_mlp_forward(p(x), B, T, H, W, C, hidden, p(gamma), p(beta), ctypes.c_float(eps), p(W1), p(b1),
+                               p(W2), p(b2), p(out), None)
+
+
+@pytest.mark.parametrize(
+    "kw",
+    [dict(B=0), dict(C=0), dict(hidden=-1), dict(x=0), dict(out=0), dict(W1=0), dict(b1=0), dict(W2=0),
+     dict(b2=0), dict(gamma=0), dict(beta=0),
+     dict(W1=A16 * 2 + 8),          # not 16-byte aligned (TMA)
+     dict(b1=A16 * 3 + 1),          # not 2-byte aligned
+     dict(eps=-1.0), dict(eps=float("nan")),
+     dict(out=A16 + 64)],           # overlaps x without being x
+)
+def test_mlp_invalid_arguments_launch_nothing(L, kw):
+    before = vswin.launch_count()
+    rc = _call_mlp(L, **kw)
+    assert rc == vswin.ERR_INVALID_ARG, (rc, vswin.last_error())
+    assert vswin.launch_count() == before
+
+
+@pytest.mark.parametrize("kw", [dict(C=160, hidden=640), dict(C=48, hidden=192), dict(C=96, hidden=100),
+                                dict(C=96, hidden=32 * 64), dict(B=1 << 20, T=16, H=56, W=56)])
+def test_mlp_unsupported_shapes(L, kw):
+    before = vswin.launch_count()
+    rc = _call_mlp(L, out=A16, **kw)  # in place passes the pointer checks
+    assert rc == vswin.ERR_UNSUPPORTED, (rc, vswin.last_error())
+    assert vswin.launch_count() == before
+
+
+def test_whole_block_checks_both_halves_before_launching(L):
+    # a bad MLP argument must stop the call before the attention half is launched
+    w = (ctypes.c_int * 3)(8, 7, 7)
+    s = (ctypes.c_int * 3)(4, 3, 3)
+    p = lambda k: ctypes.c_void_p(A16 * k)  # noqa: E731
+    before = vswin.launch_count()
+    for hidden, W1 in ((384, ctypes.c_void_p(A16 * 20 + 8)), (100, p(20))):  # misaligned W1; bad hidden
+        rc = L.vswin_block_forward(p(1), 1, 8, 14, 14, 96, 3, w, s, p(2), p(3), p(4), p(5), p(6), p(7), p(8), p(9),
+                                   p(10), hidden, W1, p(21), p(22), p(23), ctypes.c_float(1e-5), p(1), None)
+        assert rc in (vswin.ERR_INVALID_ARG, vswin.ERR_UNSUPPORTED), (rc, vswin.last_error())
+    assert vswin.launch_count() == before
