@@ -53,6 +53,28 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def cpu_model():
+    """The host CPU's model name (first processor in /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+# The MUFU (special-function unit) rate of sm_100: 16 ex2 results per clock per SM.
+MUFU_EX2_PER_CLK_SM = 16
+SMS = 148
+
+
+def exp_bound_us(exps, sm_mhz):
+    """Time the exponentials alone need on the MUFU at the given SM clock."""
+    return exps / (SMS * MUFU_EX2_PER_CLK_SM * sm_mhz * 1e6) * 1e6
+
+
 def workload_config(wl):
     layers = []
     for ly in wl.layers:
@@ -195,6 +217,7 @@ def run_reference(args):
         "config": workload_config(wl),
         "tflops": value * work["flops"] / work["tokens"] / 1e12,
         "cpu_baseline": {"kind": "oracle", "value": value, "unit": "tokens/s", "cores": cores,
+                         "cpu_model": cpu_model(),
                          "sample": f"{nwin} whole windows of each layer per step (evenly spaced), "
                                    f"double precision, OpenMP over windows"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -317,10 +340,22 @@ def run_gpu(args):
         raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_s = sum(step_ms) / 1e3
+    # the same steps with L2 left warm (no flush between steps): the inputs of one layer
+    # (77 MB) fit in the 126 MB L2, so this is the best case the cold number is bounded by
+    n_warm = max(1, min(args.steps, 20))
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step()
+    w0.record(stream)
+    for _ in range(n_warm):
+        step()
+    w1.record(stream)
+    torch.cuda.synchronize(device)
+    warm_s = w0.elapsed_time(w1) / 1e3
     step_stats = {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}
     work = step_work(wl)
     max_s, tokens, nranks = replicas.combine(total_s, work["tokens"] * args.steps, device)
     value = tokens / max_s
+    warm_max_s, warm_tokens, _ = replicas.combine(warm_s, work["tokens"] * n_warm, device)
     tflops = nranks * work["flops"] * args.steps / max_s / 1e12
 
     # end to end through the host-buffer entry point: H2D of x and D2H of out inside the timing
@@ -370,13 +405,23 @@ def run_gpu(args):
         peak = float(peaks["bf16_tflops"])
         traffic_kernel = "gemm_kernel"
     tr = traffic_record(traffic_kernel)
+    avg_us = 1e3 * dom_ms / max(1, dom_launches)
     roofline = {
         "kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
         "frac": achieved / peak, "peak_source": f"{peak_src} bf16 dense (burst)",
-        "avg_launch_us": 1e3 * dom_ms / max(1, dom_launches), "launches": dom_launches,
+        "avg_launch_us": avg_us, "launches": dom_launches,
         "traffic": tr["bytes_per_launch"] if tr else None,
         "units_per_launch": "windows x heads of one chunk; FLOPs 4*windows*N^2*C per layer",
     }
+    if dom == "attention":
+        # the exponentials' own floor on the MUFU (16 ex2 / clock / SM) at the clock seen
+        # during the timed region, beside the tensor roofline
+        mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+        exps_launch = work["exps"] / len(layers)
+        roofline["exp_bound_us"] = exp_bound_us(exps_launch, mhz)
+        roofline["exp_bound_frac"] = roofline["exp_bound_us"] / avg_us
+        roofline["exp_bound_note"] = (f"{exps_launch:.4g} exponentials per launch (every pair, masked ones "
+                                      f"included) / (148 SMs x 16 per clock x {mhz:.0f} MHz)")
     kernel_ms = {k: v[0] / args.steps for k, v in prof.items() if v[1]}
     step_flops_time = work["flops"] / (float(peaks["bf16_tflops"]) * 1e12)
     line = {
@@ -390,6 +435,8 @@ def run_gpu(args):
         "roofline": roofline,
         "kernel_ms_per_step": kernel_ms,
         "step_ms": step_stats,
+        "warm_l2": {"value": warm_tokens / warm_max_s, "ms_per_step": 1e3 * warm_max_s / n_warm, "steps": n_warm,
+                    "note": "no L2 flush between steps"},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
@@ -399,6 +446,7 @@ def run_gpu(args):
         s = oracle_sample(wl, args.cpu_sample_s)
         line["cpu_baseline"] = {
             "value": s["tokens"] / s["seconds"], "unit": "tokens/s", "cores": s["cores"], "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"{s['windows_per_layer']} evenly spaced whole windows of each layer of the pair "
                       f"({s['tokens']} layer-tokens, {s['seconds']:.1f} s), double precision",
         }
@@ -570,6 +618,95 @@ def run_backward(args):
     return 0
 
 
+def run_mlp(args):
+    """``--mlp``: the fused MLP half (vswin_mlp_forward, hidden 4C) on each layer's token
+    tensor; ``--block-full``: whole blocks, the attention half (vswin_block_msa_forward)
+    then the MLP half, per layer of the workload. One GPU; prints its own JSON line."""
+    from shifted_window_attention_sw_b200 import build as build_mod
+    from shifted_window_attention_sw_b200 import vswin
+    from shifted_window_attention_sw_b200.inputs import make_block_inputs, make_mlp_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    build_mod.build()
+    vswin.lib()
+    wl = WORKLOADS[args.workload]
+    layers = wl.layers
+    base = 1000 * wl.index
+    mlps = [make_mlp_inputs(ly.shape, 4 * ly.C, wl.dtype, "baseline", seed=base + ly.seed_offset).to(device)
+            for ly in layers]
+    blocks = ([make_block_inputs(ly.shape, ly.heads, ly.window, wl.dtype, "baseline", seed=base + ly.seed_offset,
+                                 x_seed=base).to(device) for ly in layers] if args.block_full else None)
+    outs = [torch.empty_like(m.x) for m in mlps]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    eps = 1e-5
+
+    def step():
+        for k, (ly, m, o) in enumerate(zip(layers, mlps, outs)):
+            src = m.x
+            if blocks is not None:
+                b = blocks[k]
+                li = b.layer
+                vswin.block_msa_forward(li.x, ly.window, ly.shift, b.gamma, b.beta, eps, li.Wqkv, li.bqkv,
+                                        li.Wproj, li.bproj, li.table, ly.heads, out=o, stream=stream)
+                src = o
+            vswin.mlp_forward(src, m.gamma, m.beta, eps, m.W1, m.b1, m.W2, m.b2, out=o, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    if vswin.poll_error(stream) != vswin.OK:
+        raise RuntimeError("kernel error during warm-up: " + vswin.last_error())
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = vswin.launch_count()
+    vswin.profile_enable(True)
+    sampler = ClockSampler(device)
+    sampler.start()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    vswin.profile_enable(False)
+    prof = vswin.profile_collect()
+    if vswin.poll_error(stream) != vswin.OK:
+        raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    peaks, peak_src = load_peaks()
+    tokens = sum(ly.B * ly.T * ly.H * ly.W for ly in layers)
+    mlp_flops = sum(2 * 2 * ly.B * ly.T * ly.H * ly.W * ly.C * 4 * ly.C for ly in layers)
+    mlp_bytes = sum(2 * 2 * ly.B * ly.T * ly.H * ly.W * ly.C + 2 * 2 * 4 * ly.C * ly.C for ly in layers)
+    mlp_ms, mlp_n = prof["mlp"]
+    mlp_us = 1e3 * mlp_ms / max(1, mlp_n)
+    achieved = mlp_flops / len(layers) / (mlp_us / 1e6) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    gelus = sum(ly.B * ly.T * ly.H * ly.W * 4 * ly.C for ly in layers) / len(layers)
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    what = "whole block (attention half + MLP half)" if args.block_full else "MLP half (LN, fc1, GELU, fc2, residual)"
+    line = {
+        "metric": f"{what} tokens/s, {wl.name}", "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(wl), hidden="4C", ln_eps=eps),
+        "api": "vswin_block_msa_forward + vswin_mlp_forward" if args.block_full else "vswin_mlp_forward",
+        "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+        "mlp_roofline": {"kernel": "mlp_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "avg_launch_us": mlp_us, "launches": mlp_n,
+                         "hbm_floor_us": mlp_bytes / len(layers) / (float(peaks["hbm_gbs"]) * 1e9) * 1e6,
+                         "tanh_bound_us": gelus / (SMS * MUFU_EX2_PER_CLK_SM * mhz * 1e6) * 1e6,
+                         "units_per_launch": "one layer's tokens; FLOPs 4*tok*C*hidden, hidden = 4C"},
+        "gpu_launches": int(vswin.launch_count() - launches0),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -584,15 +721,35 @@ def main(argv=None):
                     help="time the blocks' attention half (LN, layer, residual), fused and unfused, on one GPU")
     ap.add_argument("--backward", action="store_true",
                     help="time the fp32 backward of each layer of the workload on one GPU")
+    ap.add_argument("--mlp", action="store_true",
+                    help="time the fused MLP half of a block (hidden 4C) on each layer's tokens, one GPU")
+    ap.add_argument("--block-full", action="store_true",
+                    help="time whole blocks (attention half then MLP half) on the workload's layers, one GPU")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.gpus > 1 and world == 0 and not (args.block or args.backward or args.mlp or args.block_full):
+        # one process per GPU: relaunch this command under torchrun
+        import socket
+
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__),
+               *(argv if argv is not None else sys.argv[1:])]
+        os.execv(sys.executable, cmd)
+    if world and world != args.gpus:
+        ap.error(f"--gpus {args.gpus} does not match WORLD_SIZE={world}")
     if args.impl == "reference":
         return run_reference(args)
     if args.block:
         return run_block(args)
     if args.backward:
         return run_backward(args)
+    if args.mlp or args.block_full:
+        return run_mlp(args)
     return run_gpu(args)
 
 
