@@ -155,6 +155,33 @@ int vswin_block_forward(const void* x, int B, int T, int H, int W, int C, int he
                         float ln_eps, void* out, void* stream);
 
 /*
+ * bf16 patch merging between stages ("Video Swin Transformer" summary page,
+ * Method step 2: each 2x2 group of spatial neighbours, 4C values, projected
+ * to 2C by a linear layer, no temporal merging; code walk-through page,
+ * section 1.2: PatchMerging is a LayerNorm over the 4C values, then
+ * Linear(4C, 2C)):
+ *   out[b,t,i,j] = LN(cat(x[b,t,2i,2j], x[b,t,2i+1,2j], x[b,t,2i,2j+1],
+ *                         x[b,t,2i+1,2j+1])) Wr + br
+ * The pages fix neither the order of the four neighbours in the 4C vector
+ * nor odd extents: the order is the one written above (channels
+ * [(2 dw + dh) C, (2 dw + dh + 1) C) hold neighbour (dh, dw)), and an odd H
+ * or W is zero-padded at the high end.
+ * x        (B, T, H, W, C) bf16, channels last, 16-byte aligned
+ * ln_gamma, ln_beta  [4C] bf16; ln_eps finite, >= 0
+ * Wr       [4C][2C] bf16 row-major, 16-byte aligned; br [2C] bf16 or NULL
+ * out      (B, T, ceil(H/2), ceil(W/2), 2C) bf16, 16-byte aligned, must not
+ *          overlap x
+ * Requires C a multiple of 32 (else VSWIN_ERR_UNSUPPORTED). The norm is
+ * folded into the weights (bf16(diag(gamma) Wr), its fp32 column sums,
+ * beta Wr + br) and applied per row in the epilogue with fp32 statistics of
+ * the gathered bf16 values. Scratch: 16 C^2 + 16 C bytes (the folded
+ * weights), from the library's pool.
+ */
+int vswin_patch_merge_forward(const void* x, int B, int T, int H, int W, int C,
+                              const void* ln_gamma, const void* ln_beta, float ln_eps,
+                              const void* Wr, const void* br, void* out, void* stream);
+
+/*
  * fp32 layer forward (plain FP32 FMA arithmetic, no tensor cores): every
  * tensor is float. The same layer as vswin_wmsa_forward, steps 1-7 above
  * ("Video Swin Transformer" summary page, Method steps 4-6 and eq. 2), with

@@ -77,4 +77,13 @@ cudaError_t launch_mlp(const KernelCtx& ctx, long long M, int C, int hidden, con
                        const void* beta, float eps, const void* W1, const void* b1, const void* W2, const void* b2,
                        void* out, cudaStream_t st);
 
+// Patch merging (merge_path.cu): LN over each 2x2 spatial neighbourhood's 4C
+// values, then Wr [4C][2C] (+ br); scratch of patch_merge_scratch_bytes(C)
+// holds the folded weights.
+bool patch_merge_supported(int C);
+size_t patch_merge_scratch_bytes(int C);
+cudaError_t launch_patch_merge(const KernelCtx& ctx, int B, int T, int H, int W, int C, const void* x,
+                               const void* gamma, const void* beta, float eps, const void* Wr, const void* br,
+                               void* out, void* scratch, cudaStream_t st);
+
 }  // namespace vswin

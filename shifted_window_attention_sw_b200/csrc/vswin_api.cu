@@ -499,6 +499,45 @@ int vswin_block_forward(const void* x, int B, int T, int H, int W, int C, int he
   return VSWIN_OK;
 }
 
+int vswin_patch_merge_forward(const void* x, int B, int T, int H, int W, int C, const void* ln_gamma,
+                              const void* ln_beta, float ln_eps, const void* Wr, const void* br, void* out,
+                              void* stream) {
+  if (B <= 0 || T <= 0 || H <= 0 || W <= 0 || C <= 0)
+    return fail(VSWIN_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d H=%d W=%d C=%d)", B, T, H, W, C);
+  const void* ptrs[] = {x, ln_gamma, ln_beta, Wr, out};
+  const char* names[] = {"x", "ln_gamma", "ln_beta", "Wr", "out"};
+  for (int k = 0; k < 5; ++k)
+    if (!ptrs[k]) return fail(VSWIN_ERR_INVALID_ARG, "%s is NULL", names[k]);
+  const void* big[] = {x, Wr, out};
+  const char* bign[] = {"x", "Wr", "out"};
+  for (int k = 0; k < 3; ++k)
+    if (!aligned(big[k], 16)) return fail(VSWIN_ERR_INVALID_ARG, "%s is not 16-byte aligned", bign[k]);
+  if (!aligned(ln_gamma, 2) || !aligned(ln_beta, 2) || (br && !aligned(br, 2)))
+    return fail(VSWIN_ERR_INVALID_ARG, "ln_gamma, ln_beta and br must be 2-byte aligned");
+  if (!(ln_eps >= 0.f) || !std::isfinite(ln_eps))
+    return fail(VSWIN_ERR_INVALID_ARG, "ln_eps must be finite and >= 0 (got %g)", (double)ln_eps);
+  const long long tokens = (long long)B * T * H * W;
+  const long long merged = (long long)B * T * ((H + 1) / 2) * ((W + 1) / 2);
+  if (tokens > (1LL << 40) || merged / 128 > (1LL << 30))
+    return fail(VSWIN_ERR_UNSUPPORTED, "input too large (%lld tokens)", tokens);
+  if (overlap(x, (size_t)tokens * C * 2, out, (size_t)merged * 2 * C * 2))
+    return fail(VSWIN_ERR_INVALID_ARG, "x and out overlap");
+  if (!patch_merge_supported(C))
+    return fail(VSWIN_ERR_UNSUPPORTED, "patch merging needs C a multiple of 32 (C=%d)", C);
+  KernelCtx ctx;
+  int st = make_ctx(&ctx);
+  if (st != VSWIN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  st = scratch_alloc(&scratch, patch_merge_scratch_bytes(C), s);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = launch_patch_merge(ctx, B, T, H, W, C, x, ln_gamma, ln_beta, ln_eps, Wr, br, out, scratch, s);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) return fail_cuda(e, "patch merging launch");
+  if (e2 != cudaSuccess) return fail_cuda(e2, "cudaFreeAsync");
+  return VSWIN_OK;
+}
+
 int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
                            const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                            const void* bproj, const void* bias_table, void* out, void* stream) {

@@ -21,6 +21,10 @@ MLP-half inputs (layer norm + two linear layers with GELU + residual), seeds
 k = 10..16: x ~ N(0, 1) plus a per-token offset ~ N(0, 0.5); gamma ~ 1 + N(0, 0.1),
 beta ~ N(0, 0.1); "baseline" W1, W2 ~ N(0, 0.02) and biases 0; "sensitivity"
 W1 ~ N(0, 1/C), W2 ~ N(0, 1/hidden), biases ~ N(0, 0.1).
+
+Patch-merging inputs, seeds k = 20..24: x as for the MLP half; gamma ~ 1 + N(0, 0.1),
+beta ~ N(0, 0.1) over 4C; "baseline" Wr ~ N(0, 0.02), no bias; "sensitivity"
+Wr ~ N(0, 1/(4C)), br ~ N(0, 0.1).
 """
 
 from __future__ import annotations
@@ -161,3 +165,39 @@ def make_mlp_inputs(shape, hidden, dtype="bf16", scale="baseline", seed=1000) ->
     b1 = _randn((hidden,), seed + 16, b_std) if b_std else torch.zeros(hidden)
     b2 = _randn((C,), seed + 17, b_std) if b_std else torch.zeros(C)
     return MlpInputs(*(t.to(dt).contiguous() for t in (x, gamma, beta, W1, b1, W2, b2)))
+
+
+@dataclass
+class MergeInputs:
+    x: torch.Tensor
+    gamma: torch.Tensor
+    beta: torch.Tensor
+    Wr: torch.Tensor
+    br: object  # torch.Tensor or None
+
+    def as_f64(self):
+        d = {k: getattr(self, k).to(torch.float64).numpy() for k in ("x", "gamma", "beta", "Wr")}
+        d["br"] = None if self.br is None else self.br.to(torch.float64).numpy()
+        return d
+
+    def to(self, device):
+        return MergeInputs(self.x.to(device), self.gamma.to(device), self.beta.to(device), self.Wr.to(device),
+                           None if self.br is None else self.br.to(device))
+
+
+def make_merge_inputs(shape, dtype="bf16", scale="baseline", seed=1000) -> MergeInputs:
+    """Inputs for one patch-merging call. ``shape`` = (B, T, H, W, C)."""
+    B, T, H, W, C = shape
+    dt = _DT[dtype]
+    if scale == "baseline":
+        w_std, b_std = 0.02, 0.0
+    elif scale == "sensitivity":
+        w_std, b_std = 1.0 / np.sqrt(4 * C), 0.1
+    else:
+        raise ValueError(scale)
+    x = _randn((B, T, H, W, C), seed + 20, 1.0) + _randn((B, T, H, W, 1), seed + 21, 0.5)
+    gamma = 1.0 + _randn((4 * C,), seed + 22, 0.1)
+    beta = _randn((4 * C,), seed + 23, 0.1)
+    Wr = _randn((4 * C, 2 * C), seed + 24, w_std)
+    br = _randn((2 * C,), seed + 25, b_std).to(dt).contiguous() if b_std else None
+    return MergeInputs(*(t.to(dt).contiguous() for t in (x, gamma, beta, Wr)), br)

@@ -38,6 +38,7 @@ EXPORTS = (
     "vswin_wmsa_backward_f32",
     "vswin_mlp_forward",
     "vswin_block_forward",
+    "vswin_patch_merge_forward",
 )
 
 KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other", "mlp")
@@ -79,6 +80,8 @@ def lib():
         L.vswin_block_forward.argtypes = (layer[:9] + [_P, _P] + [_P] * 5 + [_P, _P, _I] + [_P] * 4 +
                                           [ctypes.c_float, _P, _P])
         L.vswin_block_forward.restype = _I
+        L.vswin_patch_merge_forward.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P]
+        L.vswin_patch_merge_forward.restype = _I
         L.vswin_wmsa_index_maps.argtypes = [_I, _I, _I, _I, _IP, _IP, _P, _P, _P, _P]
         L.vswin_wmsa_index_maps.restype = _I
         L.vswin_clamp_window.argtypes = [_I, _I, _I, _IP, _IP, _IP, _IP]
@@ -264,6 +267,31 @@ def block_forward(x, window, shift, attn, mlp, heads, eps=1e-5, out=None, stream
             _ptr(attn["Wqkv"]), _ptr(attn["bqkv"]), _ptr(attn["Wproj"]), _ptr(attn["bproj"]), _ptr(attn["table"]),
             _ptr(mlp["gamma"]), _ptr(mlp["beta"]), int(hidden), _ptr(mlp["W1"]), _ptr(mlp["b1"]), _ptr(mlp["W2"]),
             _ptr(mlp["b2"]), float(eps), _ptr(out), _stream_handle(stream, x.device)))
+    return out
+
+
+def patch_merge_forward(x, gamma, beta, eps, Wr, br=None, out=None, stream=None):
+    """bf16 patch merging: LN over each 2x2 spatial neighbourhood's 4C values, then
+    Wr [4C][2C] (+ br). x (B, T, H, W, C) -> (B, T, ceil(H/2), ceil(W/2), 2C)."""
+    if x.dim() != 5:
+        raise ValueError(f"x must be (B, T, H, W, C), got shape {tuple(x.shape)}")
+    B, T, H, W, C = x.shape
+    oshape = (B, T, (H + 1) // 2, (W + 1) // 2, 2 * C)
+    if out is None:
+        out = torch.empty(oshape, dtype=x.dtype, device=x.device)
+    tensors = dict(x=x, gamma=gamma, beta=beta, Wr=Wr, out=out)
+    if br is not None:
+        tensors["br"] = br
+    _prep(x, tensors, torch.bfloat16, x.device)
+    want = {"gamma": (gamma, (4 * C,)), "beta": (beta, (4 * C,)), "Wr": (Wr, (4 * C, 2 * C)), "out": (out, oshape)}
+    if br is not None:
+        want["br"] = (br, (2 * C,))
+    for name, (t, shape) in want.items():
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    with torch.cuda.device(x.device):
+        _check(lib().vswin_patch_merge_forward(_ptr(x), B, T, H, W, C, _ptr(gamma), _ptr(beta), float(eps),
+                                               _ptr(Wr), _ptr(br), _ptr(out), _stream_handle(stream, x.device)))
     return out
 
 

@@ -336,3 +336,29 @@ def test_whole_block_checks_both_halves_before_launching(L):
                                    p(10), hidden, W1, p(21), p(22), p(23), ctypes.c_float(1e-5), p(1), None)
         assert rc in (vswin.ERR_INVALID_ARG, vswin.ERR_UNSUPPORTED), (rc, vswin.last_error())
     assert vswin.launch_count() == before
+
+
+def _call_merge(L, x=A16, B=1, T=8, H=14, W=14, C=96, gamma=A16 * 7, beta=A16 * 8, eps=1e-5, Wr=A16 * 2,
+                br=A16 * 3, out=A16 * 64):
+    p = lambda v: ctypes.c_void_p(v) if v else None  # noqa: E731
+    return L.vswin_patch_merge_forward(p(x), B, T, H, W, C, p(gamma), p(beta), ctypes.c_float(eps), p(Wr), p(br),
+                                       p(out), None)
+
+
+@pytest.mark.parametrize(
+    "kw",
+    [dict(B=0), dict(W=-2), dict(C=0), dict(x=0), dict(out=0), dict(Wr=0), dict(gamma=0), dict(beta=0),
+     dict(Wr=A16 * 2 + 4), dict(out=A16 * 64 + 2), dict(br=A16 * 3 + 1), dict(eps=float("inf")),
+     dict(out=A16 + 128)],          # overlaps x
+)
+def test_patch_merge_invalid_arguments_launch_nothing(L, kw):
+    before = vswin.launch_count()
+    rc = _call_merge(L, **kw)
+    assert rc == vswin.ERR_INVALID_ARG, (rc, vswin.last_error())
+    assert vswin.launch_count() == before
+
+
+def test_patch_merge_unsupported_width(L):
+    before = vswin.launch_count()
+    assert _call_merge(L, C=48) == vswin.ERR_UNSUPPORTED
+    assert vswin.launch_count() == before
