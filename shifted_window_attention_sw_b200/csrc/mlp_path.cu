@@ -111,6 +111,7 @@ struct MlpArgs {
   int C, hidden, hc, nch, stages;
   bool resident;  // every weight chunk has its own stage (loaded once per CTA)
   float eps;
+  const __nv_bfloat16* x;  // the residual is read back from here
   const __nv_bfloat16* gamma;
   const __nv_bfloat16* beta;
   const __nv_bfloat16* b1;
@@ -120,15 +121,14 @@ struct MlpArgs {
 
 // Shared-memory plan (bytes from the dynamically allocated base).
 struct MlpSmem {
-  int x0, x1, xn, w, wstage, w2off, gam, bet, b1, b2, bars, total;
+  int x0, x1, w, wstage, w2off, gam, bet, b1, b2, bars, total;
 };
 __host__ __device__ inline MlpSmem mlp_smem(int C, int hidden, int hc, int stages) {
   MlpSmem s;
   const int xb = 128 * C * 2;
   s.x0 = 0;
   s.x1 = xb;
-  s.xn = 2 * xb;
-  s.w = 3 * xb;
+  s.w = 2 * xb;
   s.w2off = C * hc * 2;  // W2 chunk after the W1 chunk inside a stage
   s.wstage = 2 * C * hc * 2;
   s.gam = s.w + stages * s.wstage;
@@ -136,8 +136,29 @@ __host__ __device__ inline MlpSmem mlp_smem(int C, int hidden, int hc, int stage
   s.b1 = s.bet + C * 4;
   s.b2 = s.b1 + hidden * 4;
   s.bars = (s.b2 + C * 4 + 15) / 16 * 16;
-  s.total = s.bars + 32 * 8 + 16;
+  s.total = s.bars + 40 * 8 + 16;
   return s;
+}
+
+// Byte offset of 16-byte chunk `k` (channels 8k .. 8k+7) of row r in a tile
+// stored K-major with the 64-byte swizzle: blocks of 32 channels (8 KB each:
+// 128 rows x 64 B), and inside a row the chunk index XORed with bits 1-2 of
+// the row -- what a TMA box with CU_TENSOR_MAP_SWIZZLE_64B writes and what a
+// tcgen05 descriptor of layout type SWIZZLE_64B (SBO = 512 B) reads.
+__device__ __forceinline__ int sw64_chunk(int r, int k) {
+  return (k >> 2) * 8192 + r * 64 + (((k & 3) ^ ((r >> 1) & 3)) << 4);
+}
+
+// K-major, 64-byte swizzle descriptor: LBO 16 B (unused inside one swizzle
+// atom), SBO 512 B (8 rows x 64 B), layout type 4.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
 }
 
 __global__ void __launch_bounds__(kMlpThreads, 1)
@@ -147,23 +168,22 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   const int C = a.C, NCH = a.nch, S = a.stages, HC = a.hc;
   const MlpSmem L = mlp_smem(C, a.hidden, HC, S);
   uint8_t* sX[2] = {smem + L.x0, smem + L.x1};
-  uint8_t* sXn = smem + L.xn;
   float* sGam = reinterpret_cast<float*>(smem + L.gam);
   float* sBet = reinterpret_cast<float*>(smem + L.bet);
   float* sB1 = reinterpret_cast<float*>(smem + L.b1);
   float* sB2 = reinterpret_cast<float*>(smem + L.b2);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* x_full = bars;         // [2] x tile landed
-  uint64_t* x_free = bars + 2;     // [2] x buffer's output store has read it
-  uint64_t* xn_full = bars + 4;    // normalised tile written (4 warps)
-  uint64_t* xn_free = bars + 5;    // the tile's fc1 MMAs have read it
-  uint64_t* acc1_full = bars + 6;  // [2]
-  uint64_t* h_full = bars + 8;     // [2] h written over the fc1 accumulator (8 warps)
-  uint64_t* acc2_full = bars + 10; // [2]
-  uint64_t* acc2_free = bars + 12; // [2] (8 warps)
-  uint64_t* w_full = bars + 14;    // [S <= 8]
-  uint64_t* w_free = bars + 22;    // [S <= 8]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 30);
+  uint64_t* x_full = bars;          // [2] x tile landed
+  uint64_t* xn_full = bars + 2;     // [2] tile normalised in place (4 warps)
+  uint64_t* xn_free = bars + 4;     // [2] the tile's fc1 MMAs have read it
+  uint64_t* out_full = bars + 6;    // [2] output staged over the tile (8 warps)
+  uint64_t* acc1_full = bars + 8;   // [2]
+  uint64_t* h_full = bars + 10;     // [2] h written over the fc1 accumulator (8 warps)
+  uint64_t* acc2_full = bars + 12;  // [2]
+  uint64_t* acc2_free = bars + 14;  // [2] (8 warps)
+  uint64_t* w_full = bars + 16;     // [S <= 8]
+  uint64_t* w_free = bars + 24;     // [S <= 8]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 32);
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -176,14 +196,14 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   if (tid == 0) {
     for (int k = 0; k < 2; ++k) {
       mbar_init(&x_full[k], 1);
-      mbar_init(&x_free[k], 1);
+      mbar_init(&xn_full[k], 4);
+      mbar_init(&xn_free[k], 1);
+      mbar_init(&out_full[k], 8);
       mbar_init(&acc1_full[k], 1);
       mbar_init(&h_full[k], 8);
       mbar_init(&acc2_full[k], 1);
       mbar_init(&acc2_free[k], 8);
     }
-    mbar_init(xn_full, 4);
-    mbar_init(xn_free, 1);
     for (int k = 0; k < S; ++k) {
       mbar_init(&w_full[k], 1);
       mbar_init(&w_free[k], 1);
@@ -205,23 +225,32 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  // TMEM columns: fc1 accumulators [0, 128) and [128, 256); output
+  // TMEM columns: fc1 accumulators [0, HC) and [HC, 2 HC) (2 HC <= 256); output
   // accumulators [256, 256 + C) and [256 + C, 256 + 2C).
   const uint32_t tAcc1 = tmem, tAcc2 = tmem + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Per tile t: store the output of tile t - 2 from buffer t & 1 (once the
+    // epilogue has staged it there), then load x of tile t into that buffer and
+    // the weight chunks tile t needs.
     if (lane == 0) {
       long long g = 0;  // global chunk counter
-      for (long long t = 0; t < ntiles && !s_abort; ++t) {
-        const long long m = blockIdx.x + t * gridDim.x;
+      for (long long t = 0; t < ntiles + 2 && !s_abort; ++t) {
         const int xb = (int)(t & 1);
-        if (t >= 2 && !mbar_wait(&x_free[xb], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim)) {
-          s_abort = 1;
-          break;
+        if (t >= 2) {
+          const long long ts = t - 2;
+          if (!mbar_wait(&out_full[xb], (uint32_t)(ts >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) {
+            s_abort = 1;
+            break;
+          }
+          tma_store_3d(&tm_out, sX[xb], 0, (int)((blockIdx.x + ts * gridDim.x) * 128), 0);
+          bulk_commit();
+          bulk_wait_read0();  // the buffer may be overwritten once the store has read it
         }
+        if (t >= ntiles) continue;
         mbar_arrive_expect_tx(&x_full[xb], xbytes);
-        tma_load_3d(sX[xb], &tm_x, 0, (int)(m * 128), 0, &x_full[xb]);
+        tma_load_3d(sX[xb], &tm_x, 0, (int)((blockIdx.x + t * gridDim.x) * 128), 0, &x_full[xb]);
         for (int c = 0; c < NCH; ++c, ++g) {
           if (a.resident && t > 0) continue;
           const int s = (int)(g % S);
@@ -235,16 +264,16 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           tma_load_4d(dst + L.w2off, &tm_w2, 0, 0, 0, c * (HC / 8), &w_full[s]);
         }
       }
+      bulk_wait0();  // every store has completed before the CTA ends
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t id1 = idesc_bf16(128, HC, 0, 1);  // A K-major (x), B MN-major (W1)
-      const uint32_t id2 = idesc_bf16(128, C, 0, 1);       // A from TMEM (h), B MN-major (W2)
-      const uint32_t lbo1 = (uint32_t)(HC / 8) * 128u;  // W1 chunk: K-group stride
-      const uint32_t lbo2 = (uint32_t)(C / 8) * 128u;       // W2 chunk: K-group stride
-      const uint32_t xn_addr = smem_u32(sXn);
+      const uint32_t id2 = idesc_bf16(128, C, 0, 1);   // A from TMEM (h), B MN-major (W2)
+      const uint32_t lbo1 = (uint32_t)(HC / 8) * 128u; // W1 chunk: K-group stride
+      const uint32_t lbo2 = (uint32_t)(C / 8) * 128u;  // W2 chunk: K-group stride
       const long long total = ntiles * NCH;
       auto stage_of = [&](long long g) -> int { return a.resident ? (int)(g % NCH) : (int)(g % S); };
       auto w_phase = [&](long long g) -> uint32_t { return a.resident ? 0u : (uint32_t)(g / S) & 1; };
@@ -253,18 +282,22 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       auto fc1 = [&](long long g) {
         const long long t = g / NCH;
         const int c = (int)(g % NCH);
-        if (c == 0 && !s_abort && !mbar_wait(xn_full, (uint32_t)t & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        const int xb = (int)(t & 1);
+        if (c == 0 && !s_abort && !mbar_wait(&xn_full[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim))
+          s_abort = 1;
         const int s = stage_of(g);
         if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
         tc_fence_after();
         if (s_abort) return;
+        const uint32_t xa = smem_u32(sX[xb]);
         const uint32_t wa = smem_u32(smem + L.w + s * L.wstage);
         const uint32_t d = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
+        // K step ks covers channels [16 ks, 16 ks + 16): block ks / 2, 32 B in
         for (int ks = 0; ks < C / 16; ++ks)
-          umma_ss(d, smem_desc(xn_addr + ks * 2 * 2048, 2048, 128), smem_desc(wa + ks * 2 * lbo1, lbo1, 128), id1,
-                  ks > 0);
+          umma_ss(d, smem_desc_sw64(xa + (ks >> 1) * 8192 + (ks & 1) * 32), smem_desc(wa + ks * 2 * lbo1, lbo1, 128),
+                  id1, ks > 0);
         umma_commit(&acc1_full[g & 1]);
-        if (c == NCH - 1) umma_commit(xn_free);
+        if (c == NCH - 1) umma_commit(&xn_free[xb]);
       };
       if (total > 0) fc1(0);
       if (total > 1) fc1(1);
@@ -299,25 +332,23 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue warps
-    const int q = warp & 3;               // TMEM lane quarter
-    const int hf = (warp - kMlpEpi0) >> 2; // 0: warps 2-5, 1: warps 6-9
-    const int r = q * 32 + lane;          // this thread's row of the tile
+    const int q = warp & 3;                 // TMEM lane quarter
+    const int hf = (warp - kMlpEpi0) >> 2;  // 0: warps 2-5, 1: warps 6-9
+    const int r = q * 32 + lane;            // this thread's row of the tile
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool norm_warp = hf == 0;
-    // Normalise tile t (norm warps): row r of sX[t & 1] -> sXn.
+    // Normalise tile t in place (norm warps): row r of sX[t & 1].
     auto normalise = [&](long long t) {
       const int xb = (int)(t & 1);
       if (!s_abort && !mbar_wait(&x_full[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
-      if (t >= 1 && !s_abort && !mbar_wait(xn_free, (uint32_t)(t - 1) & 1, a.ctx.err, kErrWaitMma, lim))
-        s_abort = 1;
       if (!s_abort) {
-        const uint8_t* src = sX[xb] + r * 16;
+        uint8_t* row = sX[xb];
         uint4 v[kMlpMaxC / 8];
         float sum = 0.f;
 #pragma unroll
         for (int k = 0; k < kMlpMaxC / 8; ++k) {
           if (k < C / 8) {
-            v[k] = *reinterpret_cast<const uint4*>(src + k * 2048);
+            v[k] = *reinterpret_cast<const uint4*>(row + sw64_chunk(r, k));
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -341,7 +372,6 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           }
         }
         const float rstd = 1.0f / sqrtf(ss / (float)C + a.eps);
-        uint8_t* dst = sXn + r * 16;
 #pragma unroll
         for (int k = 0; k < kMlpMaxC / 8; ++k) {
           if (k < C / 8) {
@@ -354,13 +384,13 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
               w[e] = pack2(fmaf((f.x - mean) * rstd, sGam[ch], sBet[ch]),
                            fmaf((f.y - mean) * rstd, sGam[ch + 1], sBet[ch + 1]));
             }
-            *reinterpret_cast<uint4*>(dst + k * 2048) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(row + sw64_chunk(r, k)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
       fence_proxy_async_smem();  // generic writes -> tensor-core operand reads
       __syncwarp();
-      if (lane == 0) mbar_arrive_cta(xn_full);
+      if (lane == 0) mbar_arrive_cta(&xn_full[xb]);
     };
     // GELU of chunk g: this warp's HC/2 fc1 columns (half hf of the chunk) ->
     // HC/4 columns of bf16 pairs over the first half of the same columns.
@@ -391,16 +421,21 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cta(&h_full[g & 1]);
     };
-    // Output of tile t: acc2 + b2 + x -> bf16 over x in shared memory, then one
-    // thread stores the tile with TMA and releases the x buffer.
+    // Output of tile t: acc2 + b2 + x (re-read from global memory: the tile's
+    // buffer holds the normalised tokens) -> bf16 over the tile's buffer, then
+    // the producer stores it with TMA.
     auto finish_tile = [&](long long t) {
       const int xb = (int)(t & 1), ob = (int)(t & 1);
       if (!s_abort && !mbar_wait(&acc2_full[ob], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      if (!s_abort && !mbar_wait(&xn_free[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
       tc_fence_after();
       if (!s_abort) {
         const int half = C / 2;  // a multiple of 16
         const uint32_t ta = tAcc2 + lane_base + (uint32_t)ob * (uint32_t)C + (uint32_t)(hf * half);
-        uint8_t* row = sX[xb] + r * 16;
+        const long long grow = (blockIdx.x + t * gridDim.x) * 128 + r;
+        const bool real = grow < a.M;
+        const __nv_bfloat16* xrow = a.x + (real ? grow : 0) * C;
+        uint8_t* buf = sX[xb];
         for (int c0 = 0; c0 < half; c0 += 16) {
           uint32_t u[16];
           tmem_ld16(ta + c0, u);
@@ -408,47 +443,41 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int ch = hf * half + c0 + 8 * k;  // first channel of this 8-channel group
-            uint4* p = reinterpret_cast<uint4*>(row + (ch >> 3) * 2048);
-            const uint4 xv = *p;
+            const uint4 xv = real ? *reinterpret_cast<const uint4*>(xrow + ch) : make_uint4(0, 0, 0, 0);
             const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 xf = __bfloat1622float2(x2[e]);
               const float2 bb = *reinterpret_cast<const float2*>(sB2 + ch + 2 * e);
-              float2 v = __fadd2_rn(make_float2(__uint_as_float(u[8 * k + 2 * e]), __uint_as_float(u[8 * k + 2 * e + 1])),
-                                    bb);
+              float2 v = __fadd2_rn(
+                  make_float2(__uint_as_float(u[8 * k + 2 * e]), __uint_as_float(u[8 * k + 2 * e + 1])), bb);
               v = __fadd2_rn(v, xf);
               w[e] = pack2(v.x, v.y);
             }
-            *p = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(buf + sw64_chunk(r, ch >> 3)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
       tc_fence_before();
+      fence_proxy_async_smem();  // staged rows -> the producer's TMA store
       __syncwarp();
-      if (lane == 0) mbar_arrive_cta(&acc2_free[ob]);
-      fence_proxy_async_smem();  // staged rows -> TMA store
-      named_sync(1, 8 * 32);
-      if (warp == kMlpEpi0 && lane == 0) {
-        if (!s_abort) {
-          const long long m = blockIdx.x + t * gridDim.x;
-          tma_store_3d(&tm_out, sX[xb], 0, (int)(m * 128), 0);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        mbar_arrive_cta(&x_free[xb]);
+      if (lane == 0) {
+        mbar_arrive_cta(&acc2_free[ob]);
+        mbar_arrive_cta(&out_full[xb]);
       }
     };
 
     long long g = 0;
     if (norm_warp && ntiles > 0) normalise(0);
     for (long long t = 0; t < ntiles; ++t) {
-      for (int c = 0; c < NCH; ++c, ++g) gelu_chunk(g);
-      if (norm_warp && t + 1 < ntiles) normalise(t + 1);
+      for (int c = 0; c < NCH; ++c, ++g) {
+        gelu_chunk(g);
+        // the next tile is normalised early so that its first fc1 never waits
+        if (c == 0 && norm_warp && t + 1 < ntiles) normalise(t + 1);
+      }
       finish_tile(t);
     }
-    if (warp == kMlpEpi0 && lane == 0) bulk_wait0();  // the last stores have completed
   }
   tc_fence_before();
   __syncthreads();
@@ -475,12 +504,12 @@ EncodeTiledFn encode_fn() {
 // bf16 tensor map of `rank` dims (dims[0] innermost), strides in bytes for
 // dims 1.., box sizes per dim; no swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-              const cuuint32_t* box) {
+              const cuuint32_t* box, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -516,11 +545,11 @@ cudaError_t launch_mlp(const KernelCtx& ctx, long long M, int C, int hidden, con
   const MlpPlan plan = mlp_plan(C, hidden);
   const int S = plan.stages, HC = plan.hc;
   CUtensorMap mx, mo, m1, m2;
-  // x / out as (8 channels, M rows, C/8 groups): one box is a 128-row tile in
-  // the K-major operand layout
-  const cuuint64_t xd[3] = {8, (cuuint64_t)M, (cuuint64_t)(C / 8)};
-  const cuuint64_t xs[2] = {(cuuint64_t)C * 2, 16};
-  const cuuint32_t xbox[3] = {8, 128, (cuuint32_t)(C / 8)};
+  // x / out as (32 channels, M rows, C/32 blocks) with the 64-byte swizzle: one
+  // box is a 128-row tile in the K-major SWIZZLE_64B operand layout
+  const cuuint64_t xd[3] = {32, (cuuint64_t)M, (cuuint64_t)(C / 32)};
+  const cuuint64_t xs[2] = {(cuuint64_t)C * 2, 64};
+  const cuuint32_t xbox[3] = {32, 128, (cuuint32_t)(C / 32)};
   // W1 [C][hidden] as (8 n, 8 k, hidden/8 n-groups, C/8 k-groups); box = one
   // hidden chunk, all of K
   const cuuint64_t w1d[4] = {8, 8, (cuuint64_t)(hidden / 8), (cuuint64_t)(C / 8)};
@@ -531,7 +560,8 @@ cudaError_t launch_mlp(const KernelCtx& ctx, long long M, int C, int hidden, con
   const cuuint64_t w2d[4] = {8, 8, (cuuint64_t)(C / 8), (cuuint64_t)(hidden / 8)};
   const cuuint64_t w2s[3] = {(cuuint64_t)C * 2, 16, (cuuint64_t)C * 16};
   const cuuint32_t w2box[4] = {8, 8, (cuuint32_t)(C / 8), (cuuint32_t)(HC / 8)};
-  if (!make_map(&mx, x, 3, xd, xs, xbox) || !make_map(&mo, out, 3, xd, xs, xbox) ||
+  if (!make_map(&mx, x, 3, xd, xs, xbox, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&mo, out, 3, xd, xs, xbox, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map(&m1, W1, 4, w1d, w1s, w1box) || !make_map(&m2, W2, 4, w2d, w2s, w2box))
     return cudaErrorInvalidValue;
   MlpArgs a;
@@ -543,6 +573,7 @@ cudaError_t launch_mlp(const KernelCtx& ctx, long long M, int C, int hidden, con
   a.stages = S;
   a.resident = S == a.nch;
   a.eps = eps;
+  a.x = static_cast<const __nv_bfloat16*>(x);
   a.gamma = static_cast<const __nv_bfloat16*>(gamma);
   a.beta = static_cast<const __nv_bfloat16*>(beta);
   a.b1 = static_cast<const __nv_bfloat16*>(b1);
