@@ -7,19 +7,20 @@
 // One CTA per SM walks 128-token tiles. Per tile the tokens are read from HBM
 // once (TMA) and the result is written once (TMA store); the hidden
 // activations (128 x hidden) never leave the SM:
-//   * warp 0 loads x tiles (double-buffered) and the weight chunks (W1
-//     columns and W2 rows of one hidden chunk of HC = 128) with TMA; when
-//     every chunk fits in shared memory at once they are loaded once per CTA;
-//   * warps 2-5 normalise the tile in shared memory (fp32 statistics, bf16
-//     result in the MMA operand layout);
+//   * warp 0 loads x tiles (three in flight) and the weight chunks (W1
+//     columns and W2 rows of one hidden chunk of HC = 128 or 64 columns) with
+//     TMA -- when every chunk fits in shared memory at once they are loaded
+//     once per CTA -- and stores each finished output tile with TMA;
 //   * warp 1 issues, per hidden chunk, fc1 = LN(x) W1[:, chunk] into one of
 //     two TMEM accumulators, and fc2 += h_chunk W2[chunk, :] with h read
 //     from TMEM (the A operand of a TS MMA) into one of two output
 //     accumulators;
-//   * warps 2-9 turn each fc1 accumulator into h = GELU(acc + b1) (bf16,
-//     written over the accumulator's own columns), and at the end of a tile
-//     add b2 and the residual to the output accumulator, stage the bf16
-//     result over the tile's x in shared memory and store it with TMA.
+//   * warps 2-5 normalise each tile in place as soon as it lands (fp32
+//     statistics, bf16 result in the MMA operand layout) and write each
+//     tile's output: output accumulator + b2 + x (re-read from global memory,
+//     L1-prefetched before the wait), bf16, staged over the tile's buffer;
+//   * warps 6-13 turn each fc1 accumulator into h = GELU(acc + b1) (bf16,
+//     written over the accumulator's own columns).
 //
 // GELU: the erf form x * Phi(x) (torch.nn.GELU's default) evaluated as
 // 0.5 x (1 + tanh(x (g1 + g3 x^2 + g5 x^4))) with x^2 clamped at 64, whose
@@ -28,12 +29,14 @@
 // tanh.approx.f32 (max relative error about 2^-11), so the GELU value carries
 // an absolute error below 1e-3 * |x|, under the bf16 rounding of h.
 //
-// Operand layouts in shared memory: the no-swizzle canonical layout (8-row x
-// 16-byte core matrices). A tile of x (128 rows x C) is stored as C/8 column
-// groups of 128 rows x 16 bytes (LBO = 2048 B along K, SBO = 128 B along M),
-// which is what one 3D TMA box (8 channels, 128 rows, C/8 groups) writes.
-// Weight chunks are MN-major: element (k, n) at (k/8)*LBO + (n/8)*128 +
-// (k%8)*16 + (n%8)*2, one 4D TMA box each.
+// Operand layouts in shared memory. A tile of x (128 rows x C) is K-major
+// with the 64-byte swizzle: blocks of 32 channels, 64-byte rows, the 16-byte
+// chunk index XORed with bits 1-2 of the row (one 3D TMA box of (32
+// channels, 128 rows, C/32 blocks) with CU_TENSOR_MAP_SWIZZLE_64B writes it;
+// the MMA descriptor uses layout type SWIZZLE_64B, SBO = 512 B). Weight
+// chunks are MN-major in the no-swizzle canonical layout (8 x 16-byte core
+// matrices): element (k, n) at (k/8)*LBO + (n/8)*128 + (k%8)*16 + (n%8)*2,
+// one 4D TMA box each.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -44,8 +47,10 @@ namespace vswin {
 namespace {
 
 constexpr int kMlpMaxHC = 128;       // hidden columns per chunk: 128, or 64 when two 128-column stages do not fit
-constexpr int kMlpThreads = 10 * 32;  // producer, MMA, 8 epilogue warps
-constexpr int kMlpEpi0 = 2;           // first epilogue warp
+constexpr int kMlpThreads = 14 * 32;  // producer, MMA, 4 norm / output warps, 8 GELU warps
+constexpr int kMlpNorm0 = 2;          // first norm / output warp
+constexpr int kMlpGelu0 = 6;          // first GELU warp
+constexpr int kMlpXBufs = 3;          // x tiles in flight
 constexpr int kMlpMaxC = 128;
 
 // GELU via tanh: coefficients of x (g1 + g3 x^2 + g5 x^4), least-squares fit
@@ -104,7 +109,6 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 __device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 struct MlpArgs {
   long long M;  // tokens (rows)
@@ -121,14 +125,13 @@ struct MlpArgs {
 
 // Shared-memory plan (bytes from the dynamically allocated base).
 struct MlpSmem {
-  int x0, x1, w, wstage, w2off, gam, bet, b1, b2, bars, total;
+  int x, w, wstage, w2off, gam, bet, b1, b2, bars, total;
 };
 __host__ __device__ inline MlpSmem mlp_smem(int C, int hidden, int hc, int stages) {
   MlpSmem s;
   const int xb = 128 * C * 2;
-  s.x0 = 0;
-  s.x1 = xb;
-  s.w = 2 * xb;
+  s.x = 0;  // kMlpXBufs tiles
+  s.w = kMlpXBufs * xb;
   s.w2off = C * hc * 2;  // W2 chunk after the W1 chunk inside a stage
   s.wstage = 2 * C * hc * 2;
   s.gam = s.w + stages * s.wstage;
@@ -136,7 +139,7 @@ __host__ __device__ inline MlpSmem mlp_smem(int C, int hidden, int hc, int stage
   s.b1 = s.bet + C * 4;
   s.b2 = s.b1 + hidden * 4;
   s.bars = (s.b2 + C * 4 + 15) / 16 * 16;
-  s.total = s.bars + 40 * 8 + 16;
+  s.total = s.bars + 48 * 8 + 16;
   return s;
 }
 
@@ -167,23 +170,24 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int C = a.C, NCH = a.nch, S = a.stages, HC = a.hc;
   const MlpSmem L = mlp_smem(C, a.hidden, HC, S);
-  uint8_t* sX[2] = {smem + L.x0, smem + L.x1};
+  const int xbytes_tile = 128 * C * 2;
+  auto sX = [&](int b) { return smem + L.x + b * xbytes_tile; };
   float* sGam = reinterpret_cast<float*>(smem + L.gam);
   float* sBet = reinterpret_cast<float*>(smem + L.bet);
   float* sB1 = reinterpret_cast<float*>(smem + L.b1);
   float* sB2 = reinterpret_cast<float*>(smem + L.b2);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* x_full = bars;          // [2] x tile landed
-  uint64_t* xn_full = bars + 2;     // [2] tile normalised in place (4 warps)
-  uint64_t* xn_free = bars + 4;     // [2] the tile's fc1 MMAs have read it
-  uint64_t* out_full = bars + 6;    // [2] output staged over the tile (8 warps)
-  uint64_t* acc1_full = bars + 8;   // [2]
-  uint64_t* h_full = bars + 10;     // [2] h written over the fc1 accumulator (8 warps)
-  uint64_t* acc2_full = bars + 12;  // [2]
-  uint64_t* acc2_free = bars + 14;  // [2] (8 warps)
-  uint64_t* w_full = bars + 16;     // [S <= 8]
-  uint64_t* w_free = bars + 24;     // [S <= 8]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 32);
+  uint64_t* x_full = bars;          // [3] x tile landed
+  uint64_t* xn_full = bars + 3;     // [3] tile normalised in place (4 norm warps)
+  uint64_t* xn_free = bars + 6;     // [3] the tile's fc1 MMAs have read it
+  uint64_t* out_full = bars + 9;    // [3] output staged over the tile (4 output warps)
+  uint64_t* acc1_full = bars + 12;  // [2]
+  uint64_t* h_full = bars + 14;     // [2] h written over the fc1 accumulator (8 GELU warps)
+  uint64_t* acc2_full = bars + 16;  // [2]
+  uint64_t* acc2_free = bars + 18;  // [2] (4 output warps)
+  uint64_t* w_full = bars + 20;     // [S <= 8]
+  uint64_t* w_free = bars + 28;     // [S <= 8]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 36);
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -194,15 +198,17 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   const uint32_t wbytes = (uint32_t)(2 * C * HC * 2);
 
   if (tid == 0) {
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kMlpXBufs; ++k) {
       mbar_init(&x_full[k], 1);
       mbar_init(&xn_full[k], 4);
       mbar_init(&xn_free[k], 1);
-      mbar_init(&out_full[k], 8);
+      mbar_init(&out_full[k], 4);
+    }
+    for (int k = 0; k < 2; ++k) {
       mbar_init(&acc1_full[k], 1);
       mbar_init(&h_full[k], 8);
       mbar_init(&acc2_full[k], 1);
-      mbar_init(&acc2_free[k], 8);
+      mbar_init(&acc2_free[k], 4);
     }
     for (int k = 0; k < S; ++k) {
       mbar_init(&w_full[k], 1);
@@ -231,26 +237,26 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    // Per tile t: store the output of tile t - 2 from buffer t & 1 (once the
-    // epilogue has staged it there), then load x of tile t into that buffer and
-    // the weight chunks tile t needs.
+    // Per tile t: store the output of tile t - 3 from buffer t % 3 (once it
+    // has been staged there), then load x of tile t into that buffer and the
+    // weight chunks tile t needs.
     if (lane == 0) {
       long long g = 0;  // global chunk counter
-      for (long long t = 0; t < ntiles + 2 && !s_abort; ++t) {
-        const int xb = (int)(t & 1);
-        if (t >= 2) {
-          const long long ts = t - 2;
-          if (!mbar_wait(&out_full[xb], (uint32_t)(ts >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) {
+      for (long long t = 0; t < ntiles + kMlpXBufs && !s_abort; ++t) {
+        const int xb = (int)(t % kMlpXBufs);
+        if (t >= kMlpXBufs) {
+          const long long ts = t - kMlpXBufs;
+          if (!mbar_wait(&out_full[xb], (uint32_t)(ts / kMlpXBufs) & 1, a.ctx.err, kErrWaitMma, lim)) {
             s_abort = 1;
             break;
           }
-          tma_store_3d(&tm_out, sX[xb], 0, (int)((blockIdx.x + ts * gridDim.x) * 128), 0);
+          tma_store_3d(&tm_out, sX(xb), 0, (int)((blockIdx.x + ts * gridDim.x) * 128), 0);
           bulk_commit();
           bulk_wait_read0();  // the buffer may be overwritten once the store has read it
         }
         if (t >= ntiles) continue;
         mbar_arrive_expect_tx(&x_full[xb], xbytes);
-        tma_load_3d(sX[xb], &tm_x, 0, (int)((blockIdx.x + t * gridDim.x) * 128), 0, &x_full[xb]);
+        tma_load_3d(sX(xb), &tm_x, 0, (int)((blockIdx.x + t * gridDim.x) * 128), 0, &x_full[xb]);
         for (int c = 0; c < NCH; ++c, ++g) {
           if (a.resident && t > 0) continue;
           const int s = (int)(g % S);
@@ -282,14 +288,15 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       auto fc1 = [&](long long g) {
         const long long t = g / NCH;
         const int c = (int)(g % NCH);
-        const int xb = (int)(t & 1);
-        if (c == 0 && !s_abort && !mbar_wait(&xn_full[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim))
+        const int xb = (int)(t % kMlpXBufs);
+        if (c == 0 && !s_abort &&
+            !mbar_wait(&xn_full[xb], (uint32_t)(t / kMlpXBufs) & 1, a.ctx.err, kErrWaitLoad, lim))
           s_abort = 1;
         const int s = stage_of(g);
         if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
         tc_fence_after();
         if (s_abort) return;
-        const uint32_t xa = smem_u32(sX[xb]);
+        const uint32_t xa = smem_u32(sX(xb));
         const uint32_t wa = smem_u32(smem + L.w + s * L.wstage);
         const uint32_t d = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
         // K step ks covers channels [16 ks, 16 ks + 16): block ks / 2, 32 B in
@@ -331,38 +338,39 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue warps
-    const int q = warp & 3;                 // TMEM lane quarter
-    const int hf = (warp - kMlpEpi0) >> 2;  // 0: warps 2-5, 1: warps 6-9
-    const int r = q * 32 + lane;            // this thread's row of the tile
+    // ------------------------------------------------------------ norm / output and GELU warps
+    const int q = warp & 3;  // TMEM lane quarter
+    const int r = q * 32 + lane;  // this thread's row of the tile
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    const bool norm_warp = hf == 0;
-    // Normalise tile t in place (norm warps): row r of sX[t & 1].
-    auto normalise = [&](long long t) {
-      const int xb = (int)(t & 1);
-      if (!s_abort && !mbar_wait(&x_full[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
-      if (!s_abort) {
-        uint8_t* row = sX[xb];
-        uint4 v[kMlpMaxC / 8];
-        float sum = 0.f;
-#pragma unroll
-        for (int k = 0; k < kMlpMaxC / 8; ++k) {
-          if (k < C / 8) {
-            v[k] = *reinterpret_cast<const uint4*>(row + sw64_chunk(r, k));
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+    if (warp < kMlpGelu0) {
+      // Warps 2-5: normalise each tile in place (row r of its buffer) as soon as
+      // it lands, and write each tile's output: acc2 + b2 + x (x re-read from
+      // global memory, loaded before the wait for the accumulator) -> bf16 over
+      // the tile's buffer, which the producer then stores with TMA.
+      auto normalise = [&](long long t) {
+        const int xb = (int)(t % kMlpXBufs);
+        if (!s_abort && !mbar_wait(&x_full[xb], (uint32_t)(t / kMlpXBufs) & 1, a.ctx.err, kErrWaitLoad, lim))
+          s_abort = 1;
+        if (!s_abort) {
+          // three passes over the row in shared memory (sum, squared deviations,
+          // normalised write-back) keep no copy of it in registers
+          uint8_t* row = sX(xb);
+          auto chunk = [&](int k) { return *reinterpret_cast<const uint4*>(row + sw64_chunk(r, k)); };
+          float sum = 0.f;
+          for (int k = 0; k < C / 8; ++k) {
+            const uint4 v = chunk(k);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(h2[e]);
               sum += f.x + f.y;
             }
           }
-        }
-        const float mean = sum / (float)C;
-        float ss = 0.f;
-#pragma unroll
-        for (int k = 0; k < kMlpMaxC / 8; ++k) {
-          if (k < C / 8) {
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+          const float mean = sum / (float)C;
+          float ss = 0.f;
+          for (int k = 0; k < C / 8; ++k) {
+            const uint4 v = chunk(k);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(h2[e]);
@@ -370,12 +378,10 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
               ss = fmaf(d0, d0, fmaf(d1, d1, ss));
             }
           }
-        }
-        const float rstd = 1.0f / sqrtf(ss / (float)C + a.eps);
-#pragma unroll
-        for (int k = 0; k < kMlpMaxC / 8; ++k) {
-          if (k < C / 8) {
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+          const float rstd = 1.0f / sqrtf(ss / (float)C + a.eps);
+          for (int k = 0; k < C / 8; ++k) {
+            const uint4 v = chunk(k);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -387,96 +393,99 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
             *reinterpret_cast<uint4*>(row + sw64_chunk(r, k)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-      }
-      fence_proxy_async_smem();  // generic writes -> tensor-core operand reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cta(&xn_full[xb]);
-    };
-    // GELU of chunk g: this warp's HC/2 fc1 columns (half hf of the chunk) ->
-    // HC/4 columns of bf16 pairs over the first half of the same columns.
-    auto gelu_chunk = [&](long long g) {
-      const int c = (int)(g % NCH);
-      if (!s_abort && !mbar_wait(&acc1_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
-        s_abort = 1;
-      tc_fence_after();
-      if (!s_abort) {
-        const uint32_t ta = tAcc1 + lane_base + (uint32_t)(g & 1) * (uint32_t)HC + (uint32_t)(hf * (HC / 2));
-        const float* b1 = sB1 + c * HC + hf * (HC / 2);
-        uint32_t u[32], w[16];
-        for (int part = 0; part < HC / 64; ++part) {
-          tmem_ld32(ta + 32 * part, u);
-          tmem_wait_ld_keep(u);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 bb = *reinterpret_cast<const float2*>(b1 + 32 * part + 2 * e);
-            const float2 v = __fadd2_rn(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), bb);
-            const float2 gv = gelu2(v);
-            w[e] = pack2(gv.x, gv.y);
-          }
-          tmem_st16(ta + 16 * part, w);
-        }
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cta(&h_full[g & 1]);
-    };
-    // Output of tile t: acc2 + b2 + x (re-read from global memory: the tile's
-    // buffer holds the normalised tokens) -> bf16 over the tile's buffer, then
-    // the producer stores it with TMA.
-    auto finish_tile = [&](long long t) {
-      const int xb = (int)(t & 1), ob = (int)(t & 1);
-      if (!s_abort && !mbar_wait(&acc2_full[ob], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
-      if (!s_abort && !mbar_wait(&xn_free[xb], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
-      tc_fence_after();
-      if (!s_abort) {
-        const int half = C / 2;  // a multiple of 16
-        const uint32_t ta = tAcc2 + lane_base + (uint32_t)ob * (uint32_t)C + (uint32_t)(hf * half);
+        fence_proxy_async_smem();  // generic writes -> tensor-core operand reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cta(&xn_full[xb]);
+      };
+      auto finish_tile = [&](long long t) {
+        const int xb = (int)(t % kMlpXBufs), ob = (int)(t & 1);
         const long long grow = (blockIdx.x + t * gridDim.x) * 128 + r;
         const bool real = grow < a.M;
         const __nv_bfloat16* xrow = a.x + (real ? grow : 0) * C;
-        uint8_t* buf = sX[xb];
-        for (int c0 = 0; c0 < half; c0 += 16) {
-          uint32_t u[16];
-          tmem_ld16(ta + c0, u);
-          tmem_wait_ld_keep(u);
+        // the residual row is brought into L1 while this warp waits for the accumulator
+        for (int k = 0; k < C / 8; k += 4)
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(xrow + 8 * k));
+        if (!s_abort && !mbar_wait(&acc2_full[ob], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
+          s_abort = 1;
+        if (!s_abort &&
+            !mbar_wait(&xn_free[xb], (uint32_t)(t / kMlpXBufs) & 1, a.ctx.err, kErrWaitMma, lim))
+          s_abort = 1;
+        tc_fence_after();
+        if (!s_abort) {
+          const uint32_t ta = tAcc2 + lane_base + (uint32_t)ob * (uint32_t)C;
+          uint8_t* buf = sX(xb);
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int ch = hf * half + c0 + 8 * k;  // first channel of this 8-channel group
-            const uint4 xv = real ? *reinterpret_cast<const uint4*>(xrow + ch) : make_uint4(0, 0, 0, 0);
-            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
-            uint32_t w[4];
+          for (int c0 = 0; c0 < kMlpMaxC; c0 += 16) {
+            if (c0 >= C) break;
+            uint32_t u[16];
+            tmem_ld16(ta + c0, u);
+            tmem_wait_ld_keep(u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 xf = __bfloat1622float2(x2[e]);
-              const float2 bb = *reinterpret_cast<const float2*>(sB2 + ch + 2 * e);
-              float2 v = __fadd2_rn(
-                  make_float2(__uint_as_float(u[8 * k + 2 * e]), __uint_as_float(u[8 * k + 2 * e + 1])), bb);
-              v = __fadd2_rn(v, xf);
-              w[e] = pack2(v.x, v.y);
+            for (int k = 0; k < 2; ++k) {
+              const int ch = c0 + 8 * k;  // first channel of this 8-channel group
+              const uint4 xv = real ? *reinterpret_cast<const uint4*>(xrow + ch) : make_uint4(0, 0, 0, 0);
+              const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 xf = __bfloat1622float2(x2[e]);
+                const float2 bb = *reinterpret_cast<const float2*>(sB2 + ch + 2 * e);
+                float2 v = __fadd2_rn(
+                    make_float2(__uint_as_float(u[8 * k + 2 * e]), __uint_as_float(u[8 * k + 2 * e + 1])), bb);
+                v = __fadd2_rn(v, xf);
+                w[e] = pack2(v.x, v.y);
+              }
+              *reinterpret_cast<uint4*>(buf + sw64_chunk(r, ch >> 3)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            *reinterpret_cast<uint4*>(buf + sw64_chunk(r, ch >> 3)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
+        tc_fence_before();
+        fence_proxy_async_smem();  // staged rows -> the producer's TMA store
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cta(&acc2_free[ob]);
+          mbar_arrive_cta(&out_full[xb]);
+        }
+      };
+      // tiles are normalised one ahead of the output they wait for
+      if (ntiles > 0) normalise(0);
+      for (long long t = 0; t < ntiles; ++t) {
+        if (t + 1 < ntiles) normalise(t + 1);
+        finish_tile(t);
       }
-      tc_fence_before();
-      fence_proxy_async_smem();  // staged rows -> the producer's TMA store
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cta(&acc2_free[ob]);
-        mbar_arrive_cta(&out_full[xb]);
+    } else {
+      // Warps 6-13: GELU of each hidden chunk, this warp's HC/2 fc1 columns
+      // (half hf of the chunk) -> HC/4 columns of bf16 pairs over the first half
+      // of the same columns.
+      const int hf = (warp - kMlpGelu0) >> 2;
+      const long long total = ntiles * NCH;
+      for (long long g = 0; g < total; ++g) {
+        const int c = (int)(g % NCH);
+        if (!s_abort && !mbar_wait(&acc1_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
+          s_abort = 1;
+        tc_fence_after();
+        if (!s_abort) {
+          const uint32_t ta = tAcc1 + lane_base + (uint32_t)(g & 1) * (uint32_t)HC + (uint32_t)(hf * (HC / 2));
+          const float* b1 = sB1 + c * HC + hf * (HC / 2);
+          uint32_t u[32], w[16];
+          for (int part = 0; part < HC / 64; ++part) {
+            tmem_ld32(ta + 32 * part, u);
+            tmem_wait_ld_keep(u);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 bb = *reinterpret_cast<const float2*>(b1 + 32 * part + 2 * e);
+              const float2 v = __fadd2_rn(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), bb);
+              const float2 gv = gelu2(v);
+              w[e] = pack2(gv.x, gv.y);
+            }
+            tmem_st16(ta + 16 * part, w);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cta(&h_full[g & 1]);
       }
-    };
-
-    long long g = 0;
-    if (norm_warp && ntiles > 0) normalise(0);
-    for (long long t = 0; t < ntiles; ++t) {
-      for (int c = 0; c < NCH; ++c, ++g) {
-        gelu_chunk(g);
-        // the next tile is normalised early so that its first fc1 never waits
-        if (c == 0 && norm_warp && t + 1 < ntiles) normalise(t + 1);
-      }
-      finish_tile(t);
     }
   }
   tc_fence_before();
