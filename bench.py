@@ -400,7 +400,10 @@ def run_gpu(args):
         peak = float(peaks["bf16_tflops"])
         traffic_kernel = "attention_kernel"
     else:
-        dom_work, unit, bound = work["gemm_flops"] * args.steps, "TFLOP/s", "tensor"
+        # the dominant GEMM's own FLOPs: QKV 2 tok C 3C, projection 2 tok C C, per layer
+        per = sum((2 * ly.B * ly.T * ly.H * ly.W * ly.C * (3 * ly.C if dom == "qkv_gemm" else ly.C))
+                  for ly in layers)
+        dom_work, unit, bound = per * args.steps, "TFLOP/s", "tensor"
         achieved = dom_work / (dom_ms / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
         traffic_kernel = "gemm_kernel"
