@@ -710,6 +710,77 @@ def run_mlp(args):
     return 0
 
 
+def run_merge(args):
+    """``--merge``: patch merging (vswin_patch_merge_forward) of each layer's token tensor
+    of the workload, the step between Video Swin stages. One GPU; prints its own JSON line."""
+    from shifted_window_attention_sw_b200 import build as build_mod
+    from shifted_window_attention_sw_b200 import vswin
+    from shifted_window_attention_sw_b200.inputs import make_merge_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    build_mod.build()
+    vswin.lib()
+    wl = WORKLOADS[args.workload]
+    layers = wl.layers
+    base = 1000 * wl.index
+    ins = [make_merge_inputs(ly.shape, wl.dtype, "baseline", seed=base + ly.seed_offset).to(device) for ly in layers]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    eps = 1e-5
+
+    def step():
+        for m in ins:
+            vswin.patch_merge_forward(m.x, m.gamma, m.beta, eps, m.Wr, m.br, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = vswin.launch_count()
+    vswin.profile_enable(True)
+    sampler = ClockSampler(device)
+    sampler.start()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    vswin.profile_enable(False)
+    prof = vswin.profile_collect()
+    if vswin.poll_error(stream) != vswin.OK:
+        raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    peaks, peak_src = load_peaks()
+    tokens = sum(ly.B * ly.T * ly.H * ly.W for ly in layers)
+    merged = sum(ly.B * ly.T * ((ly.H + 1) // 2) * ((ly.W + 1) // 2) for ly in layers)
+    flops = sum(2 * ly.B * ly.T * ((ly.H + 1) // 2) * ((ly.W + 1) // 2) * 4 * ly.C * 2 * ly.C for ly in layers)
+    byts = sum(2 * ly.B * ly.T * ly.H * ly.W * ly.C + 2 * ly.B * ly.T * ((ly.H + 1) // 2) * ((ly.W + 1) // 2) * 2 * ly.C
+               for ly in layers)
+    k_ms, k_n = prof["mlp"]  # the merge GEMM is timed in the MLP kind
+    k_us = 1e3 * k_ms / max(1, k_n)
+    line = {
+        "metric": f"patch merging input tokens/s, {wl.name}", "value": tokens / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(wl), merged_tokens=merged, ln_eps=eps), "api": "vswin_patch_merge_forward",
+        "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+        "merge_roofline": {"kernel": "pm_kernel", "bound": "hbm", "achieved": byts / len(layers) / (k_us / 1e6) / 1e9,
+                           "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                           "frac": byts / len(layers) / (k_us / 1e6) / 1e9 / float(peaks["hbm_gbs"]),
+                           "peak_source": f"{peak_src} HBM copy", "avg_launch_us": k_us,
+                           "tflops": flops / len(layers) / (k_us / 1e6) / 1e12,
+                           "units_per_launch": "one layer's tokens; bytes = x read + merged output written"},
+        "gpu_launches": int(vswin.launch_count() - launches0),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -726,13 +797,15 @@ def main(argv=None):
                     help="time the fp32 backward of each layer of the workload on one GPU")
     ap.add_argument("--mlp", action="store_true",
                     help="time the fused MLP half of a block (hidden 4C) on each layer's tokens, one GPU")
+    ap.add_argument("--merge", action="store_true",
+                    help="time patch merging (2x2 neighbours, LN over 4C, 4C -> 2C) of each layer's tokens, one GPU")
     ap.add_argument("--block-full", action="store_true",
                     help="time whole blocks (attention half then MLP half) on the workload's layers, one GPU")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "0"))
-    if args.gpus > 1 and world == 0 and not (args.block or args.backward or args.mlp or args.block_full):
+    if args.gpus > 1 and world == 0 and not (args.block or args.backward or args.mlp or args.block_full or args.merge):
         # one process per GPU: relaunch this command under torchrun
         import socket
 
@@ -753,6 +826,8 @@ def main(argv=None):
         return run_backward(args)
     if args.mlp or args.block_full:
         return run_mlp(args)
+    if args.merge:
+        return run_merge(args)
     return run_gpu(args)
 
 

@@ -220,11 +220,16 @@ int vswin_wmsa_backward_f32(const void* x, int B, int T, int H, int W, int C, in
 
 /*
  * bf16 layer forward with the activations in HOST memory: copies x_host to
- * the device, runs vswin_wmsa_forward, copies the result to out_host and
- * synchronises `stream`. Weights, biases and table are device pointers (they
- * stay resident between calls). Page-locked host buffers give asynchronous
- * copies; pageable ones work but are slower. Device buffers for x and out
- * come from the library's stream-ordered pool (see vswin_wmsa_forward).
+ * the device, runs the layer, copies the result to out_host and synchronises
+ * `stream`. Weights, biases and table are device pointers (they stay resident
+ * between calls). The batch goes through in up to four groups of clips (the
+ * windows of a clip read only that clip), so that the copy in of one group,
+ * the layer on the previous one and the copy out of the one before overlap:
+ * the copies run on two streams of the library's (created once per device,
+ * non-blocking), ordered against `stream` with events. Page-locked host
+ * buffers give asynchronous copies; pageable ones work but are slower. Device
+ * buffers for x and out come from the library's stream-ordered pool (see
+ * vswin_wmsa_forward). Results are bitwise those of vswin_wmsa_forward.
  */
 int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads,
                             const int* window, const int* shift,

@@ -215,23 +215,37 @@ __global__ void __launch_bounds__(kPmThreads) pm_kernel(PmArgs a) {
 }
 
 // Wt = bf16(diag(gamma) Wr), colsum of the rounded Wt, bias = beta Wr + br
-// (br may be null). One thread per output column.
-__global__ void pm_fold_kernel(int K, int N2, const __nv_bfloat16* __restrict__ gamma,
-                               const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ Wr,
-                               const __nv_bfloat16* __restrict__ br, __nv_bfloat16* __restrict__ wt,
-                               float* __restrict__ colsum, float* __restrict__ bias) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= N2) return;
+// (br may be null). Block (32 x 32): 32 output columns, the K rows split over
+// 32 thread rows (independent loads), partial sums reduced in shared memory.
+constexpr int kPmFoldCols = 32, kPmFoldRows = 32;
+__global__ void __launch_bounds__(kPmFoldCols * kPmFoldRows)
+    pm_fold_kernel(int K, int N2, const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta,
+                   const __nv_bfloat16* __restrict__ Wr, const __nv_bfloat16* __restrict__ br,
+                   __nv_bfloat16* __restrict__ wt, float* __restrict__ colsum, float* __restrict__ bias) {
+  __shared__ float s_cs[kPmFoldRows][kPmFoldCols + 1], s_bb[kPmFoldRows][kPmFoldCols + 1];
+  const int tx = threadIdx.x % kPmFoldCols, ty = threadIdx.x / kPmFoldCols;
+  const int j = blockIdx.x * kPmFoldCols + tx;
   float cs = 0.f, bb = 0.f;
-  for (int k = 0; k < K; ++k) {
-    const float w = __bfloat162float(Wr[(size_t)k * N2 + j]);
-    const __nv_bfloat16 wg = __float2bfloat16_rn(__bfloat162float(gamma[k]) * w);
-    wt[(size_t)k * N2 + j] = wg;
-    cs += __bfloat162float(wg);
-    bb = fmaf(__bfloat162float(beta[k]), w, bb);
+  if (j < N2) {
+    for (int k = ty; k < K; k += kPmFoldRows) {
+      const float w = __bfloat162float(Wr[(size_t)k * N2 + j]);
+      const __nv_bfloat16 wg = __float2bfloat16_rn(__bfloat162float(gamma[k]) * w);
+      wt[(size_t)k * N2 + j] = wg;
+      cs += __bfloat162float(wg);
+      bb = fmaf(__bfloat162float(beta[k]), w, bb);
+    }
   }
-  colsum[j] = cs;
-  bias[j] = bb + (br ? __bfloat162float(br[j]) : 0.f);
+  s_cs[ty][tx] = cs;
+  s_bb[ty][tx] = bb;
+  __syncthreads();
+  if (ty == 0 && j < N2) {
+    for (int k = 1; k < kPmFoldRows; ++k) {
+      cs += s_cs[k][tx];
+      bb += s_bb[k][tx];
+    }
+    colsum[j] = cs;
+    bias[j] = bb + (br ? __bfloat162float(br[j]) : 0.f);
+  }
 }
 
 }  // namespace
@@ -269,7 +283,7 @@ cudaError_t launch_patch_merge(const KernelCtx& ctx, int B, int T, int H, int W,
   a.eps = eps;
   a.ctx = ctx;
   prof_begin(kKindOther, st);
-  pm_fold_kernel<<<(N2 + 127) / 128, 128, 0, st>>>(
+  pm_fold_kernel<<<(N2 + kPmFoldCols - 1) / kPmFoldCols, kPmFoldCols * kPmFoldRows, 0, st>>>(
       K, N2, static_cast<const __nv_bfloat16*>(gamma), static_cast<const __nv_bfloat16*>(beta),
       static_cast<const __nv_bfloat16*>(Wr), static_cast<const __nv_bfloat16*>(br),
       reinterpret_cast<__nv_bfloat16*>(base), reinterpret_cast<float*>(base + wt_bytes),

@@ -200,6 +200,26 @@ long long chunk_windows(const Geom& g) {
   return (g.windows + nchunks - 1) / nchunks;
 }
 
+// Copy streams of the host-buffer entry, created once per device (non-blocking,
+// so that they do not serialise with the legacy default stream).
+constexpr int kHostChunks = 4;
+cudaStream_t g_h2d[kMaxDevices] = {nullptr}, g_d2h[kMaxDevices] = {nullptr};
+int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VSWIN_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_h2d[dev]) {
+    e = cudaStreamCreateWithFlags(&g_h2d[dev], cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&g_d2h[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaStreamCreateWithFlags");
+  }
+  *h2d = g_h2d[dev];
+  *d2h = g_d2h[dev];
+  return VSWIN_OK;
+}
+
 // Arguments of the MLP half (see vswin_mlp_forward); M = tokens on success.
 int check_mlp_args(const void* x, int B, int T, int H, int W, int C, int hidden, const void* ln_gamma,
                    const void* ln_beta, float ln_eps, const void* W1, const void* b1, const void* W2, const void* b2,
@@ -622,28 +642,76 @@ int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int 
   if (!x_host || !out_host) return fail(VSWIN_ERR_INVALID_ARG, "x_host and out_host must be non-NULL");
   const size_t act = (size_t)g.tokens * g.C * 2;
   if (overlap(x_host, act, out_host, act)) return fail(VSWIN_ERR_INVALID_ARG, "x_host and out_host overlap");
+  {
+    const void* w[] = {Wqkv, bqkv, Wproj, bproj, bias_table};
+    const char* wn[] = {"Wqkv", "bqkv", "Wproj", "bproj", "bias_table"};
+    for (int k = 0; k < 5; ++k) {
+      if (!w[k]) return fail(VSWIN_ERR_INVALID_ARG, "%s is NULL", wn[k]);
+      if (!aligned(w[k], k == 0 || k == 2 ? 16 : 2))
+        return fail(VSWIN_ERR_INVALID_ARG, "%s is not %d-byte aligned", wn[k], k == 0 || k == 2 ? 16 : 2);
+    }
+  }
+  if (g.d != 32) return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path needs head width 32 (C/heads = %d)", g.d);
+  if (!bf16_window_supported(g))
+    return fail(VSWIN_ERR_UNSUPPORTED, "bf16 path has no kernel for window (%d,%d,%d)", g.win[0], g.win[1],
+                g.win[2]);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  st = copy_streams(&h2d, &d2h);
+  if (st != VSWIN_OK) return st;
   void* buf = nullptr;
   const size_t act_pad = (act + 255) / 256 * 256;
   st = scratch_alloc(&buf, 2 * act_pad, s);
   if (st != VSWIN_OK) return st;
+  uint8_t* xd = static_cast<uint8_t*>(buf);
+  uint8_t* od = xd + act_pad;
+  // Clips are independent (the roll and the windows stay inside a clip), so the
+  // batch goes through in groups of clips: the copy in of group k + 1, the layer
+  // on group k and the copy out of group k - 1 overlap on three streams.
+  const int nchunk = B < kHostChunks ? B : kHostChunks;
+  const int per = (B + nchunk - 1) / nchunk;
+  const size_t clip = (size_t)T * H * W * C * 2;
+  cudaEvent_t ev[1 + 3 * kHostChunks] = {};
+  int nev = 0;
   cudaError_t e = cudaSuccess;
-  void* xd = buf;
-  void* od = static_cast<uint8_t*>(buf) + act_pad;
-  e = cudaMemcpyAsync(xd, x_host, act, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) {
-    st = check_layer_ptrs(xd, Wqkv, bqkv, Wproj, bproj, bias_table, od, g, 2, 16);
-    if (st == VSWIN_OK) st = forward_bf16_device(xd, g, Wqkv, bqkv, Wproj, bproj, bias_table, od, s);
-    if (st == VSWIN_OK) {
-      e = cudaMemcpyAsync(out_host, od, act, cudaMemcpyDeviceToHost, s);
-      if (e != cudaSuccess) st = fail_cuda(e, "cudaMemcpyAsync(out)");
-    }
-  } else {
-    st = fail_cuda(e, "cudaMemcpyAsync(x)");
+  for (int k = 0; k < 1 + 3 * nchunk && e == cudaSuccess; ++k, ++nev)
+    e = cudaEventCreateWithFlags(&ev[k], cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventRecord(ev[0], s);  // the device buffers exist on s from here
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h2d, ev[0], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(d2h, ev[0], 0);
+  int last_out = -1;
+  for (int k = 0; k < nchunk && e == cudaSuccess && st == VSWIN_OK; ++k) {
+    const int b0 = k * per, nb = (B - b0) < per ? (B - b0) : per;
+    if (nb <= 0) break;
+    const size_t off = (size_t)b0 * clip, bytes = (size_t)nb * clip;
+    cudaEvent_t ev_in = ev[1 + 3 * k], ev_comp = ev[2 + 3 * k], ev_out = ev[3 + 3 * k];
+    e = cudaMemcpyAsync(xd + off, static_cast<const uint8_t*>(x_host) + off, bytes, cudaMemcpyHostToDevice, h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in, h2d);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in, 0);
+    if (e != cudaSuccess) break;
+    Geom gk;
+    st = build_geom(nb, T, H, W, C, heads, window, shift, &gk);
+    if (st == VSWIN_OK) st = forward_bf16_device(xd + off, gk, Wqkv, bqkv, Wproj, bproj, bias_table, od + off, s);
+    if (st != VSWIN_OK) break;
+    e = cudaEventRecord(ev_comp, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(d2h, ev_comp, 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + off, od + off, bytes, cudaMemcpyDeviceToHost, d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out, d2h);
+    if (e == cudaSuccess) last_out = 3 + 3 * k;
+  }
+  if (e != cudaSuccess && st == VSWIN_OK) st = fail_cuda(e, "host-entry copy or event");
+  // the buffers are released on s only after every copy out has read them
+  if (last_out >= 0) cudaStreamWaitEvent(s, ev[last_out], 0);
+  if (st != VSWIN_OK) {  // something was refused part-way: let whatever was queued finish first
+    cudaStreamSynchronize(h2d);
+    cudaStreamSynchronize(d2h);
   }
   cudaFreeAsync(buf, s);
   e = cudaStreamSynchronize(s);
   if (st == VSWIN_OK && e != cudaSuccess) st = fail_cuda(e, "cudaStreamSynchronize");
+  for (int k = 0; k < nev; ++k)
+    if (ev[k]) cudaEventDestroy(ev[k]);
   return st;
 }
 

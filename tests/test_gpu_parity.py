@@ -206,8 +206,10 @@ def test_bf16_deterministic():
     assert torch.equal(o1, o2)
 
 
-def test_bf16_host_entry_matches_device_entry():
-    shape, heads, window, shift = (1, 16, 14, 14, 96), 3, (8, 7, 7), (4, 3, 3)
+@pytest.mark.parametrize("shape", [(1, 16, 14, 14, 96), (5, 8, 14, 21, 96), (3, 8, 7, 7, 96)])
+def test_bf16_host_entry_matches_device_entry(shape):
+    # the host entry pipelines groups of clips (5 clips: groups of 2, 2, 1; 3 clips: 1 each)
+    heads, window, shift = 3, (8, 7, 7), (4, 3, 3)
     inp = make_layer_inputs(shape, heads, window, "bf16", "sensitivity", seed=8)
     d = inp.to("cuda")
     dev = vswin.wmsa_forward(d.x, window, shift, d.Wqkv, d.bqkv, d.Wproj, d.bproj, d.table, heads)
