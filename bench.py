@@ -406,7 +406,7 @@ def run_gpu(args):
         dom_work, unit, bound = per * args.steps, "TFLOP/s", "tensor"
         achieved = dom_work / (dom_ms / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
-        traffic_kernel = "gemm_kernel"
+        traffic_kernel = "gemm_kernel" if dom == "qkv_gemm" else "proj_kernel"
     tr = traffic_record(traffic_kernel)
     avg_us = 1e3 * dom_ms / max(1, dom_launches)
     roofline = {
@@ -698,6 +698,7 @@ def run_mlp(args):
         "api": "vswin_block_msa_forward + vswin_mlp_forward" if args.block_full else "vswin_mlp_forward",
         "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
         "mlp_roofline": {"kernel": "mlp_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "traffic": (traffic_record("mlp_kernel") or {}).get("bytes_per_launch"),
                          "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_src} bf16 dense (burst)",
                          "avg_launch_us": mlp_us, "launches": mlp_n,
                          "hbm_floor_us": mlp_bytes / len(layers) / (float(peaks["hbm_gbs"]) * 1e9) * 1e6,
