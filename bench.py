@@ -591,17 +591,17 @@ def run_backward(args):
     if vswin.poll_error(stream) != vswin.OK:
         raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
     ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    # FLOPs of the kernels as built, per layer (rows = window slots):
-    # forward recompute 2 rows C 3C + 4 windows N^2 C + 2 rows C^2; dO 2 rows C^2;
-    # row pass 6 N^2 C per window; column pass 8 N^2 C; dx 2 rows 3C C; dWqkv 2 rows C 3C;
-    # dWproj 2 rows C^2
+    # FLOPs of the kernels as built, per layer (rows = window slots, masked pairs
+    # included): qkv recompute 2 rows C 3C; dO 2 rows C^2; per window, the query
+    # pass 10 N^2 C (scores twice, O, dP, dq) and the key pass 8 N^2 C (scores,
+    # dP, dk, dv); dx 2 rows 3C C; dWqkv 2 rows C 3C; dWproj 2 rows C^2
     flops = 0
     for ly in layers:
         g = layer_work(ly.B, ly.T, ly.H, ly.W, ly.C, ly.heads, ly.window, ly.shift, 4)
         win, N = g["windows"], g["N"]
         rows = win * N
         C = ly.C
-        flops += 2 * rows * C * 3 * C * 3 + 2 * rows * C * C * 3 + (4 + 6 + 8) * win * N * N * C
+        flops += 2 * rows * C * 3 * C * 3 + 2 * rows * C * C * 2 + (10 + 8) * win * N * N * C
     tokens = step_work(wl)["tokens"]
     achieved = flops / (ms / 1e3) / 1e12
     peak = 148 * 128 * 2 * 1.965e9 / 1e12
