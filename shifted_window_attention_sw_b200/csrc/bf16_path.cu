@@ -614,24 +614,25 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     // row, lane l moving chunks l%4, l%4 + 4, ... (64 contiguous bytes per row and
     // instruction).
     const int sub = lane >> 2, cq = lane & 3;
-    // Source offsets of this lane's 4 rows, fetched two tiles ahead so that the
-    // table reads (global loads) have landed by the time the copies need them.
     // Row index of each of this lane's 4 rows in the source matrix (-1:
-    // padding): QKV looks it up in the row table, two tiles ahead, and keeps the
-    // raw value so that nothing waits for the load before it is needed.
+    // padding): QKV looks it up in the row table.
     auto row_tok = [&](long long m, int grp) -> int {
       const long long r = m * kBM + warp * 32 + grp * 8 + sub;
       if (m >= mtiles || r >= a.rows) return -1;
       return MODE == kQKV ? a.rowsrc[r] : (int)r;
     };
-    int tok0[4], tok1[4], tok2[4];
+    // Three register sets in rotation: the set of tile t is refilled with tile
+    // t + 3's rows right after its copies are issued, so no instruction reads a
+    // table value before about two tiles have passed (a register copy of a
+    // pending load would stall the warp until the load lands).
+    int tokA[4], tokB[4], tokC[4];
 #pragma unroll
     for (int grp = 0; grp < 4; ++grp) {
-      tok0[grp] = row_tok(m_first, grp);
-      tok1[grp] = row_tok(m_first + m_step, grp);
+      tokA[grp] = row_tok(m_first, grp);
+      tokB[grp] = row_tok(m_first + m_step, grp);
+      tokC[grp] = row_tok(m_first + 2 * m_step, grp);
     }
-    long long t = 0;
-    for (long long m = m_first; m < mtiles; m += m_step, ++t) {
+    auto tile = [&](long long m, long long t, int (&tok)[4]) {
       const int s = (int)(t % STAGES);
       if (tid == 0) VSWIN_TRACE_EVENT(kTraceG + 0, trace_n, 50);
       if (t >= STAGES && !s_abort &&
@@ -642,7 +643,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       for (int grp = 0; grp < 4; ++grp) {
         const int row = warp * 32 + grp * 8 + sub;
         uint8_t* drow = dA + (row >> 3) * sboA + (row & 7) * 16;
-        const int tk = tok0[grp];
+        const int tk = tok[grp];
         const long long sg = tk < 0 ? 0 : (long long)tk * g.C;
         for (int kc = cq; kc < K / 8; kc += 4)
           cp_async_16(drow + kc * 128, a.A + sg + kc * 8, tk < 0 ? 0u : 16u);
@@ -650,12 +651,15 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       cp_async_mbar_arrive_noinc(&a_full[s]);  // arrives once this thread's copies have landed
       if (tid == 0) VSWIN_TRACE_EVENT(kTraceG + 0, trace_n, 51);
 #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) tok2[grp] = row_tok(m + 2 * m_step, grp);
-#pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
-        tok0[grp] = tok1[grp];
-        tok1[grp] = tok2[grp];
-      }
+      for (int grp = 0; grp < 4; ++grp) tok[grp] = row_tok(m + 3 * m_step, grp);
+    };
+    long long t = 0;
+    for (long long m = m_first; m < mtiles; m += 3 * m_step, t += 3) {
+      tile(m, t, tokA);
+      if (m + m_step >= mtiles) break;
+      tile(m + m_step, t + 1, tokB);
+      if (m + 2 * m_step >= mtiles) break;
+      tile(m + 2 * m_step, t + 2, tokC);
     }
     cp_async_wait_all();  // nothing in flight when the CTA ends
   } else if (warp == kWsMmaWarp) {
@@ -731,6 +735,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       __nv_bfloat16* rbase = nullptr;
       const __nv_bfloat16* xres = nullptr;  // kResid: this row's residual, same columns as rbase
       int q_term = 0, kv_term = 0;
+      // the last key of a 7-key line also zero-fills the line's eighth (padding)
+      // row, so that every 32-byte sector of the k / v slabs is written whole
+      // (a partly written sector costs a DRAM read to merge when it leaves L2)
+      bool kv_pad = false;
       // kLn: (-mean * rstd, rstd) of this row's token, (0, 0) for a padding row
       const float2 st = (kLn && row_ok) ? a.ln_stats[r] : make_float2(0.f, 0.f);
       if (row_ok) {
@@ -739,6 +747,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
           const int slab_win = ri / g.N;
           const int slot = ri - slab_win * g.N;
           const int kvr = a.slab.kv_row(slot);
+          kv_pad = a.slab.kv8 && (kvr & 7) == 6;
           q_term = (slot >> 3) * 256 + (slot & 7) * 8;
           kv_term = (kvr >> 3) * 256 + (kvr & 7) * 8;
           rbase = a.dst + (size_t)slab_win * win_elems;
@@ -816,6 +825,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
               __nv_bfloat16* dst =
                   MODE == kQKV ? rbase + cg.off + (cg.is_q ? q_term : kv_term) : rbase + cc;
               *reinterpret_cast<uint4*>(dst) = w;
+              if (MODE == kQKV && kv_pad && !cg.is_q) *reinterpret_cast<uint4*>(dst + 8) = make_uint4(0, 0, 0, 0);
             }
           }
         }
