@@ -621,6 +621,102 @@ def run_backward(args):
     return 0
 
 
+
+def run_backward_bf16(args):
+    """``--backward-bf16``: the bf16 tensor-core backward (vswin_wmsa_backward: the forward's
+    first three steps recomputed with the softmax statistics, dO, the attention gradients
+    on tcgen05, dX and the fp32 weight gradients) of each layer of the workload. One GPU;
+    prints its own JSON line with the attention-gradient kernel's roofline against the
+    bf16 tensor peak and its exponential (MUFU) bound."""
+    from shifted_window_attention_sw_b200 import build as build_mod
+    from shifted_window_attention_sw_b200 import vswin
+    from shifted_window_attention_sw_b200.inputs import make_layer_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    build_mod.build()
+    vswin.lib()
+    wl = WORKLOADS[args.workload]
+    layers = wl.layers
+    base = 1000 * wl.index
+    ins = [make_layer_inputs(ly.shape, ly.heads, ly.window, "bf16", "baseline", seed=base + ly.seed_offset,
+                             x_seed=base).to(device) for ly in layers]
+    dys = [torch.randn(*ly.shape, generator=torch.Generator().manual_seed(base + 77 + k)).bfloat16().to(device)
+           for k, ly in enumerate(layers)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for ly, i, dy in zip(layers, ins, dys):
+            vswin.wmsa_backward(i.x, ly.window, ly.shift, i.Wqkv, i.bqkv, i.Wproj, i.bproj, i.table, ly.heads,
+                                dy, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = vswin.launch_count()
+    vswin.profile_enable(True)
+    sampler = ClockSampler(device)
+    sampler.start()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    vswin.profile_enable(False)
+    prof = vswin.profile_collect()
+    if vswin.poll_error(stream) != vswin.OK:
+        raise RuntimeError("kernel error in the timed region: " + vswin.last_error())
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    # tensor-core FLOPs as built, per layer (rows = window slots, masked pairs
+    # included): attention gradients 10 N^2 d per (window, head) (S^T, dP^T, dV, dK,
+    # dQ), the recomputed attention 4 N^2 d, and the products qkv 2 rows C 3C, dO
+    # 2 rows C^2, dx 2 rows 3C C; the two weight-gradient sums (2 rows C 3C + 2 rows
+    # C^2) run on the FP32 pipes
+    attn_flops = tc_flops = simt_flops = exps = 0
+    for ly in layers:
+        g = layer_work(ly.B, ly.T, ly.H, ly.W, ly.C, ly.heads, ly.window, ly.shift, 4)
+        win, N = g["windows"], g["N"]
+        rows = win * N
+        C = ly.C
+        attn_flops += 10 * win * N * N * C
+        tc_flops += 14 * win * N * N * C + 2 * rows * C * 3 * C * 2 + 2 * rows * C * C
+        simt_flops += 2 * rows * C * 3 * C + 2 * rows * C * C
+        exps += win * N * N * ly.heads
+    tokens = step_work(wl)["tokens"]
+    line = {
+        "metric": "bf16 layer backward tokens/s (forward recompute + all gradients), " + wl.name,
+        "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(wl),
+        "api": "vswin_wmsa_backward",
+        "tensor_flops_per_step": tc_flops, "fp32_flops_per_step": simt_flops,
+        "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+        "gpu_launches": int(vswin.launch_count() - launches0),
+        "clocks": clocks,
+    }
+    a_ms, a_n = prof["attention_bwd"]
+    if a_n:
+        avg_us = a_ms / a_n * 1e3
+        per_launch = attn_flops * args.steps / a_n  # one launch per layer and chunk
+        achieved = per_launch / (avg_us / 1e6) / 1e12
+        peaks, psrc = load_peaks()
+        peak, src = float(peaks["bf16_tflops"]), f"{psrc} bf16 dense (burst)"
+        exp_us = exps * args.steps / a_n / (148 * 16 * 1.965e9) * 1e6
+        line["roofline"] = {
+            "kernel": "bwd_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": src, "avg_launch_us": avg_us,
+            "launches": a_n, "traffic": None,
+            "units_per_launch": "windows x heads of one chunk; FLOPs 10*windows*N^2*C (S^T, dP^T, dV, dK, dQ)",
+            "exp_bound_us": exp_us, "exp_bound_frac": exp_us / avg_us,
+            "exp_bound_note": "one exponential per (query, key, head), masked pairs included, at 16 per clock per SM"}
+    print(json.dumps(line), flush=True)
+    return 0
+
 def run_mlp(args):
     """``--mlp``: the fused MLP half (vswin_mlp_forward, hidden 4C) on each layer's token
     tensor; ``--block-full``: whole blocks, the attention half (vswin_block_msa_forward)
@@ -794,6 +890,8 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-s", type=float, default=20.0)
     ap.add_argument("--block", action="store_true",
                     help="time the blocks' attention half (LN, layer, residual), fused and unfused, on one GPU")
+    ap.add_argument("--backward-bf16", action="store_true",
+                    help="time the bf16 tensor-core backward of each layer of the workload on one GPU")
     ap.add_argument("--backward", action="store_true",
                     help="time the fp32 backward of each layer of the workload on one GPU")
     ap.add_argument("--mlp", action="store_true",
@@ -806,7 +904,7 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "0"))
-    if args.gpus > 1 and world == 0 and not (args.block or args.backward or args.mlp or args.block_full or args.merge):
+    if args.gpus > 1 and world == 0 and not (args.block or args.backward or args.backward_bf16 or args.mlp or args.block_full or args.merge):
         # one process per GPU: relaunch this command under torchrun
         import socket
 
@@ -825,6 +923,8 @@ def main(argv=None):
         return run_block(args)
     if args.backward:
         return run_backward(args)
+    if args.backward_bf16:
+        return run_backward_bf16(args)
     if args.mlp or args.block_full:
         return run_mlp(args)
     if args.merge:

@@ -219,6 +219,34 @@ int vswin_wmsa_backward_f32(const void* x, int B, int T, int H, int W, int C, in
                             void* dWproj, void* dbproj, void* dtable, void* stream);
 
 /*
+ * bf16 backward of the layer on the tensor cores ("Video Swin Transformer"
+ * summary page, Method steps 4-6 and eq. 2, differentiated as for
+ * vswin_wmsa_backward_f32): x, dy, dx (layout of x), Wqkv, bqkv, Wproj,
+ * bproj and bias_table are bf16 as in vswin_wmsa_forward; dWqkv [C][3C],
+ * dbqkv [3C], dWproj [C][C], dbproj [C] and dtable (layout of bias_table) are
+ * float, overwritten (not accumulated). The forward's first three steps are
+ * recomputed (q, k, v, the attention output and each row's softmax
+ * reference and sum), then dO = dy Wproj^T, the attention gradients per
+ * (window, head) on tcgen05 (S and dP, P and dS rebuilt in registers, dq,
+ * dk, dv as tensor-core products, the table gradient summed per CTA), dx =
+ * dqkv Wqkv^T scattered to the tokens, and the weight and bias gradients as
+ * fp32 sums. Products take bf16 operands with fp32 accumulation; P, dS and
+ * dqkv are rounded to bf16 on the way (gradient error about 1e-2 relative).
+ * Requires head width 32, C % 32 == 0 and a (P,7,7) window with P in
+ * {1, 2, 4, 8}, else VSWIN_ERR_UNSUPPORTED (vswin_wmsa_backward_f32 covers
+ * every shape). x, dy and dx 16-byte aligned; bf16 vectors, weights and
+ * table 2-byte aligned; float outputs 4-byte aligned; outputs may overlap
+ * neither one another nor any input. Not bitwise deterministic (atomics in
+ * the table and weight gradients). Scratch: from the library's pool, about
+ * (5 C + 16 heads) * 2 bytes per window slot plus the forward's chunk scratch.
+ */
+int vswin_wmsa_backward(const void* x, int B, int T, int H, int W, int C, int heads,
+                        const int* window, const int* shift,
+                        const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                        const void* bias_table, const void* dy, void* dx, void* dWqkv, void* dbqkv,
+                        void* dWproj, void* dbproj, void* dtable, void* stream);
+
+/*
  * bf16 layer forward with the activations in HOST memory: copies x_host to
  * the device, runs the layer, copies the result to out_host and synchronises
  * `stream`. Weights, biases and table are device pointers (they stay resident
@@ -336,7 +364,8 @@ enum {
   VSWIN_KERNEL_PROJ_GEMM = 2,  /* output projection + scatter (bf16) */
   VSWIN_KERNEL_OTHER = 3,      /* fp32 path, index maps, self-test */
   VSWIN_KERNEL_MLP = 4,        /* fused MLP half of a block (bf16) */
-  VSWIN_KERNEL_KINDS = 5
+  VSWIN_KERNEL_ATTN_BWD = 5,   /* attention gradients of the bf16 backward */
+  VSWIN_KERNEL_KINDS = 6
 };
 int vswin_profile_enable(int on);
 int vswin_profile_collect(double* ms, unsigned long long* launches, int nkinds);

@@ -24,6 +24,8 @@
 // Otherwise the forward is recomputed by the fp32 forward's kernels and the
 // attention gradients come from a pass per (window, query, head) and a pass per
 // (window, key, head) over global memory.
+#include <cuda_bf16.h>
+
 #include <cmath>
 
 #include "internal.h"
@@ -467,10 +469,10 @@ constexpr int kAL = kBM * kBK / kGT, kBL = kBN * kBK / kGT;
 
 struct GemmArgs {
   long long M, N, K;  // kGram: M = Ma + 1
-  const float* A;
+  const void* A;      // float or bf16 (the kernel's TA)
   long long lda;
   const int* a_src;
-  const float* Bm;
+  const void* Bm;     // float or bf16 (the kernel's TB)
   long long ldb;
   const int* b_src;
   const float* bias;
@@ -481,28 +483,33 @@ struct GemmArgs {
   long long kchunk;  // kGram: K rows per block
 };
 
-template <int MODE>
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <int MODE, class TA>
 __device__ __forceinline__ float gemm_a(const GemmArgs& a, long long m, long long k, long long k1) {
+  const TA* A = static_cast<const TA*>(a.A);
   if (MODE == kGram) {
     if (k >= k1) return 0.f;
     if (m == a.M - 1) return 1.f;
     if (m >= a.M) return 0.f;
     const long long r = a.a_src ? (long long)a.a_src[k] : k;
-    return r >= 0 ? a.A[r * a.lda + m] : 0.f;
+    return r >= 0 ? to_f32(A[r * a.lda + m]) : 0.f;
   }
   if (m >= a.M || k >= a.K) return 0.f;
   const long long r = a.a_src ? (long long)a.a_src[m] : m;
-  return r >= 0 ? a.A[r * a.lda + k] : 0.f;
+  return r >= 0 ? to_f32(A[r * a.lda + k]) : 0.f;
 }
 
-template <int MODE>
+template <int MODE, class TB>
 __device__ __forceinline__ float gemm_b(const GemmArgs& a, long long k, long long n, long long k1) {
+  const TB* Bm = static_cast<const TB*>(a.Bm);
   if (n >= a.N) return 0.f;
-  if (MODE == kRowsNT) return k < a.K ? a.Bm[n * a.ldb + k] : 0.f;
-  if (MODE == kRowsNN) return k < a.K ? a.Bm[k * a.ldb + n] : 0.f;
+  if (MODE == kRowsNT) return k < a.K ? to_f32(Bm[n * a.ldb + k]) : 0.f;
+  if (MODE == kRowsNN) return k < a.K ? to_f32(Bm[k * a.ldb + n]) : 0.f;
   if (k >= k1) return 0.f;
   const long long r = a.b_src ? (long long)a.b_src[k] : k;
-  return r >= 0 ? a.Bm[r * a.ldb + n] : 0.f;
+  return r >= 0 ? to_f32(Bm[r * a.ldb + n]) : 0.f;
 }
 
 // Element e of this thread's share of a tile: (kk, mm) with kk fastest when the
@@ -519,7 +526,7 @@ __device__ __forceinline__ void tile_pos(int e, int& kk, int& mm) {
   }
 }
 
-template <int MODE>
+template <int MODE, class TA, class TB>
 __global__ void __launch_bounds__(kGT) f32_gemm_kernel(GemmArgs a) {
   __shared__ __align__(16) float As[2][kBK][kAS];
   __shared__ __align__(16) float Bs[2][kBK][kBS];
@@ -538,13 +545,13 @@ __global__ void __launch_bounds__(kGT) f32_gemm_kernel(GemmArgs a) {
     for (int e = 0; e < kAL; ++e) {
       int kk, mm;
       tile_pos<AK, kBM>(e, kk, mm);
-      ra[e] = gemm_a<MODE>(a, m0 + mm, kb + kk, k1);
+      ra[e] = gemm_a<MODE, TA>(a, m0 + mm, kb + kk, k1);
     }
 #pragma unroll
     for (int e = 0; e < kBL; ++e) {
       int kk, nn;
       tile_pos<BK_, kBN>(e, kk, nn);
-      rb[e] = gemm_b<MODE>(a, kb + kk, n0 + nn, k1);
+      rb[e] = gemm_b<MODE, TB>(a, kb + kk, n0 + nn, k1);
     }
   };
   auto stash = [&](int buf) {
@@ -619,7 +626,7 @@ __global__ void __launch_bounds__(kGT) f32_gemm_kernel(GemmArgs a) {
   }
 }
 
-template <int MODE>
+template <int MODE, class TA = float, class TB = float>
 cudaError_t launch_gemm(GemmArgs a, cudaStream_t st) {
   const long long gx = (a.M + kBM - 1) / kBM, gy = (a.N + kBN - 1) / kBN;
   long long gz = 1;
@@ -635,13 +642,22 @@ cudaError_t launch_gemm(GemmArgs a, cudaStream_t st) {
   }
   if (gx > 2147483647LL || gy > 65535 || gz > 65535) return cudaErrorInvalidConfiguration;
   prof_begin(kKindOther, st);
-  f32_gemm_kernel<MODE><<<dim3((unsigned)gx, (unsigned)gy, (unsigned)gz), kGT, 0, st>>>(a);
+  f32_gemm_kernel<MODE, TA, TB><<<dim3((unsigned)gx, (unsigned)gy, (unsigned)gz), kGT, 0, st>>>(a);
   prof_end(kKindOther, st);
   count_launch();
   return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_gram_bf16(long long rows, int M, int N, const void* A, long long lda, const int* a_src,
+                             const void* B, long long ldb, const int* b_src, float* out, float* bias_out,
+                             cudaStream_t st) {
+  GemmArgs ga{};
+  ga.M = M + 1, ga.N = N, ga.K = rows, ga.A = A, ga.lda = lda, ga.a_src = a_src, ga.Bm = B, ga.ldb = ldb;
+  ga.b_src = b_src, ga.out = out, ga.ldo = N, ga.bias_out = bias_out;
+  return launch_gemm<kGram, __nv_bfloat16, __nv_bfloat16>(ga, st);
+}
 
 size_t f32_backward_scratch_bytes(const Geom& g) {
   const size_t rows = (size_t)g.windows * g.N;

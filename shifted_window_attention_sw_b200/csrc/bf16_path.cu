@@ -114,6 +114,7 @@ struct GemmArgs {
   const float* ln_colsum;
   const float* ln_bias;
   const __nv_bfloat16* resid;
+  long long lda;  // A row stride in elements (0: C)
 };
 
 __host__ __device__ constexpr int gemm_smem_bytes() {
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
         const long long tok = slot_source(g, gr / g.N, (int)(gr % g.N));
         src = tok < 0 ? -1 : tok * g.C;
       } else {
-        src = r * (long long)g.C;
+        src = r * (long long)(a.lda ? a.lda : g.C);
       }
     }
     s_src[tid] = src;
@@ -544,6 +545,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   const long long mtiles = (a.rows + kBM - 1) / kBM;
   const long long m_first = blockIdx.x / NT, m_step = gridDim.x / NT;
   const uint64_t lim = a.ctx.wait_limit;
+  const long long lda = a.lda ? a.lda : g.C;  // A row stride (elements)
   const uint32_t lboB = (uint32_t)(BN / 8) * 128u;  // B: K-group stride
   const uint32_t sboA = (uint32_t)(K / 8) * 128u;   // A: 8-row group stride
   const uint32_t tcols = BN <= 64 ? 128 : BN <= 128 ? 256 : 512;
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
         const int row = warp * 32 + grp * 8 + sub;
         uint8_t* drow = dA + (row >> 3) * sboA + (row & 7) * 16;
         const int tk = tok[grp];
-        const long long sg = tk < 0 ? 0 : (long long)tk * g.C;
+        const long long sg = tk < 0 ? 0 : (long long)tk * lda;
         for (int kc = cq; kc < K / 8; kc += 4)
           cp_async_16(drow + kc * 128, a.A + sg + kc * 8, tk < 0 ? 0u : 16u);
       }
@@ -884,6 +886,11 @@ struct AttnArgs {
   const __nv_bfloat16* table;  // [rows][heads]
   __nv_bfloat16* o;            // [nwin][N][C]
   long long win0, nwin;
+  // optional (null: not written): per (window slot, head) the reference and the
+  // row sum the probabilities were normalised with, in the exp2 domain --
+  // P = 2^(s + b - m) / l with s the scaled score and b the table entry
+  // (log2 e units); for an exactly recomputed row its true maximum and sum
+  float2* stats;
 };
 
 // Per-thread row context for one query tile.
@@ -1364,8 +1371,9 @@ __device__ __forceinline__ float w7_block(uint32_t tS, int L0, const float* tb_r
 // above): two-pass softmax over the allowed keys on the CUDA cores, operands
 // read from shared memory; writes the row's 32 normalised outputs.
 template <class Wn>
-__device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, const uint8_t* sV, const float* tb_row,
-                                          int i, uint32_t okt, uint32_t okh, uint32_t okw, float* o) {
+__device__ __noinline__ float2 w7_exact_row(const uint8_t* sQ, const uint8_t* sK, const uint8_t* sV,
+                                            const float* tb_row, int i, uint32_t okt, uint32_t okh, uint32_t okw,
+                                            float* o) {
   float q[32];
   for (int c = 0; c < 4; ++c) {
     const uint4 w = *reinterpret_cast<const uint4*>(sQ + (i >> 3) * 512 + c * 128 + (i & 7) * 16);
@@ -1419,6 +1427,7 @@ __device__ __noinline__ void w7_exact_row(const uint8_t* sQ, const uint8_t* sK, 
   }
   const float inv = 1.0f / l;
   for (int d = 0; d < 32; ++d) o[d] *= inv;
+  return make_float2(m, l);
 }
 
 // One elected lane of a converged warp.
@@ -1456,8 +1465,8 @@ __device__ __forceinline__ void w7_issue_pv(uint32_t dO, uint32_t dP, uint64_t v
 // The exact path for query row i of a tile of item buffer X: mask bits of the
 // row, w7_exact_row, and the row's 32 outputs to dst.
 template <class Wn>
-__device__ __noinline__ void w7_exact_store(const AttnArgs& a, const uint8_t* smem, int X, long long wl, int i,
-                                            __nv_bfloat16* dst) {
+__device__ __noinline__ float2 w7_exact_store(const AttnArgs& a, const uint8_t* smem, int X, long long wl, int i,
+                                              __nv_bfloat16* dst) {
   const Geom& g = a.g;
   const int pt_i = i / 49, ph_i = (i / 7) % 7, pw_i = i % 7;
   const int cut_t = Wn::P - g.sh[0], cut_h = 7 - g.sh[1], cut_w = 7 - g.sh[2];
@@ -1478,12 +1487,13 @@ __device__ __noinline__ void w7_exact_store(const AttnArgs& a, const uint8_t* sm
   const float* sT = reinterpret_cast<const float*>(smem + Wn::OFF_T + X * Wn::TB);
   const float* tb_row = sT + (pt_i + Wn::P - 1) * 169 + (ph_i + 6) * 13 + (pw_i + 6);
   float oe[32];
-  w7_exact_row<Wn>(smem + Wn::OFF_Q + X * Wn::QB, smem + Wn::OFF_K + X * Wn::KB, smem + Wn::OFF_V + X * Wn::KB,
-                   tb_row, i, okt, okh, okw, oe);
+  const float2 ml = w7_exact_row<Wn>(smem + Wn::OFF_Q + X * Wn::QB, smem + Wn::OFF_K + X * Wn::KB,
+                                     smem + Wn::OFF_V + X * Wn::KB, tb_row, i, okt, okh, okw, oe);
   for (int k = 0; k < 4; ++k)
     reinterpret_cast<uint4*>(dst)[k] =
         make_uint4(pack_bf16x2(oe[8 * k + 0], oe[8 * k + 1]), pack_bf16x2(oe[8 * k + 2], oe[8 * k + 3]),
                    pack_bf16x2(oe[8 * k + 4], oe[8 * k + 5]), pack_bf16x2(oe[8 * k + 6], oe[8 * k + 7]));
+  return ml;
 }
 
 __device__ __forceinline__ uint32_t bf16_bits(__nv_bfloat16 v) { return (uint32_t)__bfloat16_as_ushort(v); }
@@ -1805,7 +1815,16 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
           }
         }
         // the reference was too loose for this row (or overflowed): recompute it exactly
-        if (c.active && !common) w7_exact_store<Wn>(a, smem, c.X, c.wl, c.i, dst);
+        float2 ml = make_float2(0.f, L);
+        if (c.active && !common) ml = w7_exact_store<Wn>(a, smem, c.X, c.wl, c.i, dst);
+        if (c.active && a.stats) {
+          if (common) {  // the reference the score MMA subtracted: -2 x the extension row's first value
+            const uint8_t* sQX = smem + Wn::OFF_QX + c.X * Wn::QXB;
+            const uint32_t xw = *reinterpret_cast<const uint32_t*>(sQX + (c.i >> 3) * 128 + (c.i & 7) * 16);
+            ml.x = -2.0f * __uint_as_float(xw << 16);
+          }
+          a.stats[((size_t)c.wl * Wn::N + c.i) * g.heads + c.h] = ml;
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -2004,7 +2023,7 @@ cudaError_t launch_ln_fold(const Geom& g, const void* gamma, const void* beta, c
 cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
                               const void* bqkv, const void* Wproj, const void* bproj, const void* table,
                               void* out, void* scratch, long long win0, long long nwin, cudaStream_t st,
-                              const BlockFuse* fuse) {
+                              const BlockFuse* fuse, float2* attn_stats) {
   __nv_bfloat16* qkv = static_cast<__nv_bfloat16*>(scratch);
   const SlabLayout L = slab_layout(g);
   __nv_bfloat16* o = qkv + (size_t)nwin * g.heads * L.head_elems();
@@ -2073,7 +2092,9 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   aa.nwin = nwin;
   aa.slab = L;
   aa.exact_below = ctx.force_exact ? INFINITY : 7.8886e-31f;  // 2^-100
+  aa.stats = attn_stats;
   const int P = g.win[0], MH = g.win[1], MW = g.win[2];
+  if (attn_stats && !window_is_p77(g)) return cudaErrorInvalidValue;  // only the (P,7,7) kernel writes them
   if (P == 16 && MH == 7 && MW == 7) e = launch_attention7<W7<16>>(aa, st);
   else if (P == 8 && MH == 7 && MW == 7) e = launch_attention7<W7<8>>(aa, st);
   else if (P == 4 && MH == 7 && MW == 7) e = launch_attention7<W7<4>>(aa, st);
@@ -2084,6 +2105,7 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   else if (P == 1 && MH == 1 && MW == 1) e = launch_attention<Win<1, 1, 1>>(aa, st);
   else return cudaErrorInvalidValue;
   if (e != cudaSuccess) return e;
+  if (!Wproj) return cudaSuccess;  // the first three steps only (the backward's recomputation)
 
   GemmArgs gp = ga;
   gp.A = o;
@@ -2097,6 +2119,68 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
     gp.resid = static_cast<const __nv_bfloat16*>(x);
     return launch_gemm<kPROJ, true>(gp, st);
   }
+  return launch_gemm<kPROJ, false>(gp, st);
+}
+
+void bf16_slab_rows(const Geom& g, int* qrows, int* kvrows, int* kv8) {
+  const SlabLayout L = slab_layout(g);
+  *qrows = L.qrows;
+  *kvrows = L.kvrows;
+  *kv8 = L.kv8;
+}
+
+size_t bf16_chunk_o_offset(const Geom& g, long long nwin) {
+  return (size_t)nwin * g.heads * slab_layout(g).head_elems() * 2;
+}
+
+size_t bf16_chunk_rows_offset(const Geom& g, long long nwin) {
+  return bf16_chunk_o_offset(g, nwin) + (size_t)nwin * g.N * g.C * 2;
+}
+
+cudaError_t launch_bf16_dout_slabs(const Geom& g, const KernelCtx& ctx, const void* dy, const void* WprojT,
+                                   const void* zero_bias, void* dO, const int* rowsrc, long long win0,
+                                   long long nwin, cudaStream_t st) {
+  GemmArgs ga{};
+  ga.g = g;
+  ga.ctx = ctx;
+  ga.A = static_cast<const __nv_bfloat16*>(dy);
+  ga.Wt = static_cast<const __nv_bfloat16*>(WprojT);
+  ga.bias = static_cast<const __nv_bfloat16*>(zero_bias);
+  ga.dst = static_cast<__nv_bfloat16*>(dO);
+  ga.win0 = win0;
+  ga.rows = nwin * g.N;
+  ga.K = g.C;
+  ga.Ntot = g.C;
+  ga.BN = pick_bn(g.C);
+  ga.qscale = 1.0f;
+  ga.slab.qrows = g.Npad;  // one q-layout slab per (window, head)
+  ga.slab.kvrows = 0;
+  ga.slab.kv8 = 0;
+  ga.rowsrc = rowsrc;
+  if (ga.BN == 0) return cudaErrorInvalidValue;
+  return launch_gemm<kQKV, false>(ga, st);
+}
+
+cudaError_t launch_bf16_dx(const Geom& g, const KernelCtx& ctx, const void* dqkv, const void* WqkvT,
+                           const void* zero_bias, void* dx, const int* rowsrc, long long win0, long long nwin,
+                           cudaStream_t st) {
+  GemmArgs gp{};
+  gp.g = g;
+  gp.ctx = ctx;
+  gp.A = static_cast<const __nv_bfloat16*>(dqkv);
+  gp.lda = 3LL * g.C;
+  gp.Wt = static_cast<const __nv_bfloat16*>(WqkvT);
+  gp.bias = static_cast<const __nv_bfloat16*>(zero_bias);
+  gp.dst = static_cast<__nv_bfloat16*>(dx);
+  gp.win0 = win0;
+  gp.rows = nwin * g.N;
+  gp.K = 3 * g.C;
+  gp.Ntot = g.C;
+  gp.BN = pick_bn(g.C);
+  gp.qscale = 1.0f;
+  gp.slab = slab_layout(g);
+  gp.rowsrc = rowsrc;
+  if (gp.BN == 0) return cudaErrorInvalidValue;
   return launch_gemm<kPROJ, false>(gp, st);
 }
 

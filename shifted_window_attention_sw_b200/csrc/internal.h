@@ -26,7 +26,7 @@ void count_launch(int n = 1);
 // Optional per-kernel CUDA-event timing (vswin_profile_enable).
 void prof_begin(int kind, cudaStream_t st);
 void prof_end(int kind, cudaStream_t st);
-enum { kKindQkv = 0, kKindAttn = 1, kKindProj = 2, kKindOther = 3, kKindMlp = 4, kKinds = 5 };
+enum { kKindQkv = 0, kKindAttn = 1, kKindProj = 2, kKindOther = 3, kKindMlp = 4, kKindAttnBwd = 5, kKinds = 6 };
 
 // fp32 path (simt_path.cu)
 cudaError_t launch_f32_forward(const Geom& g, const float* x, const float* Wqkv, const float* bqkv,
@@ -65,10 +65,49 @@ cudaError_t launch_ln_fold(const Geom& g, const void* gamma, const void* beta, c
 size_t bf16_block_scratch_bytes(const Geom& g, long long nwin);
 // One chunk of windows; `fuse` null for the plain layer, else the fused block
 // (x is then also the residual, and out may be x itself).
+// With Wproj null only the first three steps run (row table, q / k / v slabs,
+// attention output o); attn_stats (only for (P,7,7) windows), when given,
+// receives each (slot, head) row's softmax reference and sum (exp2 domain).
 cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
                               const void* bqkv, const void* Wproj, const void* bproj, const void* table,
                               void* out, void* scratch, long long win0, long long nwin, cudaStream_t st,
-                              const BlockFuse* fuse = nullptr);
+                              const BlockFuse* fuse = nullptr, float2* attn_stats = nullptr);
+// Chunk scratch of launch_bf16_chunk: q / k / v slabs at 0, the attention
+// output o ([nwin * N][C] bf16) and the row table (int per slot) at these offsets.
+size_t bf16_chunk_o_offset(const Geom& g, long long nwin);
+size_t bf16_chunk_rows_offset(const Geom& g, long long nwin);
+// Slab rows of the bf16 path: q rows, k / v rows, and whether keys are stored
+// as 8-row lines of 7 keys (slot n at row (n / 7) * 8 + n % 7).
+void bf16_slab_rows(const Geom& g, int* qrows, int* kvrows, int* kv8);
+// dO slabs for the backward: dy rows gathered through the row table times
+// WprojT ([C][C], Wproj transposed), one q-layout slab (Npad rows x 32) per
+// (window, head), no bias (zero_bias: C zeros) and no scale.
+cudaError_t launch_bf16_dout_slabs(const Geom& g, const KernelCtx& ctx, const void* dy, const void* WprojT,
+                                   const void* zero_bias, void* dO, const int* rowsrc, long long win0,
+                                   long long nwin, cudaStream_t st);
+// dx for the backward: dqkv rows ([nwin * N][3C] bf16) times WqkvT ([3C][C]),
+// scattered to the tokens through the row table (padding slots dropped).
+cudaError_t launch_bf16_dx(const Geom& g, const KernelCtx& ctx, const void* dqkv, const void* WqkvT,
+                           const void* zero_bias, void* dx, const int* rowsrc, long long win0, long long nwin,
+                           cudaStream_t st);
+
+// bf16 backward (backward_bf16.cu): gradients of x (bf16) and of Wqkv, bqkv,
+// Wproj, bproj and the table (fp32, overwritten) for output gradient dy (bf16),
+// windows processed `chunk` at a time in scratch of
+// bf16_backward_scratch_bytes(g, chunk).
+bool bf16_backward_supported(const Geom& g);
+size_t bf16_backward_scratch_bytes(const Geom& g, long long chunk);
+cudaError_t launch_bf16_backward(const Geom& g, const KernelCtx& ctx, const void* x, const void* Wqkv,
+                                 const void* bqkv, const void* Wproj, const void* table, const void* dy, void* dx,
+                                 float* dWqkv, float* dbqkv, float* dWproj, float* dbproj, float* dtable,
+                                 void* scratch, long long chunk, cudaStream_t st);
+// fp32 sums over rows of bf16 inputs (backward_f32.cu): out[m][n] += sum_r
+// A[arow(r)][m] B[brow(r)][n] for m < M, and bias_out[n] += sum_r B[brow(r)][n]
+// (rows whose brow < 0 read zeros; arow < 0 reads zeros but still counts for
+// the bias). arow(r) = a_src ? a_src[r] : r, likewise brow.
+cudaError_t launch_gram_bf16(long long rows, int M, int N, const void* A, long long lda, const int* a_src,
+                             const void* B, long long ldb, const int* b_src, float* out, float* bias_out,
+                             cudaStream_t st);
 
 // MLP half of a block (mlp_path.cu): out = x + GELU(LN(x) W1 + b1) W2 + b2 for
 // M tokens of C channels, one fused persistent kernel. out may be x.

@@ -633,6 +633,62 @@ int vswin_wmsa_backward_f32(const void* x, int B, int T, int H, int W, int C, in
   return VSWIN_OK;
 }
 
+int vswin_wmsa_backward(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
+                        const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
+                        const void* bias_table, const void* dy, void* dx, void* dWqkv, void* dbqkv, void* dWproj,
+                        void* dbproj, void* dtable, void* stream) {
+  Geom g;
+  int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
+  if (st != VSWIN_OK) return st;
+  const void* ptrs[] = {x, Wqkv, bqkv, Wproj, bproj, bias_table, dy, dx, dWqkv, dbqkv, dWproj, dbproj, dtable};
+  const char* names[] = {"x", "Wqkv", "bqkv", "Wproj", "bproj", "bias_table", "dy",
+                         "dx", "dWqkv", "dbqkv", "dWproj", "dbproj", "dtable"};
+  // bf16 activations and x rows are read 16 bytes at a time; bf16 vectors and
+  // the table element-wise; the fp32 gradients element-wise
+  const size_t align[] = {16, 2, 2, 2, 2, 2, 16, 16, 4, 4, 4, 4, 4};
+  for (int k = 0; k < 13; ++k) {
+    if (!ptrs[k]) return fail(VSWIN_ERR_INVALID_ARG, "%s is NULL", names[k]);
+    if (!aligned(ptrs[k], align[k]))
+      return fail(VSWIN_ERR_INVALID_ARG, "%s is not %zu-byte aligned", names[k], align[k]);
+  }
+  const size_t act = (size_t)g.tokens * g.C * 2;
+  const size_t wq = (size_t)g.C * 3 * g.C, wp = (size_t)g.C * g.C;
+  const size_t tb = (size_t)g.table_rows * g.heads;
+  const void* outs[] = {dx, dWqkv, dbqkv, dWproj, dbproj, dtable};
+  const size_t out_n[] = {act, wq * 4, (size_t)3 * g.C * 4, wp * 4, (size_t)g.C * 4, tb * 4};
+  const void* ins[] = {x, dy, Wqkv, bqkv, Wproj, bproj, bias_table};
+  const size_t in_n[] = {act, act, wq * 2, (size_t)3 * g.C * 2, wp * 2, (size_t)g.C * 2, tb * 2};
+  for (int a = 0; a < 6; ++a) {
+    for (int b = 0; b < 7; ++b)
+      if (overlap(outs[a], out_n[a], ins[b], in_n[b]))
+        return fail(VSWIN_ERR_INVALID_ARG, "gradient buffer %s overlaps an input", names[7 + a]);
+    for (int b = a + 1; b < 6; ++b)
+      if (overlap(outs[a], out_n[a], outs[b], out_n[b]))
+        return fail(VSWIN_ERR_INVALID_ARG, "gradient buffers %s and %s overlap", names[7 + a], names[7 + b]);
+  }
+  if (!bf16_backward_supported(g))
+    return fail(VSWIN_ERR_UNSUPPORTED,
+                "bf16 backward needs head width 32, C %% 32 == 0 and a (P,7,7) window with P in {1,2,4,8} "
+                "(d = %d, C = %d, window (%d,%d,%d)); the fp32 backward covers the rest",
+                g.d, g.C, g.win[0], g.win[1], g.win[2]);
+  KernelCtx ctx;
+  st = make_ctx(&ctx);
+  if (st != VSWIN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long chunk = chunk_windows(g);
+  void* scratch = nullptr;
+  st = scratch_alloc(&scratch, bf16_backward_scratch_bytes(g, chunk), s);
+  if (st != VSWIN_OK) return st;
+  cudaError_t e = launch_bf16_backward(g, ctx, x, Wqkv, bqkv, Wproj, bias_table, dy, dx,
+                                       static_cast<float*>(dWqkv), static_cast<float*>(dbqkv),
+                                       static_cast<float*>(dWproj), static_cast<float*>(dbproj),
+                                       static_cast<float*>(dtable), scratch, chunk, s);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) return fail_cuda(e, "bf16 backward launch");
+  if (e2 != cudaSuccess) return fail_cuda(e2, "cudaFreeAsync");
+  return VSWIN_OK;
+}
+
 int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads, const int* window,
                             const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                             const void* bproj, const void* bias_table, void* out_host, void* stream) {

@@ -36,12 +36,13 @@ EXPORTS = (
     "vswin_set_exact_softmax",
     "vswin_block_msa_forward",
     "vswin_wmsa_backward_f32",
+    "vswin_wmsa_backward",
     "vswin_mlp_forward",
     "vswin_block_forward",
     "vswin_patch_merge_forward",
 )
 
-KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other", "mlp")
+KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other", "mlp", "attention_bwd")
 
 
 class VswinError(RuntimeError):
@@ -74,6 +75,8 @@ def lib():
         L.vswin_block_msa_forward.restype = _I
         L.vswin_wmsa_backward_f32.argtypes = layer[:15] + [_P] * 6 + [_P]  # ..., dy, six gradients, stream
         L.vswin_wmsa_backward_f32.restype = _I
+        L.vswin_wmsa_backward.argtypes = layer[:15] + [_P] * 6 + [_P]
+        L.vswin_wmsa_backward.restype = _I
         L.vswin_mlp_forward.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P,
                                         _P]
         L.vswin_mlp_forward.restype = _I
@@ -308,6 +311,23 @@ def wmsa_backward_f32(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, 
             _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj),
             _ptr(bproj), _ptr(table), _ptr(dy), *[_ptr(o) for o in outs], _stream_handle(stream, x.device)))
     return tuple(outs)
+
+
+def wmsa_backward(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, dy, stream=None):
+    """bf16 backward on the tensor cores: gradients (dx bf16; dWqkv, dbqkv, dWproj, dbproj,
+    dtable float32) of the layer for output gradient ``dy``. Inputs bfloat16 on one CUDA
+    device, as for wmsa_forward."""
+    _prep(x, dict(x=x, Wqkv=Wqkv, bqkv=bqkv, Wproj=Wproj, bproj=bproj, table=table, dy=dy), torch.bfloat16,
+          x.device)
+    _check_shapes(x, window, heads, Wqkv, bqkv, Wproj, bproj, table, dy=dy)
+    dx = torch.empty_like(x)
+    grads = [torch.empty(t.shape, dtype=torch.float32, device=x.device) for t in (Wqkv, bqkv, Wproj, bproj, table)]
+    B, T, H, W, C = x.shape
+    with torch.cuda.device(x.device):
+        _check(lib().vswin_wmsa_backward(
+            _ptr(x), B, T, H, W, C, int(heads), _i3(window), _i3(shift), _ptr(Wqkv), _ptr(bqkv), _ptr(Wproj),
+            _ptr(bproj), _ptr(table), _ptr(dy), _ptr(dx), *[_ptr(t) for t in grads], _stream_handle(stream, x.device)))
+    return (dx, *grads)
 
 
 def wmsa_forward_noalloc(x, window, shift, Wqkv, bqkv, Wproj, bproj, table, heads, out=None, stream=None):

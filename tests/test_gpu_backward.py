@@ -58,3 +58,49 @@ def test_backward_f32(shape, heads, window, shift):
         rel_l2 = np.linalg.norm(err) / max(np.linalg.norm(r), 1e-30)
         rel_max = np.abs(err).max() / max(np.abs(r).max(), 1e-30)
         assert rel_l2 <= REL_L2 and rel_max <= REL_MAX, (name, rel_l2, rel_max)
+
+
+# bf16 backward (vswin_wmsa_backward, tcgen05). Inputs are bf16 values (the oracle
+# gets the same values in float64). The path rounds q, k, v, O, dO, P, dS and dqkv to
+# bf16 (relative 2^-9 = 2e-3 each, independent) and sums in fp32, so a few 1e-3 of
+# relative error per gradient is expected (measured on these cases: relative L2
+# <= 4.5e-3, relative max <= 7e-3). The gates, the forward's bf16 ones widened by half,
+# leave about three times that and sit far below what a wrong sign, index, scale or
+# dropped term gives (order 1).
+BF16_REL_L2, BF16_REL_MAX = 1.5e-2, 3e-2
+BF16_CASES = [
+    # (shape, heads, window, shift)
+    ((1, 8, 14, 14, 96), 3, (8, 7, 7), (4, 3, 3)),     # Swin-T width, shifted
+    ((1, 8, 14, 14, 96), 3, (8, 7, 7), (0, 0, 0)),     # unshifted
+    ((1, 12, 12, 12, 128), 4, (8, 7, 7), (4, 3, 3)),   # padding on every axis
+    ((1, 4, 14, 14, 64), 2, (4, 7, 7), (2, 3, 3)),     # P = 4: two query tiles, two key blocks
+    ((1, 2, 7, 14, 64), 2, (2, 7, 7), (1, 0, 3)),      # P = 2
+    ((2, 1, 14, 21, 64), 2, (1, 7, 7), (0, 3, 3)),     # 2D Swin special case
+]
+
+
+@pytest.mark.parametrize("scale", ["baseline", "sensitivity"])
+@pytest.mark.parametrize("shape,heads,window,shift", BF16_CASES)
+def test_backward_bf16(shape, heads, window, shift, scale):
+    inp = make_layer_inputs(shape, heads, window, "bf16", scale, seed=7200 + sum(shape))
+    dy = torch.randn(*shape, generator=torch.Generator().manual_seed(7300 + sum(shape))).bfloat16()
+    a = inp.as_f64()
+    ref = oracle_backward.backward(a["x"], window, shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"],
+                                   a["table"], heads, dy.double().numpy())
+    d = inp.to("cuda")
+    got = vswin.wmsa_backward(d.x, window, shift, d.Wqkv, d.bqkv, d.Wproj, d.bproj, d.table, heads,
+                              dy.to("cuda"))
+    assert vswin.poll_error() == vswin.OK, vswin.last_error()
+    assert got[0].dtype == torch.bfloat16 and all(t.dtype == torch.float32 for t in got[1:])
+    stats = {}
+    for name, g, r in zip(NAMES, got, ref):
+        g = g.double().cpu().numpy()
+        assert g.shape == r.shape, name
+        assert np.isfinite(g).all(), name
+        err = g - r
+        stats[name] = (np.linalg.norm(err) / max(np.linalg.norm(r), 1e-30),
+                       np.abs(err).max() / max(np.abs(r).max(), 1e-30))
+    print("bf16 backward", shape, window, shift, scale,
+          {k: (float(f"{v[0]:.2e}"), float(f"{v[1]:.2e}")) for k, v in stats.items()})
+    for name, (rel_l2, rel_max) in stats.items():
+        assert rel_l2 <= BF16_REL_L2 and rel_max <= BF16_REL_MAX, (name, rel_l2, rel_max, stats)
