@@ -16,7 +16,7 @@
 //      shared memory. Keys in blocks of 128 (the MMA's M), queries in tiles
 //      of up to 128 (its N); per (key block, query tile):
 //        S^T = K Q^T and dP^T = V dO^T on tcgen05 into TMEM (fp32);
-//        eight warps (TMEM lane = key) rebuild P^T = 2^(S^T + B - m) / l from
+//        sixteen warps (TMEM lane = key) rebuild P^T = 2^(S^T + B - m) / l from
 //        the saved statistics and form dS^T = P^T (dP^T - D), both written
 //        back to TMEM as bf16 over their own scores, dS^T also to shared
 //        memory (the MN-major A operand of dq), and the table gradient summed
@@ -32,9 +32,10 @@
 //
 // TMEM columns of the attention CTA: S^T / P^T [0, 128), dP^T / dS^T
 // [128, 256), dK [256, 288), dV [288, 320), dQ of query tile t [320 + 32 t,
-// + 32). P^T of queries [0, 64) is packed at columns [0, 32) and of queries
-// [64, 128) at [64, 96) (each half written by its own warps over scores they
-// have read), likewise dS^T.
+// + 32). P^T of queries [32 c, 32 c + 32) is packed at columns [32 c, 32 c +
+// 16) (each quarter written by its own warps over scores they have read),
+// likewise dS^T; the TS MMA's 16-query step k reads columns 32 (k / 2) +
+// 8 (k % 2).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -44,7 +45,7 @@ namespace vswin {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kBwThreads = 256;  // warp w: TMEM lane quarter w % 4, query-column half w / 4
+constexpr int kBwThreads = 512;  // warp w: TMEM lane quarter w % 4, query-column quarter w / 4
 constexpr uint32_t kBwTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDK = 256, kColDV = 288, kColDQ = 320;
 constexpr int kRowBytes = 64;  // one slab row: 32 bf16
@@ -68,6 +69,11 @@ __device__ __forceinline__ bool elect_one() {
       "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
       : "=r"(pred));
   return pred != 0;
+}
+
+// Shared-memory add without a returned value.
+__device__ __forceinline__ void red_add_shared(float* p, float v) {
+  asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hf = warp >> 2;
+  const int qd = warp & 3, cq = warp >> 2;
   const Geom& g = a.g;
   const int C = g.C, C3 = 3 * g.C;
   const long long item = blockIdx.x;
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
     const int kb = s / Wn::QT, qt = s % Wn::QT, nq = nq_of(qt);
     const uint32_t id = idesc_bf16(128, 32, 0, 1);
     for (int ks = 0; ks < nq / 16; ++ks) {
-      const uint32_t acol = (nq == 128 && ks >= 4) ? 64u + 8u * (uint32_t)(ks - 4) : 8u * (uint32_t)ks;
+      const uint32_t acol = 32u * (uint32_t)(ks >> 1) + 8u * (uint32_t)(ks & 1);
       const uint32_t acc = (qt > 0 || ks > 0) ? 1u : 0u;
       umma_ts(tmem + kColDV, tmem + kColS + acol, smem_desc(sdo + qt * 8192 + ks * 1024, 512, 128), id, acc);
       umma_ts(tmem + kColDK, tmem + kColDP + acol, smem_desc(sq + qt * 8192 + ks * 1024, 512, 128), id, acc);
@@ -294,22 +300,23 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
     }
     __syncwarp();
   }
-  // dK / dV of key block kb (this warp: dK for hf 0, dV for hf 1) to dqkv
+  // dK / dV of key block kb to dqkv: column quarter cq of the warp takes dK
+  // (cq 0, 1) or dV (cq 2, 3), 16 channels each
   auto write_kv = [&](int kb) {
     const int n = kb * 128 + qd * 32 + lane;
-    uint32_t u[32];
-    tmem_ld8(tmem + lane_base + (hf ? kColDV : kColDK), *reinterpret_cast<uint32_t(*)[8]>(&u[0]));
-    tmem_ld8(tmem + lane_base + (hf ? kColDV : kColDK) + 8, *reinterpret_cast<uint32_t(*)[8]>(&u[8]));
-    tmem_ld8(tmem + lane_base + (hf ? kColDV : kColDK) + 16, *reinterpret_cast<uint32_t(*)[8]>(&u[16]));
-    tmem_ld8(tmem + lane_base + (hf ? kColDV : kColDK) + 24, *reinterpret_cast<uint32_t(*)[8]>(&u[24]));
+    const bool is_v = cq >= 2;
+    const int c16 = (cq & 1) * 16;
+    uint32_t u[16];
+    tmem_ld8(tmem + lane_base + (is_v ? kColDV : kColDK) + c16, *reinterpret_cast<uint32_t(*)[8]>(&u[0]));
+    tmem_ld8(tmem + lane_base + (is_v ? kColDV : kColDK) + c16 + 8, *reinterpret_cast<uint32_t(*)[8]>(&u[8]));
     tmem_wait_ld();
     const int line = n >> 3, pw = n & 7;
     if (!s_abort && pw < 7 && line < Wn::KLINES) {
       const int slot = line * 7 + pw;
-      const float sc = hf ? 1.0f : 1.0f / kLog2e;  // dk: the slab's q carries log2(e) / sqrt(d)
-      __nv_bfloat16* dst = a.dqkv + (wl * Wn::N + slot) * C3 + (hf ? 2 * C : C) + h * 32;
+      const float sc = is_v ? 1.0f : 1.0f / kLog2e;  // dk: the slab's q carries log2(e) / sqrt(d)
+      __nv_bfloat16* dst = a.dqkv + (wl * Wn::N + slot) * C3 + (is_v ? 2 * C : C) + h * 32 + c16;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
         reinterpret_cast<uint4*>(dst)[c] = make_uint4(
             pack_bf16x2(__uint_as_float(u[8 * c + 0]) * sc, __uint_as_float(u[8 * c + 1]) * sc),
             pack_bf16x2(__uint_as_float(u[8 * c + 2]) * sc, __uint_as_float(u[8 * c + 3]) * sc),
@@ -325,10 +332,9 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
     phase ^= 1;
     tc_fence_after();
     if (qt == 0 && kb > 0) write_kv(kb - 1);  // the previous block's MMAs are complete
-    // this warp's query columns of the tile: both halves of a full tile, else
-    // the first half's warps take all
-    const int c_begin = nq == 128 ? hf * 64 : 0;
-    const int c_end = nq == 128 ? c_begin + 64 : (hf ? 0 : nq);
+    // this warp's query columns of the tile: its quarter, cut at nq
+    const int c_begin = cq * 32;
+    const int c_end = c_begin + 32 < nq ? c_begin + 32 : nq;
     const int j = qd * 32 + lane;
     const int2 kinfo = sKI[kb * 128 + j];
     const int ebase = Wn::E0 - kinfo.x;
@@ -349,7 +355,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
           const float d = pr * (__uint_as_float(ud[cc]) - qi.z);
           p[cc] = pr;
           ds[cc] = d;
-          if (ok) atomicAdd(&sG[r], d);
+          if (ok) red_add_shared(&sG[r], d);
         }
         const uint32_t pp[4] = {pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
                                 pack_bf16x2(p[6], p[7])};
@@ -379,8 +385,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
   if (!s_abort && !mbar_wait(mma_done, phase, a.ctx.err, kErrBwMma, lim)) s_abort = 1;
   tc_fence_after();
   write_kv(Wn::NKB - 1);
-  // dQ of the query tiles (this warp: tiles 2 hf, 2 hf + 1)
-  for (int qt = 2 * hf; qt < 2 * hf + 2 && qt < Wn::QT; ++qt) {
+  // dQ of the query tiles (this warp: tile cq)
+  for (int qt = cq; qt < cq + 1 && qt < Wn::QT; ++qt) {
     uint32_t u[32];
     const uint32_t col = kColDQ + 32u * (uint32_t)qt;
     tmem_ld8(tmem + lane_base + col, *reinterpret_cast<uint32_t(*)[8]>(&u[0]));
@@ -418,6 +424,199 @@ cudaError_t launch_bwd_attn(const BwdArgs& a, cudaStream_t st) {
   prof_begin(kKindAttnBwd, st);
   bwd_attn_kernel<Wn><<<(unsigned)items, kBwThreads, Wn::SMEM, st>>>(a);
   prof_end(kKindAttnBwd, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Weight-gradient sums on tcgen05: out[m][n] += sum_r A(r, m) B(r, n) for m < M
+// and bias_out[n] += sum_r B(r, n), over the rows r of the grid's split, with
+// A(r, m) = A[arow(r) lda + m], B(r, n) = B[brow(r) ldb + n] (bf16; a negative
+// row reads zeros; arow(r) = a_src ? a_src[r] : r, likewise brow). The MMA is
+// D[128 x BN] += A^T B: M = the M columns of A plus a column of ones (the bias
+// row) and zeros up to 128, N = BN output columns, K = rows, 16 at a time.
+// Both operands are MN-major in shared memory (8 rows x 16 bytes per core
+// matrix; A: 128 B between column groups, 2 KB between row groups; B: 128 B,
+// BN x 16 B). 128 threads gather 64-row tiles with cp.async into four stages
+// (each thread's copies arrive on the stage's barrier), thread 0 issues the
+// MMAs; at the end each thread adds its accumulator row to out with atomics.
+constexpr int kGrThreads = 128;
+constexpr int kGrRows = 64;    // rows per tile
+constexpr int kGrStages = 4;
+constexpr int kGrABytes = kGrRows * 128 * 2;  // 16 KB
+
+__host__ __device__ inline int gram_b_bytes(int BN) { return kGrRows * BN * 2; }
+__host__ inline int gram_smem_bytes(int BN) { return kGrStages * (kGrABytes + gram_b_bytes(BN)) + 128; }
+
+struct GramArgs {
+  KernelCtx ctx;
+  long long rows, rows_per_split;  // rows of the sum, rows per CTA (multiple of 64)
+  int M, N, BN;
+  const __nv_bfloat16* A;
+  long long lda;
+  const int* a_src;
+  const __nv_bfloat16* B;
+  long long ldb;
+  const int* b_src;
+  float* out;
+  float* bias_out;
+};
+
+__global__ void __launch_bounds__(kGrThreads, 1) gram_tc_kernel(GramArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int BN = a.BN;
+  uint8_t* sA = smem;                                    // [stages][16 KB]
+  uint8_t* sB = smem + kGrStages * kGrABytes;            // [stages][64 x BN x 2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kGrStages * gram_b_bytes(BN));
+  uint64_t* empty = full + kGrStages;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(empty + kGrStages);
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * BN;
+  const long long r_begin = (long long)blockIdx.y * a.rows_per_split;
+  long long r_end = r_begin + a.rows_per_split;
+  if (r_end > a.rows) r_end = a.rows;
+  const long long ntiles = r_end > r_begin ? (r_end - r_begin + kGrRows - 1) / kGrRows : 0;
+  const uint64_t lim = a.ctx.wait_limit;
+  const uint32_t tcols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+
+  if (tid == 0) {
+    for (int k = 0; k < kGrStages; ++k) {
+      mbar_init(&full[k], kGrThreads);
+      mbar_init(&empty[k], 1);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  // the constant columns of A in every stage: ones at column M, zeros after
+  for (int k = tid; k < kGrStages * kGrRows * (16 - a.M / 8); k += kGrThreads) {
+    const int st = k / (kGrRows * (16 - a.M / 8)), rem = k % (kGrRows * (16 - a.M / 8));
+    const int r = rem / (16 - a.M / 8), mg = a.M / 8 + rem % (16 - a.M / 8);
+    const uint4 v = make_uint4(mg * 8 == a.M ? 0x3F80u : 0u, 0u, 0u, 0u);  // bf16 1.0 in the low half
+    *reinterpret_cast<uint4*>(sA + st * kGrABytes + (r >> 3) * 2048 + mg * 128 + (r & 7) * 16) = v;
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(s_tmem, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  auto load_tile = [&](long long t) {
+    const int st = (int)(t % kGrStages);
+    const long long rt = r_begin + t * kGrRows;
+    uint8_t* dA = sA + st * kGrABytes;
+    uint8_t* dB = sB + st * gram_b_bytes(BN);
+    const int ag = a.M / 8, bg = BN / 8;
+    for (int k = tid; k < kGrRows * ag; k += kGrThreads) {
+      const int r = k / ag, mg = k % ag;
+      const long long row = rt + r;
+      long long src = -1;
+      if (row < r_end) src = a.a_src ? (long long)a.a_src[row] : row;
+      cp_async_16(dA + (r >> 3) * 2048 + mg * 128 + (r & 7) * 16, a.A + (src < 0 ? 0 : src * a.lda) + mg * 8,
+                  src < 0 ? 0u : 16u);
+    }
+    for (int k = tid; k < kGrRows * bg; k += kGrThreads) {
+      const int r = k / bg, ng = k % bg;
+      const long long row = rt + r;
+      long long src = -1;
+      if (row < r_end) src = a.b_src ? (long long)a.b_src[row] : row;
+      cp_async_16(dB + (r >> 3) * (BN * 16) + ng * 128 + (r & 7) * 16,
+                  a.B + (src < 0 ? 0 : src * a.ldb) + n0 + ng * 8, src < 0 ? 0u : 16u);
+    }
+    cp_async_mbar_arrive_noinc(&full[st]);
+  };
+
+  const uint32_t id = idesc_bf16(128, BN, 1, 1);
+  for (long long t = 0; t < kGrStages - 1 && t < ntiles; ++t) load_tile(t);
+  for (long long t = 0; t < ntiles; ++t) {
+    const long long tn = t + kGrStages - 1;  // tile to load now, into the stage tile t - 1 used
+    if (tn < ntiles) {
+      if (t >= 1 && !s_abort &&
+          !mbar_wait(&empty[tn % kGrStages], (uint32_t)((tn / kGrStages) - 1) & 1, a.ctx.err, kErrBwMma, lim))
+        s_abort = 1;
+      if (!s_abort) load_tile(tn);
+    }
+    if (tid == 0) {
+      const int st = (int)(t % kGrStages);
+      if (!s_abort && !mbar_wait(&full[st], (uint32_t)(t / kGrStages) & 1, a.ctx.err, kErrBwLoad, lim)) s_abort = 1;
+      fence_proxy_async_smem();
+      tc_fence_after();
+      if (!s_abort) {
+        const uint32_t aa = smem_u32(sA + st * kGrABytes), bb = smem_u32(sB + st * gram_b_bytes(BN));
+        for (int ks = 0; ks < kGrRows / 16; ++ks)
+          umma_ss(tmem, smem_desc(aa + ks * 4096, 2048, 128), smem_desc(bb + ks * 2 * BN * 16, BN * 16, 128), id,
+                  (t > 0 || ks > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty[st]);
+    }
+  }
+  cp_async_wait_all();
+  // wait for the last tile's MMAs (its stage's empty barrier)
+  if (ntiles > 0) {
+    const long long tl = ntiles - 1;
+    if (!s_abort && !mbar_wait(&empty[tl % kGrStages], (uint32_t)(tl / kGrStages) & 1, a.ctx.err, kErrBwMma, lim))
+      s_abort = 1;
+  }
+  tc_fence_after();
+  // thread = accumulator row m (TMEM lane), BN columns
+  const int m = warp * 32 + lane;
+  if (ntiles > 0 && !s_abort) {
+    for (int c0 = 0; c0 < BN; c0 += 8) {
+      uint32_t u[8];
+      tmem_ld8(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, u);
+      tmem_wait_ld();
+      float* dst = m < a.M ? a.out + (size_t)m * a.N + n0 + c0 : (m == a.M ? a.bias_out + n0 + c0 : nullptr);
+      if (dst)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) atomicAdd(dst + k, __uint_as_float(u[k]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, tcols);
+}
+
+// Chooses the split so that every SM gets a CTA or two.
+cudaError_t launch_gram_tc(const KernelCtx& ctx, long long rows, int M, int N, const void* A, long long lda,
+                           const int* a_src, const void* B, long long ldb, const int* b_src, float* out,
+                           float* bias_out, cudaStream_t st) {
+  int BN = N;
+  if (BN > 256 || BN % 16 != 0) {
+    BN = 0;
+    for (int bn = 256; bn >= 16; bn -= 16)
+      if (N % bn == 0) {
+        BN = bn;
+        break;
+      }
+  }
+  if (BN == 0 || M % 8 != 0 || M + 1 > 128) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntile = N / BN;
+  long long splits = (sms + ntile - 1) / ntile;
+  long long per = (rows + splits - 1) / splits;
+  per = (per + kGrRows - 1) / kGrRows * kGrRows;
+  splits = (rows + per - 1) / per;
+  if (splits < 1) splits = 1;
+  if (splits > 65535) return cudaErrorInvalidConfiguration;
+  GramArgs ga{};
+  ga.ctx = ctx;
+  ga.rows = rows;
+  ga.rows_per_split = per;
+  ga.M = M, ga.N = N, ga.BN = BN;
+  ga.A = static_cast<const __nv_bfloat16*>(A), ga.lda = lda, ga.a_src = a_src;
+  ga.B = static_cast<const __nv_bfloat16*>(B), ga.ldb = ldb, ga.b_src = b_src;
+  ga.out = out, ga.bias_out = bias_out;
+  const int smem = gram_smem_bytes(BN);
+  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  prof_begin(kKindOther, st);
+  gram_tc_kernel<<<dim3((unsigned)ntile, (unsigned)splits), kGrThreads, smem, st>>>(ga);
+  prof_end(kKindOther, st);
   count_launch();
   return cudaGetLastError();
 }
@@ -544,11 +743,16 @@ cudaError_t launch_bf16_backward(const Geom& g, const KernelCtx& ctx, const void
     e = launch_bf16_dx(g, ctx, dqkv, wqkvT, zero_bias, dx, rowsrc, w0, nwin, st);
     if (e != cudaSuccess) return e;
     const long long rows = nwin * g.N;
-    // dWqkv = X^T dqkv (X gathered), dbqkv over every slot (padding included)
-    e = launch_gram_bf16(rows, C, 3 * C, x, C, rowsrc, dqkv, 3 * C, nullptr, dWqkv, dbqkv, st);
+    // dWqkv = X^T dqkv (X gathered), dbqkv over every slot (padding included);
+    // dWproj = O^T dY (dY gathered, zero on padding), dbproj over real slots. On
+    // tcgen05 when the C columns and the bias row fit one 128-row tile, else the
+    // FP32 sums.
+    const bool tc = C + 1 <= 128;
+    e = tc ? launch_gram_tc(ctx, rows, C, 3 * C, x, C, rowsrc, dqkv, 3 * C, nullptr, dWqkv, dbqkv, st)
+           : launch_gram_bf16(rows, C, 3 * C, x, C, rowsrc, dqkv, 3 * C, nullptr, dWqkv, dbqkv, st);
     if (e != cudaSuccess) return e;
-    // dWproj = O^T dY (dY gathered, zero on padding), dbproj over real slots
-    e = launch_gram_bf16(rows, C, C, o, C, nullptr, dy, C, rowsrc, dWproj, dbproj, st);
+    e = tc ? launch_gram_tc(ctx, rows, C, C, o, C, nullptr, dy, C, rowsrc, dWproj, dbproj, st)
+           : launch_gram_bf16(rows, C, C, o, C, nullptr, dy, C, rowsrc, dWproj, dbproj, st);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
