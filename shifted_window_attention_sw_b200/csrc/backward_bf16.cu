@@ -338,12 +338,22 @@ __global__ void __launch_bounds__(kBwThreads, 1) bwd_attn_kernel(BwdArgs a) {
     const int j = qd * 32 + lane;
     const int2 kinfo = sKI[kb * 128 + j];
     const int ebase = Wn::E0 - kinfo.x;
-    if (!s_abort) {
-      for (int c0 = c_begin; c0 < c_end; c0 += 8) {
-        uint32_t us[8], ud[8];
-        tmem_ld8(tmem + lane_base + kColS + c0, us);
-        tmem_ld8(tmem + lane_base + kColDP + c0, ud);
-        tmem_wait_ld();
+    if (!s_abort && c_begin < c_end) {
+      // all of this warp's scores and dP first (one wait), then 8 columns at a time
+      uint32_t us_all[32], ud_all[32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (c_begin + 8 * k < c_end) {
+          tmem_ld8(tmem + lane_base + kColS + c_begin + 8 * k, *reinterpret_cast<uint32_t(*)[8]>(&us_all[8 * k]));
+          tmem_ld8(tmem + lane_base + kColDP + c_begin + 8 * k, *reinterpret_cast<uint32_t(*)[8]>(&ud_all[8 * k]));
+        }
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c0 = c_begin + 8 * k;
+        if (c0 >= c_end) break;
+        const uint32_t* us = &us_all[8 * k];
+        const uint32_t* ud = &ud_all[8 * k];
         float p[8], ds[8];
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {

@@ -104,3 +104,38 @@ def test_backward_bf16(shape, heads, window, shift, scale):
           {k: (float(f"{v[0]:.2e}"), float(f"{v[1]:.2e}")) for k, v in stats.items()})
     for name, (rel_l2, rel_max) in stats.items():
         assert rel_l2 <= BF16_REL_L2 and rel_max <= BF16_REL_MAX, (name, rel_l2, rel_max, stats)
+
+
+def test_backward_bf16_chunked(tmp_path):
+    """Windows in several chunks (a 1 MB scratch budget: three windows a chunk, the
+    second chunk starting inside a clip) give the same gradients within the gates."""
+    import subprocess
+    import sys
+
+    shape, heads, window, shift = (2, 8, 14, 14, 96), 3, (8, 7, 7), (4, 3, 3)
+    out = tmp_path / "grads.pt"
+    code = f"""
+import torch
+from shifted_window_attention_sw_b200 import vswin
+from shifted_window_attention_sw_b200.inputs import make_layer_inputs
+inp = make_layer_inputs({shape}, {heads}, {window}, "bf16", "sensitivity", seed=7400).to("cuda")
+dy = torch.randn(*{shape}, generator=torch.Generator().manual_seed(7401)).bfloat16().cuda()
+g = vswin.wmsa_backward(inp.x, {window}, {shift}, inp.Wqkv, inp.bqkv, inp.Wproj, inp.bproj, inp.table, {heads}, dy)
+assert vswin.poll_error() == vswin.OK, vswin.last_error()
+torch.save([t.cpu() for t in g], {str(out)!r})
+"""
+    env = dict(__import__("os").environ, VSWIN_CHUNK_MB="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    got = torch.load(out)
+    inp = make_layer_inputs(shape, heads, window, "bf16", "sensitivity", seed=7400)
+    dy = torch.randn(*shape, generator=torch.Generator().manual_seed(7401)).bfloat16()
+    a = inp.as_f64()
+    ref = oracle_backward.backward(a["x"], window, shift, a["Wqkv"], a["bqkv"], a["Wproj"], a["bproj"],
+                                   a["table"], heads, dy.double().numpy())
+    for name, g, r in zip(NAMES, got, ref):
+        g = g.double().numpy()
+        err = g - r
+        rel_l2 = np.linalg.norm(err) / max(np.linalg.norm(r), 1e-30)
+        rel_max = np.abs(err).max() / max(np.abs(r).max(), 1e-30)
+        assert rel_l2 <= BF16_REL_L2 and rel_max <= BF16_REL_MAX, (name, rel_l2, rel_max)
