@@ -115,6 +115,7 @@ struct GemmArgs {
   const float* ln_bias;
   const __nv_bfloat16* resid;
   long long lda;  // A row stride in elements (0: C)
+  float ln_eps;   // fused pre-norm in the persistent QKV GEMM: statistics computed in the kernel
 };
 
 __host__ __device__ constexpr int gemm_smem_bytes() {
@@ -349,10 +350,16 @@ constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
 constexpr int kWsMaxBBytes = 96 * 1024;
 
 __host__ __device__ inline int ws_a_bytes(int K) { return kBM * K * 2; }
+constexpr int kWsStatSlots = 8;  // fused pre-norm: tiles of row statistics in flight
+constexpr int kWsResSlots = 3;   // fused residual: tiles of residual rows in flight
+__host__ __device__ inline int ws_res_row_bytes(int BN) { return BN * 2 + 16; }  // padded row of a residual tile
 // B slice, A stages, bias (BN floats), column-group table (BN / 8 x 16 B), with
-// the fused pre-norm the column sums and folded bias (2 x BN floats), barriers
-__host__ __device__ inline int ws_smem_bytes(int K, int BN, int stages, bool ln = false) {
-  return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + (ln ? BN * 8 : 0) + 256;
+// the fused pre-norm the column sums and folded bias (2 x BN floats), barriers,
+// with the fused pre-norm a ring of per-row statistics (8 tiles x 128 rows), with
+// the fused residual a ring of residual tiles (3 x 128 rows of the BN columns)
+__host__ __device__ inline int ws_smem_bytes(int K, int BN, int stages, bool ln = false, bool resid = false) {
+  return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + (ln ? BN * 8 + kWsStatSlots * kBM * 8 : 0) +
+         (resid ? kWsResSlots * kBM * ws_res_row_bytes(BN) : 0) + 256;
 }
 
 // Destination facts of one group of 8 output columns of the QKV GEMM: element
@@ -534,7 +541,15 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   uint64_t* a_free = a_full + STAGES;      // [STAGES]
   uint64_t* acc_full = a_free + STAGES;    // [2]
   uint64_t* acc_free = acc_full + 2;       // [2]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(acc_free + 2);
+  uint64_t* stats_full = acc_free + 2;     // kLn: [kWsStatSlots] a tile's row statistics written
+  uint64_t* res_full = stats_full + (kLn ? kWsStatSlots : 0);  // kResid: [kWsResSlots] residual tile landed
+  uint64_t* res_free = res_full + (kResid ? kWsResSlots : 0);  // kResid: [kWsResSlots] residual tile read
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(res_free + (kResid ? kWsResSlots : 0));
+  // kLn: (-mean * rstd, rstd) per row of a tile, (0, 0) for padding rows, slot t % 8
+  float2* sStats = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  // kResid: the residual rows of a tile (BN columns, padded rows), slot t % 3
+  uint8_t* sRes = reinterpret_cast<uint8_t*>(bars) + 256;
+  const int res_slot_bytes = kBM * ws_res_row_bytes(BN);
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -565,6 +580,13 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       mbar_init(&acc_full[k], 1);
       mbar_init(&acc_free[k], kWsEpiWarps);
     }
+    if (kLn)
+      for (int k = 0; k < kWsStatSlots; ++k) mbar_init(&stats_full[k], kProdThreads);
+    if (kResid)
+      for (int k = 0; k < kWsResSlots; ++k) {
+        mbar_init(&res_full[k], kProdThreads);
+        mbar_init(&res_free[k], kWsEpiWarps);
+      }
     fence_mbar_init();
     s_abort = 0;
   }
@@ -621,7 +643,39 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     auto row_tok = [&](long long m, int grp) -> int {
       const long long r = m * kBM + warp * 32 + grp * 8 + sub;
       if (m >= mtiles || r >= a.rows) return -1;
-      return MODE == kQKV ? a.rowsrc[r] : (int)r;
+      return (MODE == kQKV || kResid) ? a.rowsrc[r] : (int)r;
+    };
+    // kLn: the layer norm's statistics of tile t's rows (thread p: row p), from
+    // the gathered bf16 values once they have landed -- one pass of sums and
+    // sums of squares (fp32, two channels per instruction), the biased variance
+    // E[x^2] - mean^2 and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
+    // definition); (0, 0) for padding rows and rows past the end.
+    auto tile_stats = [&](long long m, long long t) {
+      const int s = (int)(t % STAGES);
+      const long long r = m * kBM + tid;
+      const int tk = (m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
+      if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      float2 stv = make_float2(0.f, 0.f);
+      if (tk >= 0 && !s_abort) {
+        const uint8_t* row = sA + s * ws_a_bytes(K) + (tid >> 3) * sboA + (tid & 7) * 16;
+        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+        for (int kc = 0; kc < K / 8; ++kc) {
+          const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 128);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(h2[k]);
+            s1 = __fadd2_rn(s1, f);
+            s2 = __ffma2_rn(f, f, s2);
+          }
+        }
+        const float mean = (s1.x + s1.y) / (float)K;
+        const float var = fmaxf((s2.x + s2.y) / (float)K - mean * mean, 0.f);
+        const float rstd = 1.0f / sqrtf(var + a.ln_eps);
+        stv = make_float2(-mean * rstd, rstd);
+      }
+      sStats[(t % kWsStatSlots) * kBM + tid] = stv;
+      mbar_arrive(&stats_full[t % kWsStatSlots]);
     };
     // Three register sets in rotation: the set of tile t is refilled with tile
     // t + 3's rows right after its copies are issued, so no instruction reads a
@@ -645,15 +699,38 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       for (int grp = 0; grp < 4; ++grp) {
         const int row = warp * 32 + grp * 8 + sub;
         uint8_t* drow = dA + (row >> 3) * sboA + (row & 7) * 16;
-        const int tk = tok[grp];
-        const long long sg = tk < 0 ? 0 : (long long)tk * lda;
+        // QKV: the row's source token; the fused projection's table holds the
+        // residual's token, its A row is the chunk row itself
+        long long src = tok[grp];
+        if (kResid) {
+          const long long rA = m * kBM + row;
+          src = (m < mtiles && rA < a.rows) ? rA : -1;
+        }
+        const long long sg = src < 0 ? 0 : src * lda;
         for (int kc = cq; kc < K / 8; kc += 4)
-          cp_async_16(drow + kc * 128, a.A + sg + kc * 8, tk < 0 ? 0u : 16u);
+          cp_async_16(drow + kc * 128, a.A + sg + kc * 8, src < 0 ? 0u : 16u);
       }
       cp_async_mbar_arrive_noinc(&a_full[s]);  // arrives once this thread's copies have landed
+      if (kResid) {
+        // the tile's residual rows (x at the output tokens, this CTA's columns)
+        const int rs = (int)(t % kWsResSlots);
+        if (t >= kWsResSlots && !s_abort &&
+            !mbar_wait(&res_free[rs], (uint32_t)((t / kWsResSlots) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+          s_abort = 1;
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+          const int row = warp * 32 + grp * 8 + sub;
+          const int tk = tok[grp];
+          uint8_t* drow = sRes + rs * res_slot_bytes + row * ws_res_row_bytes(BN);
+          const __nv_bfloat16* srow = a.resid + (tk < 0 ? 0 : (long long)tk * g.C) + n0;
+          for (int kc = cq; kc < BN / 8; kc += 4) cp_async_16(drow + kc * 16, srow + kc * 8, tk < 0 ? 0u : 16u);
+        }
+        cp_async_mbar_arrive_noinc(&res_full[rs]);
+      }
       if (tid == 0) VSWIN_TRACE_EVENT(kTraceG + 0, trace_n, 51);
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) tok[grp] = row_tok(m + 3 * m_step, grp);
+      if (kLn && t > 0) tile_stats(m - m_step, t - 1);  // the previous tile has landed by now
     };
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += 3 * m_step, t += 3) {
@@ -662,6 +739,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       tile(m + m_step, t + 1, tokB);
       if (m + 2 * m_step >= mtiles) break;
       tile(m + 2 * m_step, t + 2, tokC);
+    }
+    if (kLn) {  // the last tile's statistics
+      long long tl = 0, ml = m_first;
+      for (long long m = m_first; m < mtiles; m += m_step, ++tl) ml = m;
+      if (tl > 0) tile_stats(ml, tl - 1);
     }
     cp_async_wait_all();  // nothing in flight when the CTA ends
   } else if (warp == kWsMmaWarp) {
@@ -712,19 +794,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     // columns handled per TMEM wait (the residual's registers and the norm's
     // extra terms need room)
     constexpr int kCh = kResid ? 48 : kLn ? 72 : 96;
-    // kResid: the residual of this warp's first column chunk, loaded one tile
-    // ahead (the next tile's output row is known a tile early)
+    // kResid: the residual of this warp's column chunk, from the tile's slot
+    // in shared memory (gathered by the producer warps)
     uint4 xr[kResid ? kCh / 8 : 1];
-    auto load_resid = [&](const __nv_bfloat16* xrow, int c0) {
-      const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;
-#pragma unroll
-      for (int j = 0; j < kCh / 8; ++j)
-        xr[j] = (xrow && j * 8 < n) ? *reinterpret_cast<const uint4*>(xrow + c0 + 8 * j) : make_uint4(0, 0, 0, 0);
-    };
-    auto resid_row = [&](int dr) -> const __nv_bfloat16* {
-      return dr >= 0 ? a.resid + (long long)dr * g.C + n0 : nullptr;
-    };
-    if (kResid) load_resid(resid_row(dr_next), hf * cw);
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += m_step, ++t) {
       const int buf = (int)(t & 1);
@@ -735,14 +807,13 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       // this row's destination: QKV, the window's block and the row term of the
       // q slab and of the k / v slabs; projection, the output row
       __nv_bfloat16* rbase = nullptr;
-      const __nv_bfloat16* xres = nullptr;  // kResid: this row's residual, same columns as rbase
       int q_term = 0, kv_term = 0;
       // the last key of a 7-key line also zero-fills the line's eighth (padding)
       // row, so that every 32-byte sector of the k / v slabs is written whole
       // (a partly written sector costs a DRAM read to merge when it leaves L2)
       bool kv_pad = false;
       // kLn: (-mean * rstd, rstd) of this row's token, (0, 0) for a padding row
-      const float2 st = (kLn && row_ok) ? a.ln_stats[r] : make_float2(0.f, 0.f);
+      float2 st = make_float2(0.f, 0.f);
       if (row_ok) {
         if (MODE == kQKV) {
           const int ri = (int)r;  // rows < 2^31 (checked by the caller)
@@ -757,12 +828,20 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
           const long long dr = dr_cur;
           if (dr >= 0) {
             rbase = a.dst + dr * g.C + n0;
-            if (kResid) xres = a.resid + dr * g.C + n0;
           }
         }
       }
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 70);
       if (!s_abort && !mbar_wait(&acc_full[buf], (uint32_t)(t >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+      if (kResid && !s_abort &&
+          !mbar_wait(&res_full[t % kWsResSlots], (uint32_t)(t / kWsResSlots) & 1, a.ctx.err, kErrWaitLoad, lim))
+        s_abort = 1;
+      if (kLn) {  // this tile's row statistics, written by the gathering threads
+        if (!s_abort &&
+            !mbar_wait(&stats_full[t % kWsStatSlots], (uint32_t)(t / kWsStatSlots) & 1, a.ctx.err, kErrWaitLoad, lim))
+          s_abort = 1;
+        st = sStats[(t % kWsStatSlots) * kBM + q * 32 + lane];
+      }
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 71);
       tc_fence_after();
       if (!s_abort && m * kBM + q * 32 < a.rows) {
@@ -770,7 +849,13 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
         for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += kCh) {
           const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;  // a multiple of 8
           uint32_t u[kCh];
-          if (kResid && c0 != hf * cw) load_resid(xres, c0);
+          if (kResid) {
+            const uint8_t* xrow =
+                sRes + (t % kWsResSlots) * res_slot_bytes + (q * 32 + lane) * ws_res_row_bytes(BN) + c0 * 2;
+#pragma unroll
+            for (int j = 0; j < kCh / 8; ++j)
+              if (j * 8 < n) xr[j] = *reinterpret_cast<const uint4*>(xrow + 16 * j);
+          }
           const uint32_t ta = tmem + lane_base + buf * BN + c0;
 #pragma unroll
           for (int j = 0; j < kCh / 8; ++j)
@@ -835,8 +920,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       tc_fence_before();
       __syncwarp();
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 72);
-      if (lane == 0) mbar_arrive(&acc_free[buf]);
-      if (kResid) load_resid(resid_row(dr_next), hf * cw);  // next tile's first chunk
+      if (lane == 0) {
+        mbar_arrive(&acc_free[buf]);
+        if (kResid) mbar_arrive(&res_free[t % kWsResSlots]);
+      }
     }
   }
   tc_fence_before();
@@ -1945,13 +2032,18 @@ int pick_bn(int n) {
   return 0;
 }
 
+// The persistent GEMM runs when its weight slice and two A stages fit in shared
+// memory (227 KB per CTA, 1 KB of it static); otherwise the tiled version (e.g.
+// C = 544: BN = 32 for the projection, two 139 KB A stages).
+bool ws_fits(const GemmArgs& a, bool ln, bool resid = false) {
+  return a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0 &&
+         ws_smem_bytes(a.K, a.BN, 2, ln, resid) <= 226 * 1024;
+}
+
 template <int MODE, bool FUSE>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
-  // persistent version when its weight slice and two A stages fit in shared
-  // memory (227 KB per CTA); otherwise the tiled version (e.g. C = 544: BN = 32
-  // for the projection, two 139 KB A stages)
-  if (a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0 &&
-      ws_smem_bytes(a.K, a.BN, 2, FUSE && MODE == kQKV) <= 227 * 1024) {
+  const bool resid = FUSE && MODE == kPROJ;
+  if (ws_fits(a, FUSE && MODE == kQKV, resid)) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1963,8 +2055,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
     // four A stages when they fit, else two; at least 116 KB so that one CTA
     // (up to 512 TMEM columns) owns each SM
     const bool ln = FUSE && MODE == kQKV;
-    const bool four = ws_smem_bytes(a.K, a.BN, 4, ln) <= 220 * 1024;
-    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2, ln);
+    const bool four = ws_smem_bytes(a.K, a.BN, 4, ln, resid) <= 220 * 1024;
+    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2, ln, resid);
     if (smem_ws < 116 * 1024) smem_ws = 116 * 1024;
     auto kern = four ? gemm_ws_kernel<MODE, 4, FUSE> : gemm_ws_kernel<MODE, 2, FUSE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_ws);
@@ -2032,10 +2124,20 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   float2* stats = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(rowsrc) +
                                             ((size_t)nwin * g.N * 4 + 255) / 256 * 256);
 
+  // fused block: the persistent QKV GEMM computes the norm statistics from the
+  // rows it gathers; the tiled one reads them from row_stats_kernel
+  bool stats_in_gemm = false;
+  if (fuse) {
+    GemmArgs probe{};
+    probe.rowsrc = rowsrc;
+    probe.K = g.C;
+    probe.BN = pick_bn(3 * g.C);
+    stats_in_gemm = probe.BN != 0 && ws_fits(probe, true);
+  }
   {
     const long long rows = nwin * g.N;
     prof_begin(kKindOther, st);
-    if (fuse) {
+    if (fuse && !stats_in_gemm) {
       // one warp per 32 rows, eight warps per block
       long long blocks = (rows + 255) / 256;
       if (blocks > 4096) blocks = 4096;
@@ -2076,6 +2178,7 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
   if (fuse) {
     ga.Wt = static_cast<const __nv_bfloat16*>(fuse->wt);
     ga.ln_stats = stats;
+    ga.ln_eps = fuse->eps;
     ga.ln_colsum = fuse->colsum;
     ga.ln_bias = fuse->bias_ln;
   }
