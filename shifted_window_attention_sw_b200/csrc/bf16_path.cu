@@ -2,16 +2,18 @@
 //
 // Per chunk of windows, four launches:
 //   1. row_source_kernel: the source token of every window slot of the chunk
-//      (roll + pad + partition as index arithmetic; -1 for padding). For the
-//      block entry row_stats_kernel does this and also writes each row's
-//      layer-norm statistics, after ln_fold_kernel has folded gamma and beta
-//      into the QKV weights once per call.
+//      (roll + pad + partition as index arithmetic; -1 for padding). The block
+//      entry first folds gamma and beta into the QKV weights (ln_fold_kernel,
+//      once per call); when the tiled GEMM runs, row_stats_kernel writes the
+//      row table and each row's layer-norm statistics instead.
 //   2. gemm_ws_kernel<kQKV>: persistent warp-specialised tcgen05 GEMM (gather
-//      warps cp.async the rows named by the row table, zero-filling padding;
-//      one MMA warp; epilogue warps). The epilogue adds bqkv, scales q by
-//      log2(e)/sqrt(d) and writes per-(window, head) q / k / v slabs in the
-//      tensor-core operand layout. gemm_kernel<kQKV> is the tiled fallback
-//      used when the persistent kernel's resident weight slice does not fit.
+//      warps cp.async the rows named by the row table, zero-filling padding,
+//      and for the block entry compute each landed row's layer-norm
+//      statistics; one MMA warp; epilogue warps). The epilogue adds bqkv,
+//      scales q by log2(e)/sqrt(d) and writes per-(window, head) q / k / v
+//      slabs in the tensor-core operand layout. gemm_kernel<kQKV> is the tiled
+//      fallback used when the persistent kernel's resident weight slice does
+//      not fit.
 //   3. attention7_kernel: persistent warp-specialised attention for (P,7,7)
 //      windows: S = q k^T on tcgen05 into TMEM with the shifted-window mask
 //      and a per-row reference folded into one extra MMA step, relative-
@@ -20,8 +22,9 @@
 //      other window shapes, one (window, head) per CTA.
 //   4. gemm_ws_kernel<kPROJ> (or gemm_kernel<kPROJ>): the attention output
 //      times Wproj, epilogue adds bproj (and, for the block entry, the
-//      residual) and scatters rows back through the row table (reverse
-//      partition, roll by +shift, drop padding).
+//      residual, which the gather warps copy into shared memory) and scatters
+//      rows back through the row table (reverse partition, roll by +shift,
+//      drop padding).
 //
 // Shared-memory operand layout everywhere: the no-swizzle canonical layout of
 // 8-row x 16-byte core matrices (128 contiguous bytes).
