@@ -341,12 +341,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
 // 128-row A tiles with cp.async into a ring of STAGES buffers (each thread's
 // copies arrive on the stage's mbarrier when they land, so the gatherers only
 // wait for a free stage), warp 4 issues tcgen05.mma into two TMEM
-// accumulators (BN columns each), warps 5..12 drain an accumulator (two warps
-// per TMEM lane quarter, half of the columns each) while the next tile is
+// accumulators (BN columns each), warps 5..16 drain an accumulator (three warps
+// per TMEM lane quarter, a third of the columns each) while the next tile is
 // multiplied. CTA c keeps N-tile c % NT and walks the M-tiles
 // c / NT, c / NT + G / NT, ... (G = grid size, a multiple of NT).
 constexpr int kWsProdWarps = 4;
-constexpr int kWsEpiWarps = 8;
+constexpr int kWsEpiWarps = 12;
 constexpr int kWsMmaWarp = kWsProdWarps;
 constexpr int kWsEpi0 = kWsProdWarps + 1;
 constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
@@ -781,10 +781,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31; the eight epilogue
-    // warps cover each quarter twice, the first four taking the low column half.
+    // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31: three warps per lane
+    // quarter, each taking a third of the columns (whole 8-column groups).
     const int q = warp & 3, hf = (warp - kWsEpi0) >> 2;
-    const int cw = BN / 2;  // columns of this warp (multiple of 8)
+    constexpr int kPerQ = kWsEpiWarps / 4;
+    const int c_lo = (hf * (BN / 8)) / kPerQ * 8, c_hi = ((hf + 1) * (BN / 8)) / kPerQ * 8;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const size_t win_elems = (size_t)g.heads * a.slab.head_elems();  // one window's q / k / v block
     // projection: this row's output row, loaded one tile ahead (the loaded
@@ -796,7 +797,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     int dr_next = out_row(m_first);
     // columns handled per TMEM wait (the residual's registers and the norm's
     // extra terms need room)
-    constexpr int kCh = kResid ? 48 : kLn ? 72 : 96;
+    constexpr int kCh = kResid ? 32 : 48;
     // kResid: the residual of this warp's column chunk, from the tile's slot
     // in shared memory (gathered by the producer warps)
     uint4 xr[kResid ? kCh / 8 : 1];
@@ -849,8 +850,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       tc_fence_after();
       if (!s_abort && m * kBM + q * 32 < a.rows) {
         // all of this warp's columns (up to kCh at a time) loaded before one wait
-        for (int c0 = hf * cw; c0 < (hf + 1) * cw; c0 += kCh) {
-          const int n = (hf + 1) * cw - c0 < kCh ? (hf + 1) * cw - c0 : kCh;  // a multiple of 8
+        for (int c0 = c_lo; c0 < c_hi; c0 += kCh) {
+          const int n = c_hi - c0 < kCh ? c_hi - c0 : kCh;  // a multiple of 8
           uint32_t u[kCh];
           if (kResid) {
             const uint8_t* xrow =
