@@ -568,6 +568,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   const uint32_t sboA = (uint32_t)(K / 8) * 128u;   // A: 8-row group stride
   const uint32_t tcols = BN <= 64 ? 128 : BN <= 128 ? 256 : 512;
   constexpr int kProdThreads = kWsProdWarps * 32;
+  // the fused pre-norm runs eight epilogue warps and four statistics warps,
+  // the others twelve epilogue warps (same block size)
+  constexpr int kEpiWarps = kLn ? 8 : kWsEpiWarps;
+  constexpr int kStatWarps = kLn ? kWsEpiWarps - 8 : 0;
+  constexpr int kStat0 = kWsEpi0 + kEpiWarps;
   constexpr int kTraceG = MODE == kQKV ? 17 : 20;  // trace roles of this GEMM
   int trace_n = 0;
   (void)trace_n;
@@ -577,18 +582,18 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     mbar_init(b_full, kProdThreads);
     for (int k = 0; k < STAGES; ++k) {
       mbar_init(&a_full[k], kProdThreads);  // one asynchronous arrival per gathering thread
-      mbar_init(&a_free[k], 1);
+      mbar_init(&a_free[k], 1 + kStatWarps);  // MMA commit (+ each statistics warp once it has read the stage)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&acc_full[k], 1);
-      mbar_init(&acc_free[k], kWsEpiWarps);
+      mbar_init(&acc_free[k], kEpiWarps);
     }
     if (kLn)
       for (int k = 0; k < kWsStatSlots; ++k) mbar_init(&stats_full[k], kProdThreads);
     if (kResid)
       for (int k = 0; k < kWsResSlots; ++k) {
         mbar_init(&res_full[k], kProdThreads);
-        mbar_init(&res_free[k], kWsEpiWarps);
+        mbar_init(&res_free[k], kEpiWarps);
       }
     fence_mbar_init();
     s_abort = 0;
@@ -648,38 +653,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       if (m >= mtiles || r >= a.rows) return -1;
       return (MODE == kQKV || kResid) ? a.rowsrc[r] : (int)r;
     };
-    // kLn: the layer norm's statistics of tile t's rows (thread p: row p), from
-    // the gathered bf16 values once they have landed -- one pass of sums and
-    // sums of squares (fp32, two channels per instruction), the biased variance
-    // E[x^2] - mean^2 and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
-    // definition); (0, 0) for padding rows and rows past the end.
-    auto tile_stats = [&](long long m, long long t) {
-      const int s = (int)(t % STAGES);
-      const long long r = m * kBM + tid;
-      const int tk = (m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
-      if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
-      float2 stv = make_float2(0.f, 0.f);
-      if (tk >= 0 && !s_abort) {
-        const uint8_t* row = sA + s * ws_a_bytes(K) + (tid >> 3) * sboA + (tid & 7) * 16;
-        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-        for (int kc = 0; kc < K / 8; ++kc) {
-          const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 128);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(h2[k]);
-            s1 = __fadd2_rn(s1, f);
-            s2 = __ffma2_rn(f, f, s2);
-          }
-        }
-        const float mean = (s1.x + s1.y) / (float)K;
-        const float var = fmaxf((s2.x + s2.y) / (float)K - mean * mean, 0.f);
-        const float rstd = 1.0f / sqrtf(var + a.ln_eps);
-        stv = make_float2(-mean * rstd, rstd);
-      }
-      sStats[(t % kWsStatSlots) * kBM + tid] = stv;
-      mbar_arrive(&stats_full[t % kWsStatSlots]);
-    };
     // Three register sets in rotation: the set of tile t is refilled with tile
     // t + 3's rows right after its copies are issued, so no instruction reads a
     // table value before about two tiles have passed (a register copy of a
@@ -733,7 +706,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       if (tid == 0) VSWIN_TRACE_EVENT(kTraceG + 0, trace_n, 51);
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) tok[grp] = row_tok(m + 3 * m_step, grp);
-      if (kLn && t > 0) tile_stats(m - m_step, t - 1);  // the previous tile has landed by now
     };
     long long t = 0;
     for (long long m = m_first; m < mtiles; m += 3 * m_step, t += 3) {
@@ -742,11 +714,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       tile(m + m_step, t + 1, tokB);
       if (m + 2 * m_step >= mtiles) break;
       tile(m + 2 * m_step, t + 2, tokC);
-    }
-    if (kLn) {  // the last tile's statistics
-      long long tl = 0, ml = m_first;
-      for (long long m = m_first; m < mtiles; m += m_step, ++tl) ml = m;
-      if (tl > 0) tile_stats(ml, tl - 1);
     }
     cp_async_wait_all();  // nothing in flight when the CTA ends
   } else if (warp == kWsMmaWarp) {
@@ -779,12 +746,54 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       }
     }
     __syncwarp();
+  } else if (kLn && warp >= kStat0) {
+    // ---------------------------------------------------------------- statistics (kLn)
+    // kLn: the layer norm's statistics of tile t's rows (statistics thread p: row p), from
+    // the gathered bf16 values once they have landed -- one pass of sums and
+    // sums of squares (fp32, two channels per instruction), the biased variance
+    // E[x^2] - mean^2 and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
+    // definition); (0, 0) for padding rows and rows past the end.
+    auto tile_stats = [&](long long m, long long t) {
+      const int s = (int)(t % STAGES);
+      const int p = tid - kStat0 * 32;
+      const long long r = m * kBM + p;
+      const int tk = (m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
+      if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+      float2 stv = make_float2(0.f, 0.f);
+      if (tk >= 0 && !s_abort) {
+        const uint8_t* row = sA + s * ws_a_bytes(K) + (p >> 3) * sboA + (p & 7) * 16;
+        float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+        for (int kc = 0; kc < K / 8; ++kc) {
+          const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 128);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(h2[k]);
+            s1 = __fadd2_rn(s1, f);
+            s2 = __ffma2_rn(f, f, s2);
+          }
+        }
+        const float mean = (s1.x + s1.y) / (float)K;
+        const float var = fmaxf((s2.x + s2.y) / (float)K - mean * mean, 0.f);
+        const float rstd = 1.0f / sqrtf(var + a.ln_eps);
+        stv = make_float2(-mean * rstd, rstd);
+      }
+      sStats[(t % kWsStatSlots) * kBM + p] = stv;
+      mbar_arrive(&stats_full[t % kWsStatSlots]);
+    };
+    long long t = 0;
+    for (long long m = m_first; m < mtiles; m += m_step, ++t) {
+      tile_stats(m, t);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_free[t % STAGES]);  // this warp has read the stage
+    }
   } else {
     // ---------------------------------------------------------------- epilogue
-    // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31: three warps per lane
-    // quarter, each taking a third of the columns (whole 8-column groups).
+    // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31: three (two with
+    // the fused pre-norm) warps per lane quarter, each taking a share of the
+    // columns (whole 8-column groups).
     const int q = warp & 3, hf = (warp - kWsEpi0) >> 2;
-    constexpr int kPerQ = kWsEpiWarps / 4;
+    constexpr int kPerQ = kEpiWarps / 4;
     const int c_lo = (hf * (BN / 8)) / kPerQ * 8, c_hi = ((hf + 1) * (BN / 8)) / kPerQ * 8;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const size_t win_elems = (size_t)g.heads * a.slab.head_elems();  // one window's q / k / v block
