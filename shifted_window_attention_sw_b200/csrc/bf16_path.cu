@@ -353,6 +353,9 @@ constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
 constexpr int kWsMaxBBytes = 96 * 1024;
 
 __host__ __device__ inline int ws_a_bytes(int K) { return kBM * K * 2; }
+// The fused pre-norm's extra K step (16 columns of A: the row's -mean in two
+// bf16 halves; 16 rows of the folded weights: the column sums in two halves).
+constexpr int kLnExtraK = 16;
 constexpr int kWsStatSlots = 8;  // fused pre-norm: tiles of row statistics in flight
 constexpr int kWsResSlots = 3;   // fused residual: tiles of residual rows in flight
 __host__ __device__ inline int ws_res_row_bytes(int BN) { return BN * 2 + 16; }  // padded row of a residual tile
@@ -360,7 +363,8 @@ __host__ __device__ inline int ws_res_row_bytes(int BN) { return BN * 2 + 16; } 
 // the fused pre-norm the column sums and folded bias (2 x BN floats), barriers,
 // with the fused pre-norm a ring of per-row statistics (8 tiles x 128 rows), with
 // the fused residual a ring of residual tiles (3 x 128 rows of the BN columns)
-__host__ __device__ inline int ws_smem_bytes(int K, int BN, int stages, bool ln = false, bool resid = false) {
+__host__ __device__ inline int ws_smem_bytes(int K0, int BN, int stages, bool ln = false, bool resid = false) {
+  const int K = ln ? K0 + kLnExtraK : K0;
   return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + (ln ? BN * 8 + kWsStatSlots * kBM * 8 : 0) +
          (resid ? kWsResSlots * kBM * ws_res_row_bytes(BN) : 0) + 256;
 }
@@ -421,6 +425,13 @@ __global__ void __launch_bounds__(kFoldCols * kFoldRows) ln_fold_kernel(
     }
     colsum[j] = cs;
     bias_ln[j] = __bfloat162float(bqkv[j]) + bb;
+    // rows C .. C + 15 of wt: the column sum as two bf16 halves (hi, lo, hi, lo),
+    // then zeros -- the persistent GEMM's extra K step multiplies them with the
+    // row's -mean (also two halves), so that the MMA itself subtracts mean x colsum
+    const __nv_bfloat16 hi = __float2bfloat16_rn(cs);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(cs - __bfloat162float(hi));
+    for (int k = 0; k < kLnExtraK; ++k)
+      wt[(size_t)(C + k) * N3 + j] = k < 4 ? ((k & 1) ? lo : hi) : __float2bfloat16_rn(0.f);
   }
 }
 
@@ -531,7 +542,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   constexpr bool kLn = FUSE && MODE == kQKV;      // pre-norm folded into the QKV epilogue
   constexpr bool kResid = FUSE && MODE == kPROJ;  // residual added in the projection epilogue
-  const int K = a.K, BN = a.BN;
+  // K: the MMA's depth -- the x columns, plus for the fused pre-norm one extra
+  // step of 16 (the row's -mean against the weights' column sums)
+  const int Kx = a.K, K = kLn ? a.K + kLnExtraK : a.K, BN = a.BN;
   uint8_t* sB = smem;                                     // K x BN, MN-major operand layout
   uint8_t* sA = sB + K * BN * 2;                          // STAGES x (128 x K), K-major
   float* sBias = reinterpret_cast<float*>(sA + STAGES * ws_a_bytes(K));  // bias x column scale
@@ -545,7 +558,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   uint64_t* acc_full = a_free + STAGES;    // [2]
   uint64_t* acc_free = acc_full + 2;       // [2]
   uint64_t* stats_full = acc_free + 2;     // kLn: [kWsStatSlots] a tile's row statistics written
-  uint64_t* res_full = stats_full + (kLn ? kWsStatSlots : 0);  // kResid: [kWsResSlots] residual tile landed
+  uint64_t* a_ext = stats_full + (kLn ? kWsStatSlots : 0);  // kLn: [STAGES] the stage's -mean columns written
+  uint64_t* res_full = a_ext + (kLn ? STAGES : 0);          // kResid: [kWsResSlots] residual tile landed
   uint64_t* res_free = res_full + (kResid ? kWsResSlots : 0);  // kResid: [kWsResSlots] residual tile read
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(res_free + (kResid ? kWsResSlots : 0));
   // kLn: (-mean * rstd, rstd) per row of a tile, (0, 0) for padding rows, slot t % 8
@@ -582,7 +596,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     mbar_init(b_full, kProdThreads);
     for (int k = 0; k < STAGES; ++k) {
       mbar_init(&a_full[k], kProdThreads);  // one asynchronous arrival per gathering thread
-      mbar_init(&a_free[k], 1 + kStatWarps);  // MMA commit (+ each statistics warp once it has read the stage)
+      mbar_init(&a_free[k], 1);  // MMA commit
+      if (kLn) mbar_init(&a_ext[k], kStatWarps * 32);  // every statistics thread, after its row's extra columns
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&acc_full[k], 1);
@@ -683,7 +698,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
           src = (m < mtiles && rA < a.rows) ? rA : -1;
         }
         const long long sg = src < 0 ? 0 : src * lda;
-        for (int kc = cq; kc < K / 8; kc += 4)
+        for (int kc = cq; kc < Kx / 8; kc += 4)
           cp_async_16(drow + kc * 128, a.A + sg + kc * 8, src < 0 ? 0u : 16u);
       }
       cp_async_mbar_arrive_noinc(&a_full[s]);  // arrives once this thread's copies have landed
@@ -728,6 +743,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
         const int s = (int)(t % STAGES), buf = (int)(t & 1);
         VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 60);
         if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+        if (kLn && !s_abort && !mbar_wait(&a_ext[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim))
+          s_abort = 1;
         fence_proxy_async_smem();
         VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 61);
         if (t >= 2 && !s_abort &&
@@ -748,22 +765,26 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     __syncwarp();
   } else if (kLn && warp >= kStat0) {
     // ---------------------------------------------------------------- statistics (kLn)
-    // kLn: the layer norm's statistics of tile t's rows (statistics thread p: row p), from
-    // the gathered bf16 values once they have landed -- one pass of sums and
-    // sums of squares (fp32, two channels per instruction), the biased variance
-    // E[x^2] - mean^2 and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
-    // definition); (0, 0) for padding rows and rows past the end.
+    // kLn: the layer norm's statistics of tile t's rows (statistics thread p:
+    // row p), from the gathered bf16 values once they have landed -- one pass of
+    // sums and sums of squares (fp32, two channels per instruction), the biased
+    // variance E[x^2] - mean^2 and rstd = 1 / sqrt(var + eps) (torch.nn.LayerNorm's
+    // definition). The row's -mean goes into the stage's extra K step as two bf16
+    // halves (-mean_hi, -mean_hi, -mean_lo, -mean_lo, 0 ...), against the folded
+    // weights' rows (colsum_hi, colsum_lo, colsum_hi, colsum_lo, 0 ...): the MMA
+    // then accumulates x Wt - mean colsum. Padding rows and rows past the end get
+    // zeros there and rstd 0; the epilogue reads (0, rstd) from the ring.
     auto tile_stats = [&](long long m, long long t) {
       const int s = (int)(t % STAGES);
       const int p = tid - kStat0 * 32;
       const long long r = m * kBM + p;
       const int tk = (m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
       if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
-      float2 stv = make_float2(0.f, 0.f);
+      uint8_t* row = sA + s * ws_a_bytes(K) + (p >> 3) * sboA + (p & 7) * 16;
+      float mean = 0.f, rstd = 0.f;
       if (tk >= 0 && !s_abort) {
-        const uint8_t* row = sA + s * ws_a_bytes(K) + (p >> 3) * sboA + (p & 7) * 16;
         float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-        for (int kc = 0; kc < K / 8; ++kc) {
+        for (int kc = 0; kc < Kx / 8; ++kc) {
           const uint4 v = *reinterpret_cast<const uint4*>(row + kc * 128);
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -773,20 +794,23 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
             s2 = __ffma2_rn(f, f, s2);
           }
         }
-        const float mean = (s1.x + s1.y) / (float)K;
-        const float var = fmaxf((s2.x + s2.y) / (float)K - mean * mean, 0.f);
-        const float rstd = 1.0f / sqrtf(var + a.ln_eps);
-        stv = make_float2(-mean * rstd, rstd);
+        mean = (s1.x + s1.y) / (float)Kx;
+        const float var = fmaxf((s2.x + s2.y) / (float)Kx - mean * mean, 0.f);
+        rstd = 1.0f / sqrtf(var + a.ln_eps);
       }
-      sStats[(t % kWsStatSlots) * kBM + p] = stv;
+      const __nv_bfloat16 mh = __float2bfloat16_rn(-mean);
+      const __nv_bfloat16 ml = __float2bfloat16_rn(-mean - __bfloat162float(mh));
+      const uint32_t mhb = __bfloat16_as_ushort(mh), mlb = __bfloat16_as_ushort(ml);
+      const uint32_t hh = mhb | (mhb << 16), ll = mlb | (mlb << 16);
+      *reinterpret_cast<uint4*>(row + (Kx / 8) * 128) = make_uint4(hh, ll, 0u, 0u);
+      *reinterpret_cast<uint4*>(row + (Kx / 8 + 1) * 128) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();  // the extra columns are a tensor-core operand
+      mbar_arrive(&a_ext[s]);
+      sStats[(t % kWsStatSlots) * kBM + p] = make_float2(0.f, rstd);
       mbar_arrive(&stats_full[t % kWsStatSlots]);
     };
     long long t = 0;
-    for (long long m = m_first; m < mtiles; m += m_step, ++t) {
-      tile_stats(m, t);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_free[t % STAGES]);  // this warp has read the stage
-    }
+    for (long long m = m_first; m < mtiles; m += m_step, ++t) tile_stats(m, t);
   } else {
     // ---------------------------------------------------------------- epilogue
     // A warp may only touch TMEM lanes 32 * (warp % 4) .. +31: three (two with
@@ -886,23 +910,14 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
             // plain: v = acc * scale + bias * scale. kLn (a token row): v = rs * acc
             // + (ns * colsum + folded bias * scale) with rs = rstd * scale, ns =
             // -mean * rstd * scale; a padding row (rstd = 0) keeps the plain bias.
+            // kLn (a token row): the accumulator already holds x Wt - mean colsum
+            // (the extra K step), so v = rstd * scale * acc + folded bias * scale; a
+            // padding row (rstd = 0) keeps the plain bias
             const float* bsrc = (kLn && st.y != 0.f) ? sBb : sBias;
-            float4 b0 = *reinterpret_cast<const float4*>(bsrc + cc);
-            float4 b1 = *reinterpret_cast<const float4*>(bsrc + cc + 4);
+            const float4 b0 = *reinterpret_cast<const float4*>(bsrc + cc);
+            const float4 b1 = *reinterpret_cast<const float4*>(bsrc + cc + 4);
             float2 sc = make_float2(cg.scale, cg.scale);
-            if (kLn) {
-              const float rs = st.y * cg.scale, ns = st.x * cg.scale;
-              const float4 c0v = *reinterpret_cast<const float4*>(sCs + cc);
-              const float4 c1v = *reinterpret_cast<const float4*>(sCs + cc + 4);
-              const float2 ns2 = make_float2(ns, ns);
-              const float2 t01 = __ffma2_rn(make_float2(c0v.x, c0v.y), ns2, make_float2(b0.x, b0.y));
-              const float2 t23 = __ffma2_rn(make_float2(c0v.z, c0v.w), ns2, make_float2(b0.z, b0.w));
-              const float2 t45 = __ffma2_rn(make_float2(c1v.x, c1v.y), ns2, make_float2(b1.x, b1.y));
-              const float2 t67 = __ffma2_rn(make_float2(c1v.z, c1v.w), ns2, make_float2(b1.z, b1.w));
-              b0 = make_float4(t01.x, t01.y, t23.x, t23.y);
-              b1 = make_float4(t45.x, t45.y, t67.x, t67.y);
-              if (st.y != 0.f) sc = make_float2(rs, rs);
-            }
+            if (kLn && st.y != 0.f) sc = make_float2(st.y * cg.scale, st.y * cg.scale);
             // two columns per instruction
             float2 v01 = __ffma2_rn(make_float2(__uint_as_float(u[g8 * 8 + 0]), __uint_as_float(u[g8 * 8 + 1])),
                                     sc, make_float2(b0.x, b0.y));

@@ -54,7 +54,7 @@ size_t bf16_scratch_bytes(const Geom& g, long long nwin);
 // the QKV weights (launch_ln_fold fills these buffers once per call) and
 // applied per row in the QKV epilogue; x added in the projection epilogue.
 struct BlockFuse {
-  void* wt;        // [C][3C] bf16: diag(gamma) Wqkv
+  void* wt;        // [C + 16][3C] bf16: diag(gamma) Wqkv, then the column sums (hi, lo, hi, lo) and zeros
   float* colsum;   // [3C] column sums of wt
   float* bias_ln;  // [3C] bqkv + beta Wqkv
   float eps;

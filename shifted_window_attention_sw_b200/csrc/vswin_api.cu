@@ -297,7 +297,8 @@ int forward_block_device(const void* x, const Geom& g, const void* gamma, const 
   if (status != VSWIN_OK) return status;
   const long long per_chunk = chunk_windows(g);
   const size_t chunk_bytes = (bf16_block_scratch_bytes(g, per_chunk) + 255) / 256 * 256;
-  const size_t wt_bytes = ((size_t)g.C * 3 * g.C * 2 + 255) / 256 * 256;
+  // folded weights: C rows, plus 16 rows of column sums for the fused GEMM's extra K step
+  const size_t wt_bytes = ((size_t)(g.C + 16) * 3 * g.C * 2 + 255) / 256 * 256;
   const size_t vec_bytes = ((size_t)3 * g.C * 4 + 255) / 256 * 256;
   void* scratch = nullptr;
   status = scratch_alloc(&scratch, chunk_bytes + wt_bytes + 2 * vec_bytes, st);
