@@ -363,10 +363,15 @@ __host__ __device__ inline int ws_res_row_bytes(int BN) { return BN * 2 + 16; } 
 // the fused pre-norm the column sums and folded bias (2 x BN floats), barriers,
 // with the fused pre-norm a ring of per-row statistics (8 tiles x 128 rows), with
 // the fused residual a ring of residual tiles (3 x 128 rows of the BN columns)
-__host__ __device__ inline int ws_smem_bytes(int K0, int BN, int stages, bool ln = false, bool resid = false) {
+// The projection's epilogue stages each tile's rows in shared memory (two
+// buffers of 128 padded rows and their output-row indices) and copies them out
+// row by row.
+__host__ __device__ inline int ws_stage_out_bytes(int BN) { return 2 * kBM * ws_res_row_bytes(BN) + 2 * kBM * 4; }
+__host__ __device__ inline int ws_smem_bytes(int K0, int BN, int stages, bool ln = false, bool resid = false,
+                                             bool stage_out = false) {
   const int K = ln ? K0 + kLnExtraK : K0;
   return K * BN * 2 + stages * ws_a_bytes(K) + BN * 6 + (ln ? BN * 8 + kWsStatSlots * kBM * 8 : 0) +
-         (resid ? kWsResSlots * kBM * ws_res_row_bytes(BN) : 0) + 256;
+         (resid ? kWsResSlots * kBM * ws_res_row_bytes(BN) : 0) + (stage_out ? ws_stage_out_bytes(BN) : 0) + 256;
 }
 
 // Destination facts of one group of 8 output columns of the QKV GEMM: element
@@ -567,6 +572,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
   // kResid: the residual rows of a tile (BN columns, padded rows), slot t % 3
   uint8_t* sRes = reinterpret_cast<uint8_t*>(bars) + 256;
   const int res_slot_bytes = kBM * ws_res_row_bytes(BN);
+  // projection: staged output tiles [2][128 padded rows], then their output rows [2][128]
+  uint8_t* sOut = sRes + (kResid ? kWsResSlots * res_slot_bytes : 0);
+  int* sDst = reinterpret_cast<int*>(sOut + 2 * res_slot_bytes);
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -907,10 +915,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
             if (g8 * 8 >= n) break;
             const int cc = c0 + g8 * 8;
             const ColGroup cg = sGrp[cc >> 3];
-            // plain: v = acc * scale + bias * scale. kLn (a token row): v = rs * acc
-            // + (ns * colsum + folded bias * scale) with rs = rstd * scale, ns =
-            // -mean * rstd * scale; a padding row (rstd = 0) keeps the plain bias.
-            // kLn (a token row): the accumulator already holds x Wt - mean colsum
+            // plain: v = acc * scale + bias * scale. kLn (a token row): the
+            // accumulator already holds x Wt - mean colsum
             // (the extra K step), so v = rstd * scale * acc + folded bias * scale; a
             // padding row (rstd = 0) keeps the plain bias
             const float* bsrc = (kLn && st.y != 0.f) ? sBb : sBias;
@@ -936,21 +942,41 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
             }
             const uint4 w = make_uint4(pack_bf16x2(v01.x, v01.y), pack_bf16x2(v23.x, v23.y),
                                        pack_bf16x2(v45.x, v45.y), pack_bf16x2(v67.x, v67.y));
-            if (rbase) {
-              __nv_bfloat16* dst =
-                  MODE == kQKV ? rbase + cg.off + (cg.is_q ? q_term : kv_term) : rbase + cc;
+            if (MODE == kPROJ) {  // staged; copied out row by row below
+              *reinterpret_cast<uint4*>(sOut + (t & 1) * res_slot_bytes + (q * 32 + lane) * ws_res_row_bytes(BN) +
+                                        cc * 2) = w;
+            } else if (rbase) {
+              __nv_bfloat16* dst = rbase + cg.off + (cg.is_q ? q_term : kv_term);
               *reinterpret_cast<uint4*>(dst) = w;
-              if (MODE == kQKV && kv_pad && !cg.is_q) *reinterpret_cast<uint4*>(dst + 8) = make_uint4(0, 0, 0, 0);
+              if (kv_pad && !cg.is_q) *reinterpret_cast<uint4*>(dst + 8) = make_uint4(0, 0, 0, 0);
             }
           }
         }
       }
+      if (MODE == kPROJ && hf == 0) sDst[(t & 1) * kBM + q * 32 + lane] = rbase ? dr_cur : -1;
       tc_fence_before();
       __syncwarp();
       if (warp == kWsEpi0 && lane == 0) VSWIN_TRACE_EVENT(kTraceG + 2, trace_n, 72);
       if (lane == 0) {
         mbar_arrive(&acc_free[buf]);
         if (kResid) mbar_arrive(&res_free[t % kWsResSlots]);
+      }
+      if (MODE == kPROJ) {
+        // the staged tile to its output rows: consecutive threads take consecutive
+        // 16-byte chunks of a row (whole rows per warp instruction, not one
+        // scattered chunk per thread); the buffer is rewritten two tiles later,
+        // after every epilogue warp has passed the next tile's barrier
+        named_bar_sync(1, kEpiWarps * 32);
+        const int cpr = BN / 8;  // chunks per row
+        const uint8_t* sb = sOut + (t & 1) * res_slot_bytes;
+        const int* db = sDst + (t & 1) * kBM;
+        for (int k = tid - kWsEpi0 * 32; k < kBM * cpr; k += kEpiWarps * 32) {
+          const int row = k / cpr, c8 = k - row * cpr;
+          const int dr = db[row];
+          if (dr >= 0 && !s_abort)
+            *reinterpret_cast<uint4*>(a.dst + (long long)dr * g.C + n0 + c8 * 8) =
+                *reinterpret_cast<const uint4*>(sb + row * ws_res_row_bytes(BN) + c8 * 16);
+        }
       }
     }
   }
@@ -2063,15 +2089,16 @@ int pick_bn(int n) {
 // The persistent GEMM runs when its weight slice and two A stages fit in shared
 // memory (227 KB per CTA, 1 KB of it static); otherwise the tiled version (e.g.
 // C = 544: BN = 32 for the projection, two 139 KB A stages).
-bool ws_fits(const GemmArgs& a, bool ln, bool resid = false) {
+bool ws_fits(const GemmArgs& a, bool ln, bool resid = false, bool stage_out = false) {
   return a.rowsrc && a.K * a.BN * 2 <= kWsMaxBBytes && a.K % 32 == 0 && (a.BN / 2) % 8 == 0 &&
-         ws_smem_bytes(a.K, a.BN, 2, ln, resid) <= 226 * 1024;
+         ws_smem_bytes(a.K, a.BN, 2, ln, resid, stage_out) <= 226 * 1024;
 }
 
 template <int MODE, bool FUSE>
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
   const bool resid = FUSE && MODE == kPROJ;
-  if (ws_fits(a, FUSE && MODE == kQKV, resid)) {
+  const bool stage_out = MODE == kPROJ;
+  if (ws_fits(a, FUSE && MODE == kQKV, resid, stage_out)) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -2083,8 +2110,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st) {
     // four A stages when they fit, else two; at least 116 KB so that one CTA
     // (up to 512 TMEM columns) owns each SM
     const bool ln = FUSE && MODE == kQKV;
-    const bool four = ws_smem_bytes(a.K, a.BN, 4, ln, resid) <= 220 * 1024;
-    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2, ln, resid);
+    const bool four = ws_smem_bytes(a.K, a.BN, 4, ln, resid, stage_out) <= 220 * 1024;
+    int smem_ws = ws_smem_bytes(a.K, a.BN, four ? 4 : 2, ln, resid, stage_out);
     if (smem_ws < 116 * 1024) smem_ws = 116 * 1024;
     auto kern = four ? gemm_ws_kernel<MODE, 4, FUSE> : gemm_ws_kernel<MODE, 2, FUSE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_ws);
