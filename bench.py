@@ -264,9 +264,9 @@ def _oracle_prep(wl, nwin):
 
 
 # ------------------------------------------------------------------ GPU arm
-def traffic_record(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the kernel
-    source has not changed since the counters were taken (else None)."""
+def traffic_record(kernel, workload):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the counters
+    were taken on `workload` and the kernel source has not changed since (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -274,7 +274,7 @@ def traffic_record(kernel):
     except (OSError, ValueError):
         return None
     entry = rec.get(kernel)
-    if not entry:
+    if not entry or entry.get("workload") != workload:
         return None
     src = os.path.join(ROOT, "shifted_window_attention_sw_b200", "csrc", entry.get("source", ""))
     try:
@@ -407,7 +407,7 @@ def run_gpu(args):
         achieved = dom_work / (dom_ms / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
         traffic_kernel = "gemm_kernel" if dom == "qkv_gemm" else "proj_kernel"
-    tr = traffic_record(traffic_kernel)
+    tr = traffic_record(traffic_kernel, args.workload)
     avg_us = 1e3 * dom_ms / max(1, dom_launches)
     roofline = {
         "kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
@@ -794,7 +794,7 @@ def run_mlp(args):
         "api": "vswin_block_msa_forward + vswin_mlp_forward" if args.block_full else "vswin_mlp_forward",
         "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
         "mlp_roofline": {"kernel": "mlp_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
-                         "traffic": (traffic_record("mlp_kernel") or {}).get("bytes_per_launch"),
+                         "traffic": (traffic_record("mlp_kernel", args.workload) or {}).get("bytes_per_launch"),
                          "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_src} bf16 dense (burst)",
                          "avg_launch_us": mlp_us, "launches": mlp_n,
                          "hbm_floor_us": mlp_bytes / len(layers) / (float(peaks["hbm_gbs"]) * 1e9) * 1e6,
