@@ -62,7 +62,8 @@ typedef enum {
   VSWIN_ERR_UNSUPPORTED = 2,  /* valid layer that this path does not implement (see each entry) */
   VSWIN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   VSWIN_ERR_TIMEOUT = 4,      /* a kernel's bounded wait gave up (reported by vswin_poll_error) */
-  VSWIN_ERR_NO_MEMORY = 5     /* scratch allocation failed */
+  VSWIN_ERR_NO_MEMORY = 5,    /* scratch allocation failed */
+  VSWIN_ERR_BOUNDS = 6        /* a build with VSWIN_DEBUG_BOUNDS caught an index out of its extent */
 } vswin_status;
 
 /*
@@ -324,7 +325,9 @@ const char* vswin_last_error(void);
 /*
  * Synchronises `stream`, then returns and clears the device error word:
  * VSWIN_OK, or VSWIN_ERR_TIMEOUT if a kernel's bounded wait gave up since the
- * last poll, or VSWIN_ERR_CUDA if synchronisation failed.
+ * last poll, VSWIN_ERR_BOUNDS if a build with VSWIN_DEBUG_BOUNDS caught an
+ * index out of its extent (the access was skipped), or VSWIN_ERR_CUDA if
+ * synchronisation failed.
  */
 int vswin_poll_error(void* stream);
 
@@ -343,6 +346,31 @@ void vswin_set_wait_limit_ns(unsigned long long ns);
  * that exact path, so that tests can check it; 0 restores the normal rule.
  */
 void vswin_set_exact_softmax(int on);
+
+/*
+ * Test hook: host-side fault injection. kind VSWIN_INJECT_CUDA makes the next
+ * `count` entry calls fail as if a CUDA runtime call had failed (status
+ * VSWIN_ERR_CUDA, message naming the injection) before they touch the device;
+ * VSWIN_INJECT_ALLOC makes the next `count` scratch allocations fail (status
+ * VSWIN_ERR_NO_MEMORY) before anything is launched. count 0 clears the kind.
+ * No kernel runs and nothing is allocated for an injected failure. Returns
+ * VSWIN_OK, or VSWIN_ERR_INVALID_ARG for an unknown kind or count < 0.
+ */
+enum { VSWIN_INJECT_CUDA = 1, VSWIN_INJECT_ALLOC = 2 };
+int vswin_test_inject_failure(int kind, int count);
+
+/*
+ * Test hook of builds with VSWIN_DEBUG_BOUNDS (index checks in the gathers and
+ * scatters: an index outside its extent sets the error word and the access is
+ * skipped). Every following bf16 layer forward overwrites its row table entry
+ * for window slot `slot` (counted over the whole layer) with `token`, after the
+ * table is computed; slot < 0 turns this off. In other builds it returns
+ * VSWIN_ERR_UNSUPPORTED and changes nothing.
+ */
+int vswin_debug_plant_row(long long slot, int token);
+
+/* 1 in a build with VSWIN_DEBUG_BOUNDS, else 0. */
+int vswin_debug_bounds_enabled(void);
 
 /*
  * Self-test of the timeout path: launches one kernel that waits, with the

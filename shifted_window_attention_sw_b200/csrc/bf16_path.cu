@@ -59,6 +59,11 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Tokens of the layer: the extent of every row-table entry (-1 = padding).
+__host__ __device__ inline long long layer_tokens(const Geom& g) {
+  return (long long)g.B * g.T * g.H * g.W;
+}
+
 // ============================================================================ GEMM
 constexpr int kBM = 128;
 constexpr int kBK = 32;
@@ -171,7 +176,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
     if (r < a.rows) {
       if (MODE == kQKV) {
         const long long gr = a.win0 * g.N + r;
-        const long long tok = slot_source(g, gr / g.N, (int)(gr % g.N));
+        long long tok = slot_source(g, gr / g.N, (int)(gr % g.N));
+        if (!index_ok(tok, -1, layer_tokens(g), a.ctx.err)) tok = -1;
         src = tok < 0 ? -1 : tok * g.C;
       } else {
         src = r * (long long)(a.lda ? a.lda : g.C);
@@ -280,6 +286,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
     } else if (row_ok) {
       const long long gr = a.win0 * g.N + r;
       dst_row = slot_source(g, gr / g.N, (int)(gr % g.N));
+      if (!index_ok(dst_row, -1, layer_tokens(g), a.ctx.err)) dst_row = -1;
     }
     for (int c = 0; c < BN / 16; ++c) {
       uint32_t u[16];
@@ -385,13 +392,20 @@ struct ColGroup {
 
 // Row sources of one chunk: token index (x row) of each window slot, -1 for
 // padding. Consumed by the QKV gather and the projection scatter.
-__global__ void row_source_kernel(Geom g, long long win0, long long rows, int* __restrict__ out) {
+__global__ void row_source_kernel(Geom g, long long win0, long long rows, int* __restrict__ out, int* err) {
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < rows; r += stride) {
     const long long gr = win0 * g.N + r;
-    out[r] = (int)slot_source(g, gr / g.N, (int)(gr % g.N));
+    long long tok = slot_source(g, gr / g.N, (int)(gr % g.N));
+    if (!index_ok(tok, -1, layer_tokens(g), err)) tok = -1;
+    out[r] = (int)tok;
   }
 }
+
+#ifdef VSWIN_DEBUG_BOUNDS
+// Test hook: overwrite one row-table entry.
+__global__ void plant_row_kernel(int* rowsrc, long long r, int token) { rowsrc[r] = token; }
+#endif
 
 // Pre-norm folded into the QKV weights ("Video Swin Transformer" summary page,
 // eq. 1: the layer reads LN(x)). Since LN(x) = rstd * (x - mean) * gamma + beta,
@@ -452,7 +466,8 @@ __global__ void __launch_bounds__(kFoldCols * kFoldRows) ln_fold_kernel(
 template <int NCH>
 __global__ void __launch_bounds__(256) row_stats_kernel(Geom g, long long win0, long long rows,
                                                         const __nv_bfloat16* __restrict__ x, float eps,
-                                                        int* __restrict__ rowsrc, float2* __restrict__ stats) {
+                                                        int* __restrict__ rowsrc, float2* __restrict__ stats,
+                                                        int* err) {
   const int lane = threadIdx.x & 31, cq = lane & 3, sub = lane >> 2;
   const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
   const long long warp0 = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -492,6 +507,7 @@ __global__ void __launch_bounds__(256) row_stats_kernel(Geom g, long long win0, 
       const int gr = (int)(win0 * g.N + R + lane);
       const int gw = gr / g.N;
       my_tok = slot_source32(g, gw, gr - gw * g.N);
+      if (!index_ok(my_tok, -1, layer_tokens(g), err)) my_tok = -1;
       rowsrc[R + lane] = my_tok;
     }
     if (NCH > 0) {
@@ -676,6 +692,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       if (m >= mtiles || r >= a.rows) return -1;
       return (MODE == kQKV || kResid) ? a.rowsrc[r] : (int)r;
     };
+    // the row table's tokens (or, unfused projection, chunk rows) against their extent
+    const long long tok_extent = (MODE == kQKV || kResid) ? layer_tokens(g) : a.rows;
     // Three register sets in rotation: the set of tile t is refilled with tile
     // t + 3's rows right after its copies are issued, so no instruction reads a
     // table value before about two tiles have passed (a register copy of a
@@ -701,6 +719,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
         // QKV: the row's source token; the fused projection's table holds the
         // residual's token, its A row is the chunk row itself
         long long src = tok[grp];
+        if (!index_ok(src, -1, tok_extent, a.ctx.err)) src = -1;
         if (kResid) {
           const long long rA = m * kBM + row;
           src = (m < mtiles && rA < a.rows) ? rA : -1;
@@ -719,7 +738,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) {
           const int row = warp * 32 + grp * 8 + sub;
-          const int tk = tok[grp];
+          const int tk = index_ok(tok[grp], -1, tok_extent, a.ctx.err) ? tok[grp] : -1;
           uint8_t* drow = sRes + rs * res_slot_bytes + row * ws_res_row_bytes(BN);
           const __nv_bfloat16* srow = a.resid + (tk < 0 ? 0 : (long long)tk * g.C) + n0;
           for (int kc = cq; kc < BN / 8; kc += 4) cp_async_16(drow + kc * 16, srow + kc * 8, tk < 0 ? 0u : 16u);
@@ -833,7 +852,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
     // value is first used a tile later)
     auto out_row = [&](long long m) -> int {
       const long long r = m * kBM + q * 32 + lane;
-      return (MODE == kPROJ && m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
+      const int dr = (MODE == kPROJ && m < mtiles && r < a.rows) ? a.rowsrc[r] : -1;
+      return index_ok(dr, -1, layer_tokens(g), a.ctx.err) ? dr : -1;
     };
     int dr_next = out_row(m_first);
     // columns handled per TMEM wait (the residual's registers and the norm's
@@ -2198,19 +2218,28 @@ cudaError_t launch_bf16_chunk(const Geom& g, const KernelCtx& ctx, const void* x
       if (blocks > 4096) blocks = 4096;
       const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
       switch (g.C / 32) {
-        case 1: row_stats_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
-        case 2: row_stats_kernel<2><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
-        case 3: row_stats_kernel<3><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
-        case 4: row_stats_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats); break;
-        default: row_stats_kernel<0><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats);
+        case 1: row_stats_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats, ctx.err); break;
+        case 2: row_stats_kernel<2><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats, ctx.err); break;
+        case 3: row_stats_kernel<3><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats, ctx.err); break;
+        case 4: row_stats_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats, ctx.err); break;
+        default: row_stats_kernel<0><<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, xb, fuse->eps, rowsrc, stats, ctx.err);
       }
     } else {
       long long blocks = (rows + 255) / 256;
       if (blocks > 2048) blocks = 2048;
-      row_source_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, rowsrc);
+      row_source_kernel<<<(unsigned)blocks, 256, 0, st>>>(g, win0, rows, rowsrc, ctx.err);
     }
     prof_end(kKindOther, st);
     count_launch();
+#ifdef VSWIN_DEBUG_BOUNDS
+    long long plant_slot = -1;
+    int plant_token = 0;
+    debug_plant(&plant_slot, &plant_token);
+    if (plant_slot >= win0 * g.N && plant_slot < win0 * g.N + rows) {
+      plant_row_kernel<<<1, 1, 0, st>>>(rowsrc, plant_slot - win0 * g.N, plant_token);
+      count_launch();
+    }
+#endif
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
   }

@@ -19,7 +19,25 @@ enum : int {
   kErrWaitLoad = 0x101,
   kErrWaitMma = 0x102,
   kErrWaitSelftest = 0x1FF,
+  kErrBounds = 0x201,  // VSWIN_DEBUG_BOUNDS: an index outside its extent (access skipped)
 };
+
+// Index check of the gathers and scatters: with VSWIN_DEBUG_BOUNDS, an index
+// outside [lo, n) records kErrBounds in the error word and the caller skips
+// the access; otherwise every index is taken as valid and nothing is checked.
+#ifdef VSWIN_DEBUG_BOUNDS
+__device__ __forceinline__ bool index_ok(long long i, long long lo, long long n, int* err) {
+  if (i >= lo && i < n) return true;
+  atomicCAS(err, 0, kErrBounds);
+  return false;
+}
+#else
+__device__ __forceinline__ bool index_ok(long long, long long, long long, int*) { return true; }
+#endif
+
+// VSWIN_DEBUG_BOUNDS test hook (vswin_debug_plant_row): the layer slot whose
+// row-table entry is overwritten, and the value; slot < 0 when off.
+void debug_plant(long long* slot, int* token);
 
 void count_launch(int n = 1);
 

@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(kPmThreads) pm_kernel(PmArgs a) {
       for (int q = 0; q < 4; ++q) {
         const long long h = 2 * i + (q & 1), w = 2 * j + (q >> 1);
         if (h < a.H && w < a.W) src[q] = ((bt * a.H + h) * a.W + w) * (long long)C;
+        // extent: the B * T clips' H * W tokens of C channels
+        if (!index_ok(src[q], -1, a.rows / ((long long)a.Hh * a.Wh) * a.H * a.W * C, a.ctx.err)) src[q] = -1;
       }
     }
     for (int q = 0; q < 4; ++q) s_src[q * kPmBM + tid] = src[q];

@@ -11,6 +11,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/vswin.h"
 #include "internal.h"
 
@@ -24,6 +26,29 @@ thread_local std::string t_last_error;
 std::atomic<unsigned long long> g_launches{0};
 std::atomic<unsigned long long> g_wait_limit_ns{1000000000ULL};
 std::atomic<int> g_force_exact{0};
+// Host-side fault injection (vswin_test_inject_failure): failures still to inject.
+std::atomic<int> g_inject_cuda{0}, g_inject_alloc{0};
+// VSWIN_DEBUG_BOUNDS test hook (vswin_debug_plant_row).
+std::atomic<long long> g_plant_slot{-1};
+std::atomic<int> g_plant_token{0};
+
+// Takes one pending injected failure of a kind, if any.
+bool take_injected(std::atomic<int>& pending) {
+  int n = pending.load();
+  while (n > 0)
+    if (pending.compare_exchange_weak(n, n - 1)) return true;
+  return false;
+}
+
+// Names every entry call on the NVTX timeline (a no-op unless a tool listens).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+const char* const kKindNames[kKinds] = {"vswin.qkv_gemm", "vswin.attention", "vswin.proj_gemm",
+                                        "vswin.other",    "vswin.mlp",       "vswin.attention_bwd"};
 std::mutex g_mu;
 constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices] = {nullptr};
@@ -61,6 +86,7 @@ int error_word(int** out) {
 }
 
 int make_ctx(KernelCtx* ctx) {
+  if (take_injected(g_inject_cuda)) return fail(VSWIN_ERR_CUDA, "injected CUDA failure (test hook)");
   int* err = nullptr;
   const int st = error_word(&err);
   if (st != VSWIN_OK) return st;
@@ -100,6 +126,9 @@ int scratch_pool(cudaMemPool_t* out) {
 }
 
 int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
+  if (take_injected(g_inject_cuda)) return fail(VSWIN_ERR_CUDA, "injected CUDA failure (test hook)");
+  if (take_injected(g_inject_alloc))
+    return fail(VSWIN_ERR_NO_MEMORY, "scratch allocation of %zu bytes: injected failure (test hook)", bytes);
   cudaMemPool_t pool = nullptr;
   const int status = scratch_pool(&pool);
   if (status != VSWIN_OK) return status;
@@ -350,7 +379,13 @@ cudaEvent_t prof_event() {
 }
 }  // namespace
 
+void debug_plant(long long* slot, int* token) {
+  *slot = g_plant_slot.load();
+  *token = g_plant_token.load();
+}
+
 void prof_begin(int kind, cudaStream_t st) {
+  nvtxRangePushA(kKindNames[kind]);
   if (!g_prof_on.load()) return;
   std::lock_guard<std::mutex> lock(g_prof_mu);
   cudaEvent_t e = prof_event();
@@ -360,6 +395,7 @@ void prof_begin(int kind, cudaStream_t st) {
 }
 
 void prof_end(int kind, cudaStream_t st) {
+  nvtxRangePop();
   if (!g_prof_on.load()) return;
   std::lock_guard<std::mutex> lock(g_prof_mu);
   cudaEvent_t s = g_prof_open[kind];
@@ -425,6 +461,33 @@ void vswin_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns ?
 
 void vswin_set_exact_softmax(int on) { g_force_exact.store(on ? 1 : 0); }
 
+int vswin_test_inject_failure(int kind, int count) {
+  if (count < 0) return fail(VSWIN_ERR_INVALID_ARG, "count=%d must be >= 0", count);
+  if (kind == VSWIN_INJECT_CUDA)
+    g_inject_cuda.store(count);
+  else if (kind == VSWIN_INJECT_ALLOC)
+    g_inject_alloc.store(count);
+  else
+    return fail(VSWIN_ERR_INVALID_ARG, "unknown injection kind %d", kind);
+  return VSWIN_OK;
+}
+
+int vswin_debug_bounds_enabled(void) {
+#ifdef VSWIN_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int vswin_debug_plant_row(long long slot, int token) {
+  if (!vswin_debug_bounds_enabled())
+    return fail(VSWIN_ERR_UNSUPPORTED, "vswin_debug_plant_row needs a build with VSWIN_DEBUG_BOUNDS");
+  g_plant_token.store(token);
+  g_plant_slot.store(slot < 0 ? -1 : slot);
+  return VSWIN_OK;
+}
+
 int vswin_clamp_window(int T, int H, int W, const int* window_in, const int* shift_in, int* window_out,
                        int* shift_out) {
   if (!window_in || !shift_in || !window_out || !shift_out)
@@ -447,6 +510,7 @@ int vswin_clamp_window(int T, int H, int W, const int* window_in, const int* shi
 int vswin_wmsa_forward(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
                        const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
                        const void* bias_table, void* out, void* stream) {
+  NvtxRange nvtx_range("vswin_wmsa_forward");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;
@@ -459,6 +523,7 @@ int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, in
                             const int* shift, const void* ln_gamma, const void* ln_beta, float ln_eps,
                             const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
                             const void* bias_table, void* out, void* stream) {
+  NvtxRange nvtx_range("vswin_block_msa_forward");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;
@@ -476,6 +541,7 @@ int vswin_block_msa_forward(const void* x, int B, int T, int H, int W, int C, in
 int vswin_mlp_forward(const void* x, int B, int T, int H, int W, int C, int hidden, const void* ln_gamma,
                       const void* ln_beta, float ln_eps, const void* W1, const void* b1, const void* W2,
                       const void* b2, void* out, void* stream) {
+  NvtxRange nvtx_range("vswin_mlp_forward");
   long long M = 0;
   int st = check_mlp_args(x, B, T, H, W, C, hidden, ln_gamma, ln_beta, ln_eps, W1, b1, W2, b2, out, &M);
   if (st != VSWIN_OK) return st;
@@ -493,6 +559,7 @@ int vswin_block_forward(const void* x, int B, int T, int H, int W, int C, int he
                         const void* bqkv, const void* Wproj, const void* bproj, const void* bias_table,
                         const void* ln2_gamma, const void* ln2_beta, int hidden, const void* W1, const void* b1,
                         const void* W2, const void* b2, float ln_eps, void* out, void* stream) {
+  NvtxRange nvtx_range("vswin_block_forward");
   // every argument of both halves is checked before anything is launched
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
@@ -523,6 +590,7 @@ int vswin_block_forward(const void* x, int B, int T, int H, int W, int C, int he
 int vswin_patch_merge_forward(const void* x, int B, int T, int H, int W, int C, const void* ln_gamma,
                               const void* ln_beta, float ln_eps, const void* Wr, const void* br, void* out,
                               void* stream) {
+  NvtxRange nvtx_range("vswin_patch_merge_forward");
   if (B <= 0 || T <= 0 || H <= 0 || W <= 0 || C <= 0)
     return fail(VSWIN_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d H=%d W=%d C=%d)", B, T, H, W, C);
   const void* ptrs[] = {x, ln_gamma, ln_beta, Wr, out};
@@ -562,6 +630,7 @@ int vswin_patch_merge_forward(const void* x, int B, int T, int H, int W, int C, 
 int vswin_wmsa_forward_f32(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
                            const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                            const void* bproj, const void* bias_table, void* out, void* stream) {
+  NvtxRange nvtx_range("vswin_wmsa_forward_f32");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;
@@ -589,6 +658,7 @@ int vswin_wmsa_backward_f32(const void* x, int B, int T, int H, int W, int C, in
                             const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                             const void* bproj, const void* bias_table, const void* dy, void* dx, void* dWqkv,
                             void* dbqkv, void* dWproj, void* dbproj, void* dtable, void* stream) {
+  NvtxRange nvtx_range("vswin_wmsa_backward_f32");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;
@@ -638,6 +708,7 @@ int vswin_wmsa_backward(const void* x, int B, int T, int H, int W, int C, int he
                         const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj, const void* bproj,
                         const void* bias_table, const void* dy, void* dx, void* dWqkv, void* dbqkv, void* dWproj,
                         void* dbproj, void* dtable, void* stream) {
+  NvtxRange nvtx_range("vswin_wmsa_backward");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;
@@ -693,6 +764,7 @@ int vswin_wmsa_backward(const void* x, int B, int T, int H, int W, int C, int he
 int vswin_wmsa_forward_host(const void* x_host, int B, int T, int H, int W, int C, int heads, const int* window,
                             const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                             const void* bproj, const void* bias_table, void* out_host, void* stream) {
+  NvtxRange nvtx_range("vswin_wmsa_forward_host");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;
@@ -797,6 +869,7 @@ int vswin_poll_error(void* stream) {
   const int zero = 0;
   e = cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return fail_cuda(e, "clearing the error word");
+  if (word == kErrBounds) return fail(VSWIN_ERR_BOUNDS, "an index check failed; the access was skipped (code 0x%x)", word);
   return fail(VSWIN_ERR_TIMEOUT, "a kernel wait gave up (code 0x%x)", word);
 }
 
@@ -841,6 +914,7 @@ int vswin_selftest_timeout(void* stream) {
 int vswin_wmsa_forward_noalloc(const void* x, int B, int T, int H, int W, int C, int heads, const int* window,
                                const int* shift, const void* Wqkv, const void* bqkv, const void* Wproj,
                                const void* bproj, const void* bias_table, void* out, void* stream) {
+  NvtxRange nvtx_range("vswin_wmsa_forward_noalloc");
   Geom g;
   int st = build_geom(B, T, H, W, C, heads, window, shift, &g);
   if (st != VSWIN_OK) return st;

@@ -13,9 +13,12 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libvswin.so")
+# VSWIN_LIBRARY may name another build of the same library (the in-tree
+# libvswin_debug.so, built with VSWIN_DEBUG_BOUNDS) to load instead.
+LIB_PATH = os.environ.get("VSWIN_LIBRARY") or os.path.join(_PKG, "libvswin.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_MEMORY = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_MEMORY, ERR_BOUNDS = range(7)
+INJECT_CUDA, INJECT_ALLOC = 1, 2
 
 # Every symbol include/vswin.h declares.
 EXPORTS = (
@@ -40,6 +43,9 @@ EXPORTS = (
     "vswin_mlp_forward",
     "vswin_block_forward",
     "vswin_patch_merge_forward",
+    "vswin_test_inject_failure",
+    "vswin_debug_plant_row",
+    "vswin_debug_bounds_enabled",
 )
 
 KERNEL_KINDS = ("qkv_gemm", "attention", "proj_gemm", "other", "mlp", "attention_bwd")
@@ -107,6 +113,12 @@ def lib():
         L.vswin_profile_collect.restype = _I
         L.vswin_version.argtypes = []
         L.vswin_version.restype = _I
+        L.vswin_test_inject_failure.argtypes = [_I, _I]
+        L.vswin_test_inject_failure.restype = _I
+        L.vswin_debug_plant_row.argtypes = [ctypes.c_longlong, _I]
+        L.vswin_debug_plant_row.restype = _I
+        L.vswin_debug_bounds_enabled.argtypes = []
+        L.vswin_debug_bounds_enabled.restype = _I
         _lib = L
     return _lib
 
@@ -390,7 +402,8 @@ def clamp_window(T, H, W, window, shift):
 
 
 def poll_error(stream=None) -> int:
-    """Synchronise and return the device error status (0 = OK, 4 = a kernel wait gave up)."""
+    """Synchronise and return the device error status (0 = OK, 4 = a kernel wait gave up,
+    6 = an index check of a VSWIN_DEBUG_BOUNDS build failed)."""
     return int(lib().vswin_poll_error(_stream_handle(stream)))
 
 
@@ -426,3 +439,19 @@ def profile_collect():
 
 def version() -> int:
     return int(lib().vswin_version())
+
+
+def inject_failure(kind: int, count: int = 1) -> None:
+    """Test hook: the next `count` entry calls fail as a CUDA call would (INJECT_CUDA) or
+    the next `count` scratch allocations fail (INJECT_ALLOC); count 0 clears."""
+    _check(lib().vswin_test_inject_failure(int(kind), int(count)))
+
+
+def debug_bounds_enabled() -> bool:
+    return bool(lib().vswin_debug_bounds_enabled())
+
+
+def debug_plant_row(slot: int, token: int) -> None:
+    """Test hook of VSWIN_DEBUG_BOUNDS builds: every following bf16 layer forward
+    overwrites its row-table entry for layer slot `slot` with `token` (slot < 0: off)."""
+    _check(lib().vswin_debug_plant_row(int(slot), int(token)))

@@ -362,3 +362,66 @@ def test_patch_merge_unsupported_width(L):
     before = vswin.launch_count()
     assert _call_merge(L, C=48) == vswin.ERR_UNSUPPORTED
     assert vswin.launch_count() == before
+
+
+# ------------------------------------------------------------------ host-side fault injection
+def _host_only():
+    import torch
+
+    return pytest.mark.skipif(torch.cuda.is_available(),
+                              reason="calls with fake device pointers: only where no GPU can run them")
+
+
+@_host_only()
+def test_injected_cuda_failure_returns_before_the_device(L):
+    """An injected CUDA failure makes the next entry calls return VSWIN_ERR_CUDA,
+    naming the injection, before any device access; the count is exact."""
+    before = vswin.launch_count()
+    assert L.vswin_test_inject_failure(vswin.INJECT_CUDA, 2) == vswin.OK
+    for name in ("vswin_wmsa_forward", "vswin_wmsa_forward_f32"):  # bf16 and fp32 entries
+        assert _call(getattr(L, name)) == vswin.ERR_CUDA
+        assert "injected" in vswin.last_error()
+    # both consumed: the next call reaches the CUDA runtime, which has no device here
+    assert _call(L.vswin_wmsa_forward) == vswin.ERR_CUDA
+    assert "injected" not in vswin.last_error()
+    assert vswin.launch_count() == before
+
+
+@_host_only()
+def test_injected_failure_cleared_by_count_zero(L):
+    assert L.vswin_test_inject_failure(vswin.INJECT_CUDA, 5) == vswin.OK
+    assert L.vswin_test_inject_failure(vswin.INJECT_CUDA, 0) == vswin.OK
+    assert _call(L.vswin_wmsa_forward) == vswin.ERR_CUDA
+    assert "injected" not in vswin.last_error()
+
+
+def test_injection_rejects_bad_arguments(L):
+    assert L.vswin_test_inject_failure(7, 1) == vswin.ERR_INVALID_ARG
+    assert L.vswin_test_inject_failure(vswin.INJECT_ALLOC, -1) == vswin.ERR_INVALID_ARG
+    assert L.vswin_test_inject_failure(vswin.INJECT_ALLOC, 0) == vswin.OK
+
+
+def test_invalid_arguments_do_not_consume_an_injection(L):
+    """Validation comes first: a rejected call leaves a pending injection in place."""
+    assert L.vswin_test_inject_failure(vswin.INJECT_CUDA, 1) == vswin.OK
+    assert _call(L.vswin_wmsa_forward, B=0) == vswin.ERR_INVALID_ARG
+    assert L.vswin_test_inject_failure(vswin.INJECT_CUDA, 0) == vswin.OK
+
+
+# ------------------------------------------------------------------ VSWIN_DEBUG_BOUNDS build
+def test_plant_hook_needs_the_debug_build(L):
+    assert L.vswin_debug_bounds_enabled() == 0
+    assert L.vswin_debug_plant_row(3, 5) == vswin.ERR_UNSUPPORTED
+    assert "VSWIN_DEBUG_BOUNDS" in vswin.last_error()
+
+
+def test_debug_bounds_library_builds_and_exports_every_symbol():
+    path = build_mod.build(debug_bounds=True)
+    assert path == build_mod.LIB_DEBUG and os.path.exists(path)
+    D = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(D, name), name
+    D.vswin_debug_plant_row.argtypes = [ctypes.c_longlong, ctypes.c_int]
+    assert D.vswin_debug_bounds_enabled() == 1
+    assert D.vswin_debug_plant_row(3, 5) == vswin.OK
+    assert D.vswin_debug_plant_row(-1, 0) == vswin.OK
