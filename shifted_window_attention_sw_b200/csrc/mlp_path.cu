@@ -12,15 +12,16 @@
 //     TMA -- when every chunk fits in shared memory at once they are loaded
 //     once per CTA -- and stores each finished output tile with TMA;
 //   * warp 1 issues, per hidden chunk, fc1 = LN(x) W1[:, chunk] into one of
-//     two TMEM accumulators, and fc2 += h_chunk W2[chunk, :] with h read
-//     from TMEM (the A operand of a TS MMA) into one of two output
-//     accumulators;
+//     two TMEM accumulators, and the last warp fc2 += h_chunk W2[chunk, :]
+//     with h read from TMEM (the A operand of a TS MMA) into one of two output
+//     accumulators -- two issuing threads on different SM sub-partitions;
 //   * warps 2-5 normalise each tile in place as soon as it lands (fp32
 //     statistics, bf16 result in the MMA operand layout) and write each
 //     tile's output: output accumulator + b2 + x (re-read from global memory,
 //     L1-prefetched before the wait), bf16, staged over the tile's buffer;
-//   * warps 6-13 turn each fc1 accumulator into h = GELU(acc + b1) (bf16,
-//     written over the accumulator's own columns).
+//   * the GELU warps (four per TMEM lane quarter) turn each fc1 accumulator
+//     into h = GELU(acc + b1) (bf16, written over the accumulator's own
+//     columns).
 //
 // GELU: the erf form x * Phi(x) (torch.nn.GELU's default) evaluated as
 // 0.5 x (1 + tanh(x (g1 + g3 x^2 + g5 x^4))) with x^2 clamped at 64, whose
@@ -47,7 +48,14 @@ namespace vswin {
 namespace {
 
 constexpr int kMlpMaxHC = 128;       // hidden columns per chunk: 128, or 64 when two 128-column stages do not fit
-constexpr int kMlpThreads = 14 * 32;  // producer, MMA, 4 norm / output warps, 8 GELU warps
+#ifndef VSWIN_MLP_GELU_PER_QUARTER
+#define VSWIN_MLP_GELU_PER_QUARTER 4
+#endif
+constexpr int kMlpGeluPerQ = VSWIN_MLP_GELU_PER_QUARTER;  // GELU warps per TMEM lane quarter
+constexpr int kMlpGeluWarps = 4 * kMlpGeluPerQ;  // each takes 1 / kMlpGeluPerQ of a chunk's columns
+constexpr int kMlpFc2Warp = 6 + kMlpGeluWarps;  // issues fc2 (warp 1 issues fc1)
+// producer, fc1 issue, 4 norm / output warps, GELU warps, fc2 issue
+constexpr int kMlpThreads = (kMlpFc2Warp + 1) * 32;
 constexpr int kMlpNorm0 = 2;          // first norm / output warp
 constexpr int kMlpGelu0 = 6;          // first GELU warp
 constexpr int kMlpXBufs = 3;          // x tiles in flight
@@ -182,12 +190,13 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
   uint64_t* xn_free = bars + 6;     // [3] the tile's fc1 MMAs have read it
   uint64_t* out_full = bars + 9;    // [3] output staged over the tile (4 output warps)
   uint64_t* acc1_full = bars + 12;  // [2]
-  uint64_t* h_full = bars + 14;     // [2] h written over the fc1 accumulator (8 GELU warps)
+  uint64_t* h_full = bars + 14;     // [2] h written over the fc1 accumulator (every GELU warp)
   uint64_t* acc2_full = bars + 16;  // [2]
   uint64_t* acc2_free = bars + 18;  // [2] (4 output warps)
   uint64_t* w_full = bars + 20;     // [S <= 8]
   uint64_t* w_free = bars + 28;     // [S <= 8]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 36);
+  uint64_t* fc2_done = bars + 36;   // [2] fc2 of the chunk in fc1 accumulator k has read h
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 38);
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -206,9 +215,10 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&acc1_full[k], 1);
-      mbar_init(&h_full[k], 8);
+      mbar_init(&h_full[k], kMlpGeluWarps);
       mbar_init(&acc2_full[k], 1);
       mbar_init(&acc2_free[k], 4);
+      mbar_init(&fc2_done[k], 1);
     }
     for (int k = 0; k < S; ++k) {
       mbar_init(&w_full[k], 1);
@@ -273,8 +283,15 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       bulk_wait0();  // every store has completed before the CTA ends
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kMlpFc2Warp) {
     // ------------------------------------------------------------ MMA issue
+    // Two issuing threads on different SM sub-partitions, so that each chunk's
+    // 6 + 8 MMAs are issued side by side (a thread's issue slows sharply when
+    // its sub-partition's other warps keep the issue slots busy): warp 1
+    // issues fc1 = LN(x) W1[:, chunk] into an fc1 accumulator, the fc2 warp
+    // fc2 += h W2[chunk, :] once the GELU warps have written h. fc1 of chunk
+    // g + 2 reuses the accumulator of chunk g only after chunk g's fc2 has
+    // completed (fc2_done).
     if (lane == 0) {
       const uint32_t id1 = idesc_bf16(128, HC, 0, 1);  // A K-major (x), B MN-major (W1)
       const uint32_t id2 = idesc_bf16(128, C, 0, 1);   // A from TMEM (h), B MN-major (W2)
@@ -283,57 +300,63 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       const long long total = ntiles * NCH;
       auto stage_of = [&](long long g) -> int { return a.resident ? (int)(g % NCH) : (int)(g % S); };
       auto w_phase = [&](long long g) -> uint32_t { return a.resident ? 0u : (uint32_t)(g / S) & 1; };
-      // fc1 of global chunk g: waits for its tile's normalised x (first chunk
-      // of a tile) and its weight stage
-      auto fc1 = [&](long long g) {
-        const long long t = g / NCH;
-        const int c = (int)(g % NCH);
-        const int xb = (int)(t % kMlpXBufs);
-        if (c == 0 && !s_abort &&
-            !mbar_wait(&xn_full[xb], (uint32_t)(t / kMlpXBufs) & 1, a.ctx.err, kErrWaitLoad, lim))
-          s_abort = 1;
-        const int s = stage_of(g);
-        if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
-        tc_fence_after();
-        if (s_abort) return;
-        const uint32_t xa = smem_u32(sX(xb));
-        const uint32_t wa = smem_u32(smem + L.w + s * L.wstage);
-        const uint32_t d = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
-        // K step ks covers channels [16 ks, 16 ks + 16): block ks / 2, 32 B in
-        for (int ks = 0; ks < C / 16; ++ks)
-          umma_ss(d, smem_desc_sw64(xa + (ks >> 1) * 8192 + (ks & 1) * 32), smem_desc(wa + ks * 2 * lbo1, lbo1, 128),
-                  id1, ks > 0);
-        umma_commit(&acc1_full[g & 1]);
-        if (c == NCH - 1) umma_commit(&xn_free[xb]);
-      };
-      if (total > 0) fc1(0);
-      if (total > 1) fc1(1);
-      for (long long g = 0; g < total && !s_abort; ++g) {
-        const long long t = g / NCH;
-        const int c = (int)(g % NCH);
-        const int ob = (int)(t & 1);
-        // h of chunk g is in TMEM (and its fc1 accumulator was read)
-        if (!mbar_wait(&h_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
-        // the output accumulator of this tile was drained two tiles ago
-        if (c == 0 && t >= 2 && !s_abort &&
-            !mbar_wait(&acc2_free[ob], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
-          s_abort = 1;
-        tc_fence_after();
-        if (s_abort) break;
-        const int s = stage_of(g);
-        const uint32_t wa2 = smem_u32(smem + L.w + s * L.wstage + L.w2off);
-        const uint32_t hb = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
-        const uint32_t d2 = tAcc2 + (uint32_t)ob * (uint32_t)C;
-        // h element k of the chunk sits at column hf * HC/2 + (k - hf * HC/2) / 2,
-        // hf = k / (HC/2) (each epilogue half packs its own columns in place)
-        for (int j = 0; j < HC / 16; ++j) {
-          const int hf = (16 * j) / (HC / 2);
-          const uint32_t hcol = (uint32_t)(hf * (HC / 2) + (16 * j - hf * (HC / 2)) / 2);
-          umma_ts(d2, hb + hcol, smem_desc(wa2 + j * 2 * lbo2, lbo2, 128), id2, (c > 0 || j > 0) ? 1u : 0u);
+      if (warp == 1) {
+        for (long long g = 0; g < total && !s_abort; ++g) {
+          const long long t = g / NCH;
+          const int c = (int)(g % NCH);
+          const int xb = (int)(t % kMlpXBufs);
+          // the accumulator's previous chunk (g - 2) has been read by its fc2
+          if (g >= 2 && !mbar_wait(&fc2_done[g & 1], (uint32_t)((g - 2) >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
+            s_abort = 1;
+          // the tile's normalised x (first chunk of a tile) and the weight stage
+          if (c == 0 && !s_abort &&
+              !mbar_wait(&xn_full[xb], (uint32_t)(t / kMlpXBufs) & 1, a.ctx.err, kErrWaitLoad, lim))
+            s_abort = 1;
+          const int s = stage_of(g);
+          if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+          tc_fence_after();
+          if (s_abort) break;
+          const uint32_t xa = smem_u32(sX(xb));
+          const uint32_t wa = smem_u32(smem + L.w + s * L.wstage);
+          const uint32_t d = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
+          // K step ks covers channels [16 ks, 16 ks + 16): block ks / 2, 32 B in
+          for (int ks = 0; ks < C / 16; ++ks)
+            umma_ss(d, smem_desc_sw64(xa + (ks >> 1) * 8192 + (ks & 1) * 32),
+                    smem_desc(wa + ks * 2 * lbo1, lbo1, 128), id1, ks > 0);
+          umma_commit(&acc1_full[g & 1]);
+          if (c == NCH - 1) umma_commit(&xn_free[xb]);
         }
-        if (!a.resident) umma_commit(&w_free[s]);
-        if (c == NCH - 1) umma_commit(&acc2_full[ob]);
-        if (g + 2 < total) fc1(g + 2);
+      } else {
+        for (long long g = 0; g < total && !s_abort; ++g) {
+          const long long t = g / NCH;
+          const int c = (int)(g % NCH);
+          const int ob = (int)(t & 1);
+          // h of chunk g is in TMEM (and its fc1 accumulator was read)
+          if (!mbar_wait(&h_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
+          // the output accumulator of this tile was drained two tiles ago
+          if (c == 0 && t >= 2 && !s_abort &&
+              !mbar_wait(&acc2_free[ob], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
+            s_abort = 1;
+          const int s = stage_of(g);
+          if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+          tc_fence_after();
+          if (s_abort) break;
+          const uint32_t wa2 = smem_u32(smem + L.w + s * L.wstage + L.w2off);
+          const uint32_t hb = tAcc1 + (uint32_t)(g & 1) * (uint32_t)HC;
+          const uint32_t d2 = tAcc2 + (uint32_t)ob * (uint32_t)C;
+          // h element k of the chunk sits at column hq * CW + (k - hq * CW) / 2,
+          // hq = k / CW, CW = HC / kMlpGeluPerQ (each GELU warp packs its own
+          // columns in place)
+          const int CW = HC / kMlpGeluPerQ;
+          for (int j = 0; j < HC / 16; ++j) {
+            const int hq = (16 * j) / CW;
+            const uint32_t hcol = (uint32_t)(hq * CW + (16 * j - hq * CW) / 2);
+            umma_ts(d2, hb + hcol, smem_desc(wa2 + j * 2 * lbo2, lbo2, 128), id2, (c > 0 || j > 0) ? 1u : 0u);
+          }
+          if (!a.resident) umma_commit(&w_free[s]);
+          if (c == NCH - 1) umma_commit(&acc2_full[ob]);
+          umma_commit(&fc2_done[g & 1]);
+        }
       }
     }
     __syncwarp();
@@ -454,10 +477,11 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
         finish_tile(t);
       }
     } else {
-      // Warps 6-13: GELU of each hidden chunk, this warp's HC/2 fc1 columns
-      // (half hf of the chunk) -> HC/4 columns of bf16 pairs over the first half
-      // of the same columns.
-      const int hf = (warp - kMlpGelu0) >> 2;
+      // GELU warps: GELU of each hidden chunk, this warp's CW fc1 columns
+      // (part hq of the chunk) -> CW/2 columns of bf16 pairs over the first
+      // half of the same columns.
+      const int hq = (warp - kMlpGelu0) >> 2;
+      const int CW = HC / kMlpGeluPerQ;  // this warp's columns of a chunk: 16, 32 or 64
       const long long total = ntiles * NCH;
       for (long long g = 0; g < total; ++g) {
         const int c = (int)(g % NCH);
@@ -465,20 +489,30 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           s_abort = 1;
         tc_fence_after();
         if (!s_abort) {
-          const uint32_t ta = tAcc1 + lane_base + (uint32_t)(g & 1) * (uint32_t)HC + (uint32_t)(hf * (HC / 2));
-          const float* b1 = sB1 + c * HC + hf * (HC / 2);
-          uint32_t u[32], w[16];
-          for (int part = 0; part < HC / 64; ++part) {
-            tmem_ld32(ta + 32 * part, u);
+          const uint32_t ta = tAcc1 + lane_base + (uint32_t)(g & 1) * (uint32_t)HC + (uint32_t)(hq * CW);
+          const float* b1 = sB1 + c * HC + hq * CW;
+          for (int p0 = 0; p0 < CW; p0 += 32) {  // up to 32 columns at a time
+            const int n = CW - p0 < 32 ? CW - p0 : 32;
+            uint32_t u[32], w[16];
+            if (n == 32)
+              tmem_ld32(ta + p0, u);
+            else
+              tmem_ld16(ta + p0, u);
             tmem_wait_ld_keep(u);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float2 bb = *reinterpret_cast<const float2*>(b1 + 32 * part + 2 * e);
-              const float2 v = __fadd2_rn(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), bb);
+              if (2 * e >= n) break;
+              const float2 bb = *reinterpret_cast<const float2*>(b1 + p0 + 2 * e);
+              const float2 v =
+                  __fadd2_rn(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), bb);
               const float2 gv = gelu2(v);
               w[e] = pack2(gv.x, gv.y);
             }
-            tmem_st16(ta + 16 * part, w);
+            // packed pairs over the first half of this warp's columns
+            if (n == 32)
+              tmem_st16(ta + p0 / 2, w);
+            else
+              tmem_st8(ta + p0 / 2, w);
           }
           tmem_wait_st();
         }
