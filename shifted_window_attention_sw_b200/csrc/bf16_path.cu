@@ -347,16 +347,21 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(GemmArgs a) {
 // per-CTA weight slice (K x BN bf16) fits in shared memory: warps 0-3 gather
 // 128-row A tiles with cp.async into a ring of STAGES buffers (each thread's
 // copies arrive on the stage's mbarrier when they land, so the gatherers only
-// wait for a free stage), warp 4 issues tcgen05.mma into two TMEM
-// accumulators (BN columns each), warps 5..16 drain an accumulator (three warps
-// per TMEM lane quarter, a third of the columns each) while the next tile is
-// multiplied. CTA c keeps N-tile c % NT and walks the M-tiles
+// wait for a free stage), warps 4 and 17 issue tcgen05.mma (the even and the
+// odd tiles) into two TMEM accumulators (BN columns each), warps 5..16 drain an
+// accumulator (three warps per TMEM lane quarter, a third of the columns each)
+// while the next tile is multiplied. CTA c keeps N-tile c % NT and walks the M-tiles
 // c / NT, c / NT + G / NT, ... (G = grid size, a multiple of NT).
 constexpr int kWsProdWarps = 4;
 constexpr int kWsEpiWarps = 12;
 constexpr int kWsMmaWarp = kWsProdWarps;
 constexpr int kWsEpi0 = kWsProdWarps + 1;
-constexpr int kWsThreads = 32 * (kWsProdWarps + 1 + kWsEpiWarps);
+// A second MMA warp, after the epilogue warps (another SM sub-partition):
+// warp kWsMmaWarp issues the even tiles, this one the odd tiles -- each tile
+// has its own accumulator (t & 1) and A stage, and a thread's MMA issue slows
+// when its sub-partition's other warps keep the issue slots busy.
+constexpr int kWsMma2Warp = kWsProdWarps + 1 + kWsEpiWarps;
+constexpr int kWsThreads = 32 * (kWsMma2Warp + 1);
 constexpr int kWsMaxBBytes = 96 * 1024;
 
 __host__ __device__ inline int ws_a_bytes(int K) { return kBM * K * 2; }
@@ -758,22 +763,23 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
       tile(m + 2 * m_step, t + 2, tokC);
     }
     cp_async_wait_all();  // nothing in flight when the CTA ends
-  } else if (warp == kWsMmaWarp) {
+  } else if (warp == kWsMmaWarp || warp == kWsMma2Warp) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
+      const int parity = warp == kWsMmaWarp ? 0 : 1;  // the tiles (and accumulator) of this thread
       if (!mbar_wait(b_full, 0, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
       fence_proxy_async_smem();  // the gathered bytes, written by cp.async, are read by the tensor core
       const uint32_t idesc = idesc_bf16(kBM, BN, 0, 1);
       const uint32_t baddr = smem_u32(sB);
-      long long t = 0;
-      for (long long m = m_first; m < mtiles; m += m_step, ++t) {
+      long long t = parity;
+      for (long long m = m_first + parity * m_step; m < mtiles; m += 2 * m_step, t += 2) {
         const int s = (int)(t % STAGES), buf = (int)(t & 1);
-        VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 60);
+        if (parity == 0) VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 60);
         if (!s_abort && !mbar_wait(&a_full[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
         if (kLn && !s_abort && !mbar_wait(&a_ext[s], (uint32_t)(t / STAGES) & 1, a.ctx.err, kErrWaitLoad, lim))
           s_abort = 1;
         fence_proxy_async_smem();
-        VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 61);
+        if (parity == 0) VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 61);
         if (t >= 2 && !s_abort &&
             !mbar_wait(&acc_free[buf], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
           s_abort = 1;
@@ -785,7 +791,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) gemm_ws_kernel(GemmArgs a) {
                     smem_desc(baddr + ks * 2 * lboB, lboB, 128), idesc, ks > 0);
           umma_commit(&a_free[s]);
           umma_commit(&acc_full[buf]);
-          VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 62);
+          if (parity == 0) VSWIN_TRACE_EVENT(kTraceG + 1, trace_n, 62);
         }
       }
     }
