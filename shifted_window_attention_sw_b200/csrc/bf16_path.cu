@@ -1392,6 +1392,10 @@ constexpr int kA7PrepWarps = 4;
 constexpr int kA7Groups = 3;
 constexpr int kA7Soft0 = kA7PrepWarps;                               // first softmax warp
 constexpr int kA7Threads = (kA7PrepWarps + 4 * kA7Groups) * 32;  // 512
+// Registers per thread: launched at 128 (the most 512 threads get), then the
+// preparation warpgroup gives some to the three softmax warpgroups.
+constexpr int kA7RegsLaunch = 128, kA7RegsPrep = 64, kA7RegsSoft = 144;
+static_assert(128 * kA7RegsPrep + 384 * kA7RegsSoft <= kA7Threads * kA7RegsLaunch, "register budgets");
 constexpr uint32_t kA7TmemCols = 512;
 // TMEM columns: group g has S / P at [144 g, 144 g + 112) and O at
 // [144 g + 112, 144 g + 144); the q rows of its tile at [432 + 16 g, + 16) and
@@ -1713,6 +1717,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
 
   if (warp < kA7PrepWarps) {
     // ------------------------------------------------------------ preparation
+    setmaxnreg_dec<kA7RegsPrep>();
     const int pt_ = tid;
     int tab_head0 = -1, tab_head1 = -1;
     float tab_max0 = 0.f, tab_max1 = 0.f;
@@ -1860,6 +1865,7 @@ __global__ void __launch_bounds__(kA7Threads, 1) attention7_kernel(AttnArgs a) {
     }
   } else {
     // ------------------------------------------------------------ softmax groups
+    setmaxnreg_inc<kA7RegsSoft>();
     const int grp = (warp - kA7Soft0) >> 2;
     const int qd = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t tG = tmem + (uint32_t)grp * kA7GroupCols;  // the group's columns, lane 0
@@ -2095,6 +2101,13 @@ cudaError_t launch_attention7(const AttnArgs& a, cudaStream_t st) {
   cudaError_t e =
       cudaFuncSetAttribute(attention7_kernel<Wn>, cudaFuncAttributeMaxDynamicSharedMemorySize, Wn::SMEM);
   if (e != cudaSuccess) return e;
+  // the warpgroups' register budgets draw on the pool the block is launched
+  // with: refuse a build whose register count would leave the softmax
+  // warpgroups waiting for registers
+  cudaFuncAttributes fa{};
+  e = cudaFuncGetAttributes(&fa, attention7_kernel<Wn>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < kA7RegsLaunch) return cudaErrorInvalidConfiguration;
   const long long items = a.nwin * a.g.heads;
   long long grid = sms;
   if (grid > items) grid = items;
