@@ -1394,7 +1394,7 @@ constexpr int kA7Soft0 = kA7PrepWarps;                               // first so
 constexpr int kA7Threads = (kA7PrepWarps + 4 * kA7Groups) * 32;  // 512
 // Registers per thread: launched at 128 (the most 512 threads get), then the
 // preparation warpgroup gives some to the three softmax warpgroups.
-constexpr int kA7RegsLaunch = 128, kA7RegsPrep = 64, kA7RegsSoft = 144;
+constexpr int kA7RegsLaunch = 128, kA7RegsPrep = 48, kA7RegsSoft = 152;
 static_assert(128 * kA7RegsPrep + 384 * kA7RegsSoft <= kA7Threads * kA7RegsLaunch, "register budgets");
 constexpr uint32_t kA7TmemCols = 512;
 // TMEM columns: group g has S / P at [144 g, 144 g + 112) and O at
