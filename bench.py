@@ -865,7 +865,7 @@ def run_merge(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(wl), merged_tokens=merged, ln_eps=eps), "api": "vswin_patch_merge_forward",
         "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
-        "merge_roofline": {"kernel": "pm_kernel", "bound": "hbm", "achieved": byts / len(layers) / (k_us / 1e6) / 1e9,
+        "merge_roofline": {"kernel": "pm_ws_kernel", "bound": "hbm", "achieved": byts / len(layers) / (k_us / 1e6) / 1e9,
                            "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                            "frac": byts / len(layers) / (k_us / 1e6) / 1e9 / float(peaks["hbm_gbs"]),
                            "peak_source": f"{peak_src} HBM copy", "avg_launch_us": k_us,

@@ -63,9 +63,38 @@ def test_patch_merge(shape, scale):
         assert np.abs(err).max() <= ABS_MAX and np.abs(err).mean() <= ABS_MEAN
 
 
+def test_patch_merge_column_slices_several_tiles_per_cta():
+    # Swin-T stage 2 -> 3 at batch 8: 2C = 384 in four resident 96-column weight
+    # slices, 200 row tiles of 9 lines x 14 merged tokens (TMA gather) over 37 CTAs
+    # per slice (five or six tiles each, both accumulators and the statistics ring
+    # reused), every element against the oracle
+    out, ref = _run((8, 16, 28, 28, 192), "sensitivity", 11600)
+    err = out - ref
+    assert np.linalg.norm(err) / np.linalg.norm(ref) <= REL_L2
+    assert np.abs(err).max() / np.abs(ref).max() <= REL_MAX
+
+
+def test_patch_merge_odd_sizes_several_tiles_per_cta():
+    # odd H and W (the cp.async gather, zero-filled neighbours on the last row and
+    # column): 784 row tiles on 148 CTAs, every element against the oracle
+    out, ref = _run((8, 16, 55, 55, 96), "sensitivity", 11650)
+    err = out - ref
+    assert np.linalg.norm(err) / np.linalg.norm(ref) <= REL_L2
+    assert np.abs(err).max() / np.abs(ref).max() <= REL_MAX
+
+
+def test_patch_merge_widest_channels_tiled_kernel():
+    # C = 1536: a 16-column slice of the 6144-row folded weights would not leave
+    # room for four A stages, so the tiled kernel runs
+    out, ref = _run((1, 2, 3, 4, 1536), "baseline", 11700)
+    err = out - ref
+    assert np.linalg.norm(err) / np.linalg.norm(ref) <= REL_L2
+    assert np.abs(err).max() / np.abs(ref).max() <= REL_MAX
+
+
 def test_patch_merge_headline_whole_tensor():
-    # the headline stage-1 token tensor (8, 16, 56, 56, 96) -> (8, 16, 28, 28, 192): 784
-    # tiles, every element against the oracle
+    # the headline stage-1 token tensor (8, 16, 56, 56, 96) -> (8, 16, 28, 28, 192): 896
+    # tiles of 4 lines x 28 merged tokens (TMA gather), every element against the oracle
     out, ref = _run((8, 16, 56, 56, 96), "sensitivity", 11500)
     err = out - ref
     assert np.linalg.norm(err) / np.linalg.norm(ref) <= REL_L2
