@@ -866,6 +866,7 @@ def run_merge(args):
         "config": dict(workload_config(wl), merged_tokens=merged, ln_eps=eps), "api": "vswin_patch_merge_forward",
         "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
         "merge_roofline": {"kernel": "pm_ws_kernel", "bound": "hbm", "achieved": byts / len(layers) / (k_us / 1e6) / 1e9,
+                           "traffic": (traffic_record("merge_kernel", wl.name) or {}).get("bytes_per_launch"),
                            "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                            "frac": byts / len(layers) / (k_us / 1e6) / 1e9 / float(peaks["hbm_gbs"]),
                            "peak_source": f"{peak_src} HBM copy", "avg_launch_us": k_us,

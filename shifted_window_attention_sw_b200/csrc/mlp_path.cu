@@ -298,12 +298,25 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       const uint32_t lbo1 = (uint32_t)(HC / 8) * 128u; // W1 chunk: K-group stride
       const uint32_t lbo2 = (uint32_t)(C / 8) * 128u;  // W2 chunk: K-group stride
       const long long total = ntiles * NCH;
-      auto stage_of = [&](long long g) -> int { return a.resident ? (int)(g % NCH) : (int)(g % S); };
-      auto w_phase = [&](long long g) -> uint32_t { return a.resident ? 0u : (uint32_t)(g / S) & 1; };
+      // chunk g = t * NCH + c; its weight stage and the parity of that stage's
+      // use count, all kept incrementally (a 64-bit division by a runtime
+      // count costs hundreds of cycles of this thread's issue time): resident
+      // weights, stage c and phase 0; streamed, a ring of S stages
+      long long t = 0;
+      int c = 0, ws = 0;
+      uint32_t wph = 0;
+      auto advance = [&]() {
+        if (++c == NCH) {
+          c = 0;
+          ++t;
+        }
+        if (!a.resident && ++ws == S) {
+          ws = 0;
+          wph ^= 1u;
+        }
+      };
       if (warp == 1) {
-        for (long long g = 0; g < total && !s_abort; ++g) {
-          const long long t = g / NCH;
-          const int c = (int)(g % NCH);
+        for (long long g = 0; g < total && !s_abort; ++g, advance()) {
           const int xb = (int)(t % kMlpXBufs);
           // the accumulator's previous chunk (g - 2) has been read by its fc2
           if (g >= 2 && !mbar_wait(&fc2_done[g & 1], (uint32_t)((g - 2) >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
@@ -312,8 +325,8 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           if (c == 0 && !s_abort &&
               !mbar_wait(&xn_full[xb], (uint32_t)(t / kMlpXBufs) & 1, a.ctx.err, kErrWaitLoad, lim))
             s_abort = 1;
-          const int s = stage_of(g);
-          if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+          const int s = a.resident ? c : ws;
+          if (!s_abort && !mbar_wait(&w_full[s], a.resident ? 0u : wph, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
           tc_fence_after();
           if (s_abort) break;
           const uint32_t xa = smem_u32(sX(xb));
@@ -327,9 +340,7 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           if (c == NCH - 1) umma_commit(&xn_free[xb]);
         }
       } else {
-        for (long long g = 0; g < total && !s_abort; ++g) {
-          const long long t = g / NCH;
-          const int c = (int)(g % NCH);
+        for (long long g = 0; g < total && !s_abort; ++g, advance()) {
           const int ob = (int)(t & 1);
           // h of chunk g is in TMEM (and its fc1 accumulator was read)
           if (!mbar_wait(&h_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim)) s_abort = 1;
@@ -337,8 +348,8 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
           if (c == 0 && t >= 2 && !s_abort &&
               !mbar_wait(&acc2_free[ob], (uint32_t)((t >> 1) - 1) & 1, a.ctx.err, kErrWaitMma, lim))
             s_abort = 1;
-          const int s = stage_of(g);
-          if (!s_abort && !mbar_wait(&w_full[s], w_phase(g), a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
+          const int s = a.resident ? c : ws;
+          if (!s_abort && !mbar_wait(&w_full[s], a.resident ? 0u : wph, a.ctx.err, kErrWaitLoad, lim)) s_abort = 1;
           tc_fence_after();
           if (s_abort) break;
           const uint32_t wa2 = smem_u32(smem + L.w + s * L.wstage + L.w2off);
@@ -483,8 +494,8 @@ __global__ void __launch_bounds__(kMlpThreads, 1)
       const int hq = (warp - kMlpGelu0) >> 2;
       const int CW = HC / kMlpGeluPerQ;  // this warp's columns of a chunk: 16, 32 or 64
       const long long total = ntiles * NCH;
-      for (long long g = 0; g < total; ++g) {
-        const int c = (int)(g % NCH);
+      int c = 0;  // chunk of the tile (g mod NCH, kept incrementally)
+      for (long long g = 0; g < total; ++g, c = c + 1 == NCH ? 0 : c + 1) {
         if (!s_abort && !mbar_wait(&acc1_full[g & 1], (uint32_t)(g >> 1) & 1, a.ctx.err, kErrWaitMma, lim))
           s_abort = 1;
         tc_fence_after();
