@@ -20,8 +20,10 @@
 // chunks with cp.async (zero-fill for padding), later reads them back from
 // shared memory for the row statistics (Welford per 32-value block, merged with
 // Chan's formula), and in the epilogue holds that row's TMEM lane. Thread 0
-// issues the MMAs. Both take the same steps in the same order (K blocks, MMAs,
-// statistics, epilogue), so they give the same bits.
+// issues the MMAs. pm_kernel and the cp.async form of pm_ws_kernel take the
+// same steps in the same order (32-channel K blocks, MMAs, statistics,
+// epilogue), so they give the same bits; the TMA form takes the K blocks in
+// the order (dh, dw, c), 64 channels at a time, so its sums round differently.
 #include <cuda.h>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -232,13 +234,13 @@ __global__ void __launch_bounds__(kPmThreads) pm_kernel(PmArgs a) {
 // shared memory next to four A stages): one CTA per SM keeps its K x BN weight
 // slice resident and walks row tiles, with the roles in warps of their own:
 //
-//   warps 0-3   gather: the K blocks (32 channels of one neighbour) of a tile's
+//   warps 0-3   gather: the K blocks (32 or 64 channels, below) of a tile's
 //               merged rows into a ring of A stages
-//   warp 4      MMA issue (one thread): two K = 16 steps a K block into one of
-//               two TMEM accumulators
-//   warps 5-8   row statistics (thread = row): each K block's 32 values read
-//               back from the stage (Welford block, Chan's merge -- the same
-//               arithmetic as the tiled kernel)
+//   warp 4      MMA issue (one thread): two or four K = 16 steps a K block
+//               into one of two TMEM accumulators
+//   warps 5-8   row statistics (thread = row): each K block's values read
+//               back from the stage, 32 at a time (Welford block, Chan's
+//               merge -- the tiled kernel's arithmetic)
 //   warps 9-16  epilogue: rstd * acc + (-mean * rstd) * colsum + bias, bf16,
 //               16-byte stores of the merged rows (two warps a lane quarter)
 //
@@ -247,14 +249,16 @@ __global__ void __launch_bounds__(kPmThreads) pm_kernel(PmArgs a) {
 //
 // Two gathers. With even H and W (every Video Swin stage that merges) the 2x2
 // neighbours are a plain view of x: x[bt, 2i + dh, 2j + dw, c] is the element
-// (c, dw, j, dh, bt * H/2 + i) of a 5-D tensor with byte strides (2, 2C, 4C,
-// 2WC, 4WC), so one TMA box (32 channels, dw, Wh columns j, dh, Lt lines)
-// brings a K block of a tile of Lt whole lines of merged tokens (Lt * Wh <=
-// 128 rows) into the stage, 64-byte swizzled (rows of 64 bytes, 16-byte chunk
-// index XORed with bits 1-2 of the row) -- one instruction a K block, issued
-// by one thread. Otherwise the four gather warps move 128-row tiles with
-// cp.async (4 lanes a row, 64 contiguous bytes a row and instruction,
-// zero-fill for padding) into the no-swizzle core-matrix layout.
+// (dw * C + c, j, dh, bt * H/2 + i) of a 4-D tensor with byte strides (2, 4C,
+// 2WC, 4WC) -- the 2C channels of the token pair (2j, 2j + 1) are contiguous.
+// One TMA box (64 channels, Wh columns j, one dh, Lt lines) brings a K block
+// of a tile of Lt whole lines of merged tokens (Lt * Wh <= 128 rows) into the
+// stage, 128-byte swizzled (rows of 128 bytes, 16-byte chunk index XORed with
+// the row's low three bits) -- one instruction a K block, issued by one thread;
+// the K order is then (dh, dw, c) and the weight fold permutes Wr's rows to
+// match. Otherwise the four gather warps move 128-row tiles with cp.async (4
+// lanes a row, 64 contiguous bytes a row and instruction, zero-fill for
+// padding) in the pages' K order into the no-swizzle core-matrix layout.
 // K block: 32 channels (cp.async gather) or 64 (TMA gather); A stage 8 or 16 KB
 __host__ __device__ constexpr int pw_bk(bool tma) { return tma ? 64 : 32; }
 __host__ __device__ constexpr int pw_stage_bytes(bool tma) { return kPmBM * pw_bk(tma) * 2; }
