@@ -7,9 +7,11 @@
 //      once per call); when the tiled GEMM runs, row_stats_kernel writes the
 //      row table and each row's layer-norm statistics instead.
 //   2. gemm_ws_kernel<kQKV>: persistent warp-specialised tcgen05 GEMM (gather
-//      warps cp.async the rows named by the row table, zero-filling padding,
-//      and for the block entry compute each landed row's layer-norm
-//      statistics; one MMA warp; epilogue warps). The epilogue adds bqkv,
+//      warps cp.async the rows named by the row table, zero-filling padding;
+//      two MMA-issuing warps on different sub-partitions, even and odd tiles;
+//      epilogue warps; for the block entry four of them are statistics warps
+//      that compute each landed row's layer-norm mean and rstd from the
+//      stage and write its -mean as one extra K step). The epilogue adds bqkv,
 //      scales q by log2(e)/sqrt(d) and writes per-(window, head) q / k / v
 //      slabs in the tensor-core operand layout. gemm_kernel<kQKV> is the tiled
 //      fallback used when the persistent kernel's resident weight slice does
@@ -22,7 +24,7 @@
 //      other window shapes, one (window, head) per CTA.
 //   4. gemm_ws_kernel<kPROJ> (or gemm_kernel<kPROJ>): the attention output
 //      times Wproj, epilogue adds bproj (and, for the block entry, the
-//      residual, which the gather warps copy into shared memory) and scatters
+//      residual, which the producer warps copy into shared memory) and scatters
 //      rows back through the row table (reverse partition, roll by +shift,
 //      drop padding).
 //
