@@ -1,7 +1,8 @@
 """Host logic of bench.py on CPU: a committed ncu traffic record is used only for
 the workload it was taken on and only while the kernel source it names still
 hashes to the recorded value; the peaks fall back to the stated figures when the
-measured file is absent."""
+measured file is absent; the reference arm (the oracle) prints the contract's
+line and refuses fewer than three warm-up steps."""
 
 import hashlib
 import json
@@ -69,3 +70,37 @@ def test_peaks_read_from_the_measured_file(tmp_path, monkeypatch):
     peaks, src = bench.load_peaks()
     assert src == "measured"
     assert peaks["hbm_gbs"] == pytest.approx(6500.0)
+
+
+def _reference_line(*extra):
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "swin_t_s1_small_f32", *extra], capture_output=True, text=True, timeout=600,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    return r
+
+
+def test_reference_arm_line_contract():
+    # the oracle timed as the reference arm (small workload, a few seconds): one JSON
+    # line with the arm's metric and unit, its own value as cpu_baseline and e2e, and
+    # no host<->device bytes
+    r = _reference_line("--steps", "1", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
+    assert line["higher_is_better"] is True
+    assert (line["steps"], line["warmup"]) == (1, 3)
+    assert line["value"] > 0
+    assert line["config"]["workload"] == "swin_t_s1_small_f32"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == pytest.approx(line["value"])
+    e2e = line["e2e"]
+    assert e2e["value"] == pytest.approx(line["value"]) and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_refuses_fewer_than_three_warmup_steps():
+    r = _reference_line("--steps", "1", "--warmup", "1")
+    assert r.returncode != 0
