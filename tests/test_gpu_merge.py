@@ -84,8 +84,8 @@ def test_patch_merge_odd_sizes_several_tiles_per_cta():
 
 
 def test_patch_merge_widest_channels_tiled_kernel():
-    # C = 1536: a 16-column slice of the 6144-row folded weights would not leave
-    # room for four A stages, so the tiled kernel runs
+    # C = 1536: even 16-column slices would be 192 of them, more than the SMs (and one
+    # of 6144 rows would not leave room for four A stages), so the tiled kernel runs
     out, ref = _run((1, 2, 3, 4, 1536), "baseline", 11700)
     err = out - ref
     assert np.linalg.norm(err) / np.linalg.norm(ref) <= REL_L2
